@@ -1,0 +1,163 @@
+"""Pins for the oracle's expert-cache simulator.
+
+* hand-worked event sequences (tests/golden/cache_traces.txt);
+* a second simulator written here with a different data structure (a lazy
+  min-heap keyed by (count, last use, id) instead of a linear scan) must give
+  the identical event sequence on long random traces;
+* Belady's farthest-in-future policy on the flattened trace is optimal for
+  demand paging, so no policy can miss less: it bounds the oracle from below;
+* a cache at least as large as the number of distinct ids only takes
+  compulsory misses.
+"""
+import heapq
+from pathlib import Path
+
+import numpy as np
+import pytest
+
+import workloads as W
+
+GOLDEN = Path(__file__).parent / "golden"
+
+
+def _golden_traces():
+    traces, cur = [], None
+    for line in (GOLDEN / "cache_traces.txt").read_text().splitlines():
+        line = line.strip()
+        if not line or line.startswith("#"):
+            continue
+        f = line.split()
+        if f[0] == "trace":
+            cur = dict(name=f[1], experts=int(f[2]), cap=int(f[3]), decay=int(f[4]), n=int(f[5]),
+                       ids=[], ev=[])
+        elif f[0] == "ids":
+            cur["ids"].append([int(v) for v in f[2:]])
+        elif f[0] == "ev":
+            cur["ev"].append(tuple(int(v) for v in f[1:]))
+        elif f[0] == "end":
+            traces.append(cur)
+    return traces
+
+
+@pytest.mark.parametrize("tr", _golden_traces(), ids=lambda t: t["name"])
+def test_cache_hand_worked(oracle_lib, tr):
+    ids = np.array(tr["ids"], np.int32)
+    r = oracle_lib.cache_sim(ids, tr["experts"], tr["cap"], tr["decay"])
+    got = []
+    for s in range(ids.shape[0]):
+        for j in range(ids.shape[1]):
+            got.append((s, j, int(ids[s, j]), int(r["hit"][s, j]), int(r["slot"][s, j]), int(r["victim"][s, j])))
+    assert got == tr["ev"]
+
+
+def heap_sim(ids, n_experts, capacity, decay):
+    """Independent re-implementation with a lazily invalidated heap."""
+    steps, n = ids.shape
+    slot_of, expert_in = {}, [None] * capacity
+    free = list(range(capacity))
+    heapq.heapify(free)
+    cnt = [0] * n_experts
+    last = [-1] * n_experts
+    heap = []                       # (cnt, last, id, version)
+    ver = [0] * n_experts
+    out = []
+
+    def push(e):
+        ver[e] += 1
+        heapq.heappush(heap, (cnt[e], last[e], e, ver[e]))
+
+    for s in range(steps):
+        if decay > 0 and s > 0 and s % decay == 0:
+            cnt = [c // 2 for c in cnt]
+            heap = []
+            for e in slot_of:
+                push(e)
+        step = set(int(v) for v in ids[s])
+        for j in range(n):
+            e = int(ids[s, j])
+            cnt[e] += 1
+            last[e] = s
+            if e in slot_of:
+                out.append((1, slot_of[e], -1))
+                push(e)
+                continue
+            if free:
+                sl = heapq.heappop(free)
+                victim = -1
+            else:
+                skipped = []
+                while True:
+                    c, l, v, vv = heapq.heappop(heap)
+                    if v not in slot_of or vv != ver[v]:
+                        continue
+                    if v in step:
+                        skipped.append((c, l, v, vv))
+                        continue
+                    break
+                for it in skipped:
+                    heapq.heappush(heap, it)
+                victim = v
+                sl = slot_of.pop(v)
+            slot_of[e] = sl
+            expert_in[sl] = e
+            push(e)
+            out.append((0, sl, victim))
+    return out
+
+
+@pytest.mark.parametrize("seed,E,cap,decay,n,steps", [
+    (1, 64, 8, 16, 4, 400), (2, 300, 40, 64, 10, 600), (3, 24576, 2048, 256, 10, 300),
+    (4, 50, 10, 0, 10, 200), (5, 500, 64, 7, 10, 500)])
+def test_cache_matches_independent_simulator(oracle_lib, seed, E, cap, decay, n, steps):
+    gen = W.paging_trace(seed, E, n, steps, drift_every=50, hot=min(cap, E // 2))
+    ids = np.stack([np.argsort(-l, kind="stable")[:n] for l in gen]).astype(np.int32)
+    r = oracle_lib.cache_sim(ids, E, cap, decay)
+    ref = heap_sim(ids, E, cap, decay)
+    got = [(int(r["hit"][s, j]), int(r["slot"][s, j]), int(r["victim"][s, j]))
+           for s in range(steps) for j in range(n)]
+    assert got == ref
+    assert r["misses"] == sum(1 for h, _, _ in ref if h == 0)
+
+
+def belady_misses(seq, capacity):
+    nxt = {}
+    future = [0] * len(seq)
+    for i in range(len(seq) - 1, -1, -1):
+        future[i] = nxt.get(seq[i], 1 << 60)
+        nxt[seq[i]] = i
+    cache, misses = {}, 0
+    for i, e in enumerate(seq):
+        if e in cache:
+            cache[e] = future[i]
+            continue
+        misses += 1
+        if len(cache) >= capacity:
+            v = max(cache, key=lambda c: cache[c])
+            del cache[v]
+        cache[e] = future[i]
+    return misses
+
+
+@pytest.mark.parametrize("seed,cap", [(11, 6), (12, 12), (13, 30)])
+def test_cache_not_below_belady(oracle_lib, seed, cap):
+    gen = W.paging_trace(seed, 80, 4, 300, drift_every=40, hot=20)
+    ids = np.stack([np.argsort(-l, kind="stable")[:4] for l in gen]).astype(np.int32)
+    r = oracle_lib.cache_sim(ids, 80, cap, 32)
+    assert r["misses"] >= belady_misses(ids.ravel().tolist(), cap)
+
+
+def test_cache_large_enough_only_compulsory(oracle_lib):
+    rng = np.random.default_rng(4)
+    ids = np.stack([rng.choice(40, 5, replace=False) for _ in range(200)]).astype(np.int32)
+    r = oracle_lib.cache_sim(ids, 40, 40, 8)
+    assert r["misses"] == len(np.unique(ids))
+    assert np.all(r["victim"] == -1)
+
+
+def test_cache_rejects_bad_trace(oracle_lib):
+    with pytest.raises(ValueError):
+        oracle_lib.cache_sim(np.array([[1, 1]], np.int32), 4, 2, 0)   # repeated id
+    with pytest.raises(ValueError):
+        oracle_lib.cache_sim(np.array([[1, 2, 3]], np.int32), 4, 2, 0)  # n > capacity
+    with pytest.raises(ValueError):
+        oracle_lib.cache_sim(np.array([[7]], np.int32), 4, 2, 0)      # id out of range

@@ -1,0 +1,467 @@
+#!/usr/bin/env python
+"""Benchmark of the quantized MoE expert step on B200 (one JSON line on rank 0).
+
+Workloads (seeded synthetic inputs, shapes from the pages; see workloads/):
+  decode  (default) hidden 2048, 512 experts + 1 shared, top-10, 4-bit blocks,
+          1 token per step; steps rotate over --layers copies of the layer so
+          the weights streamed per step come from HBM, not L2
+  verify  same layer with 2-bit blocks, Zipf-skewed router bias, a window of
+          --window tokens per step
+  prefill same layer as decode, --chunk tokens per step (tensor-core path)
+  paging  24,576 two-bit experts in page-locked host memory, 2048 HBM slots,
+          Gumbel-top-10 routing over drifting Zipf popularity, 1 token per step
+
+A step is one pass of the whole step (route -> permute -> expert FFN ->
+combine; paging adds the cache) over one batch.  The timed region is a CUDA
+graph replay of exactly --steps steps (paging: an eager loop, since every
+step synchronises with the host), bracketed by a barrier and
+torch.cuda.synchronize(); multi-GPU runs are replicas (weak scaling) timed as
+the max over ranks.
+
+--impl reference times the fp64 CPU oracle on the host cores instead (each
+step a bounded sample of the same workload).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+from pathlib import Path
+
+import numpy as np
+
+ROOT = Path(__file__).resolve().parent
+sys.path.insert(0, str(ROOT))
+
+METRIC = "MoE-layer tokens/s and expert weight GB/s vs HBM peak (decode, prefill, paging)"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ----------------------------------------------------------------- helpers
+def peaks():
+    p = ROOT / "MEASURED_PEAKS.json"
+    if p.exists():
+        d = json.loads(p.read_text())
+        d["source"] = "measured"
+        return d
+    d = dict(FALLBACK_PEAKS)
+    d["source"] = "fallback"
+    return d
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,utilization.gpu,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", f"--id={device_index}", f"--query-gpu={self.FIELDS}",
+                                       "--format=csv,noheader,nounits", "-lms", "200"],
+                                      stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.p = None
+
+    def stop(self):
+        if self.p is None:
+            return None
+        time.sleep(0.25)
+        self.p.terminate()
+        try:
+            self.p.wait(timeout=5)
+        except Exception:
+            self.p.kill()
+        self.f.flush()
+        rows = []
+        for line in Path(self.f.name).read_text().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 10:
+                continue
+            try:
+                rows.append(dict(sm=float(parts[1]), smax=float(parts[2]), util=float(parts[4]),
+                                 hw=parts[6], hwt=parts[7], swt=parts[8], swp=parts[9]))
+            except ValueError:
+                continue
+        os.unlink(self.f.name)
+        if not rows:
+            return None
+        load = [r for r in rows if r["util"] >= 50] or rows
+        reasons = set()
+        for r in load:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                              ("swt", "sw_thermal_slowdown"), ("swp", "sw_power_cap")):
+                if r[key].lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in load), "sm_max_mhz": max(r["smax"] for r in rows),
+                "reasons": sorted(reasons), "samples": len(rows), "samples_under_load": len(load)}
+
+
+def src_hash(*names):
+    h = hashlib.sha256()
+    for n in names:
+        h.update((ROOT / "quantized_expert_ffn_route_b200" / "csrc" / n).read_bytes())
+    return h.hexdigest()[:16]
+
+
+def traffic_from_profiles(key: str, sha: str):
+    """DRAM bytes per launch from a committed ncu summary, if taken on this kernel source."""
+    p = ROOT / "profiles" / "traffic.txt"
+    if not p.exists():
+        return None
+    for line in p.read_text().splitlines():
+        f = line.split()
+        if len(f) >= 3 and f[0] == key and f[1] == sha:
+            return float(f[2])
+    return None
+
+
+def dist_setup(n_gpus):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    import torch
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+# --------------------------------------------------------------- workloads
+def build_layer(kind):
+    import workloads as W
+    if kind == "verify":
+        return W.verify_layer()
+    c = W.DECODE
+    return W.make_layer(W.SEED["decode"], 4, c["H"], c["I"], c["E"], c["k"], shared=True, w_dtype="bf16")
+
+
+def gpu_copies(layer, n):
+    import quantized_expert_ffn_route_b200 as M
+    base = M.MoELayer(layer.bits, layer.H, layer.I, layer.E, layer.k, layer.blobs, layer.shared, layer.w_router,
+                      layer.w_dtype, layer.bias)
+    return [base] + [base.clone() for _ in range(n - 1)]
+
+
+def cpu_baseline(layer, tokens, seconds, T_batch=8):
+    """The oracle, as it stands, on a bounded sample: token batches until `seconds` pass."""
+    import oracle
+    n, t0 = 0, time.perf_counter()
+    while True:
+        i = (n // T_batch) % max(1, tokens.shape[0] // T_batch)
+        x = tokens[i * T_batch:(i + 1) * T_batch]
+        oracle.moe_layer(layer.bits, x, "bf16", layer.blobs, k=layer.k, H=layer.H, I=layer.I, E=layer.E,
+                         w_router=layer.w_router, w_dtype="bf16", bias=layer.bias, shared_blob=layer.shared)
+        n += x.shape[0]
+        dt = time.perf_counter() - t0
+        if dt >= seconds and n >= T_batch:
+            return n, dt
+
+
+def run_graph_steps(step_fn, first, count, time_ffn=True):
+    """Captures `count` steps in one CUDA graph; returns (graph, ffn event pairs)."""
+    import torch
+    g = torch.cuda.CUDAGraph()
+    pairs = []
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            for i in range(first, first + count):
+                if time_ffn:
+                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    step_fn(i, e0, e1)
+                    pairs.append((e0, e1))
+                else:
+                    step_fn(i, None, None)
+    torch.cuda.current_stream().wait_stream(s)
+    return g, pairs
+
+
+def bench_layer(args, world, rank, pk):
+    """decode / verify / prefill: resident layer, graph-replayed steps."""
+    import torch
+    import quantized_expert_ffn_route_b200 as M
+    import workloads as W
+
+    kind = args.workload
+    layer = build_layer(kind)
+    H, I, E, k, bits = layer.H, layer.I, layer.E, layer.k, layer.bits
+    T = {"decode": 1, "verify": args.window, "prefill": args.chunk}[kind]
+    mode = M.MOE_MODE_GEMM if kind == "prefill" else M.MOE_MODE_AUTO
+    blob = M.moe_expert_blob_bytes(bits, H, I)
+    # layer copies at distinct addresses: the steps of one sweep touch far more
+    # than the 126 MB L2 (decode: 16 x 908 MB), so weights come from HBM
+    n_layers = args.layers or (2 if kind == "prefill" else 16)
+    copies = gpu_copies(layer, n_layers)
+    n_steps = args.warmup + args.steps
+    seed = W.SEED[kind] + 7919 * rank
+    x_host = W.make_tokens(seed, n_steps * T if kind != "prefill" else 2 * T, H, "bf16")
+    xs = torch.from_numpy(x_host.view(np.int16)).view(torch.bfloat16).cuda()
+    bufs = copies[0].buffers(T, mode)
+
+    def x_of(i):
+        if kind == "prefill":
+            j = i % 2
+            return xs[j * T:(j + 1) * T]
+        return xs[i * T:(i + 1) * T]
+
+    def step(i, e0=None, e1=None):
+        L = copies[i % n_layers]
+        b = bufs
+        x = x_of(i)
+        M.moe_route_topk(x, M.MOE_BF16, L.w_router, L.w_dtype, None, L.bias, T, H, E, k, b.ids, b.w, b.logits,
+                         b.ws_route, b.sizes["route"])
+        M.moe_permute(b.ids, T, k, E, b.offsets, b.perm_src, b.perm_dst, b.active, b.ws_perm, b.sizes["perm"])
+        ffn = M.moe_expert_ffn_q4 if bits == 4 else M.moe_expert_ffn_q2
+        if e0 is not None:
+            e0.record()
+        ffn(L.table, b.offsets, b.active, b.perm_src, x, M.MOE_BF16, T, k, H, I, E, L.shared, b.y_perm, b.y_shared,
+            mode, b.ws_ffn, b.sizes["ffn"])
+        if e1 is not None:
+            e1.record()
+        M.moe_combine(b.y_perm, b.perm_dst, b.w, b.y_shared, T, k, H, b.y)
+
+    for i in range(args.warmup):                      # eager warm-up
+        step(i)
+    torch.cuda.synchronize()
+    assert M.moe_device_error() == 0
+    n0 = M.moe_kernel_launches()
+    graph, pairs = run_graph_steps(step, args.warmup, args.steps)
+    launches = M.moe_kernel_launches() - n0
+    graph.replay()                                     # first replay uploads the graph
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(torch.cuda.current_device())
+    # keep the GPU busy long enough for the clock sampler to see it under load
+    t_end = time.perf_counter() + 1.0
+    while time.perf_counter() < t_end:
+        graph.replay()
+        torch.cuda.synchronize()
+    barrier(world)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record()
+    graph.replay()
+    ev1.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    ms = ev0.elapsed_time(ev1)
+    ms_max = max_over_ranks(ms, world)
+    ffn_ms = [a.elapsed_time(b) for a, b in pairs]
+    ffn_avg_ms = float(np.mean(ffn_ms))
+    assert M.moe_device_error() == 0
+
+    # distinct experts actually touched in the last timed step (all routed + shared)
+    n_act = int(bufs.active[0].item())
+    tokens_total = sum_over_ranks(args.steps * T, world)
+    value = tokens_total / (ms_max / 1e3)
+
+    # algorithmic bytes/FLOPs of one expert-FFN launch
+    if kind == "prefill":
+        flops = 2 * 3 * H * I * T * (k + 1)
+        bytes_ffn = (n_act + 1) * blob + T * H * 2 + T * (k + 1) * H * 4
+        tf = flops / (ffn_avg_ms / 1e3) / 1e12
+        peak_tf = pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+        gbs = bytes_ffn / (ffn_avg_ms / 1e3) / 1e9
+        if flops / bytes_ffn > peak_tf * 1e12 / (pk["hbm_gbs"] * 1e9):
+            roof = {"bound": "tensor", "achieved": round(tf, 2), "peak": peak_tf, "unit": "TFLOP/s",
+                    "frac": round(tf / peak_tf, 4)}
+        else:
+            roof = {"bound": "hbm", "achieved": round(gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+                    "frac": round(gbs / pk["hbm_gbs"], 4)}
+    else:
+        # per-window distinct experts differ; average over the timed steps is not tracked on device,
+        # so credit the experts of the last window (decode: always k routed + 1 shared)
+        bytes_ffn = (n_act + 1) * blob + T * H * 2 + T * (k + 1) * H * 4
+        gbs = bytes_ffn / (ffn_avg_ms / 1e3) / 1e9
+        roof = {"bound": "hbm", "achieved": round(gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": round(gbs / pk["hbm_gbs"], 4)}
+    sha = src_hash("gemv.cu") if kind != "prefill" else src_hash("gemm_tc.cu")
+    roof["traffic"] = traffic_from_profiles(f"expert_ffn_{kind}", sha)
+    roof["kernel"] = "moe_expert_ffn (gate/up + down kernels)"
+    roof["ms_per_launch"] = round(ffn_avg_ms, 5)
+    roof["algorithmic_bytes_per_launch"] = int(bytes_ffn)
+    roof["peak_source"] = pk["source"]
+
+    # end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        n_e2e = min(args.steps, args.e2e_steps)
+        xh = torch.from_numpy(x_host[: max(T, n_e2e * T if kind != "prefill" else T)].view(np.int16)).view(
+            torch.bfloat16).pin_memory()
+        yh = torch.empty(T * H, dtype=torch.float32).pin_memory()
+        xd = torch.empty(T, H, dtype=torch.bfloat16, device="cuda")
+        s = torch.cuda.current_stream()
+        for i in range(3):
+            xd.copy_(xh[:T], non_blocking=True)
+            copies[i % n_layers].forward(xd, M.MOE_BF16, T=T, mode=mode, bufs=bufs)
+            yh.copy_(bufs.y[:T * H], non_blocking=True)
+            s.synchronize()
+        barrier(world)
+        a, b2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for i in range(n_e2e):
+            j = i * T if kind != "prefill" else 0
+            xd.copy_(xh[j:j + T], non_blocking=True)
+            copies[i % n_layers].forward(xd, M.MOE_BF16, T=T, mode=mode, bufs=bufs)
+            yh.copy_(bufs.y[:T * H], non_blocking=True)
+            s.synchronize()
+        b2.record()
+        torch.cuda.synchronize()
+        e_ms = max_over_ranks(a.elapsed_time(b2), world)
+        e2e = {"value": round(sum_over_ranks(n_e2e * T, world) / (e_ms / 1e3), 1), "unit": "tokens/s",
+               "h2d_bytes_per_step": T * H * 2, "d2h_bytes_per_step": T * H * 4, "steps": n_e2e,
+               "note": "MoELayer.forward via the C ABI; pinned host x in, fp32 y out, stream sync every step"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        oracle.set_threads(host_cores())
+        ntok, dt = cpu_baseline(layer, x_host, args.cpu_seconds, T_batch=8)
+        cpu = {"value": round(ntok / dt, 3), "unit": "tokens/s", "cores": host_cores(), "kind": "oracle",
+               "sample": f"{ntok} tokens of the {kind} workload through the fp64 oracle in batches of 8, {dt:.1f} s"}
+
+    cfg = {"workload": f"{kind}: hidden {H}, {E} experts + 1 shared, top-{k}, intermediate {I}, "
+                       f"{bits}-bit blocks of 32 + fp16 scale, {T} token(s)/step",
+           "tokens_per_step": T, "layer_copies": n_layers,
+           "l2": f"inputs larger than L2: {n_layers} layer copies x {E + 1} experts x {blob} B rotate per step",
+           "mode": {0: "auto", 1: "gemv", 2: "gemm"}[mode], "parallelism": f"replicas x{world}"}
+    return dict(value=value, ms=ms_max, steps=args.steps, roofline=roof, e2e=e2e, cpu=cpu, clocks=clk,
+                launches=launches, config=cfg, dtype="fp32 (CUDA-core FMA on 4-bit codes)" if kind == "decode"
+                else ("fp32 (CUDA-core FMA on 2-bit codes)" if kind == "verify" else "fp16 tensor cores, fp32 accum"))
+
+
+def bench_reference(args, world, rank):
+    """The oracle on the host cores, each step a bounded sample (one token / window)."""
+    import oracle
+    import workloads as W
+    if rank != 0:
+        return None
+    oracle.set_threads(host_cores())
+    kind = args.workload if args.workload != "paging" else "decode"
+    layer = build_layer(kind)
+    T = {"decode": 1, "verify": args.window, "prefill": 8}[kind]
+    x = W.make_tokens(W.SEED[kind], (args.warmup + args.steps) * T, layer.H, "bf16")
+
+    def one(i):
+        oracle.moe_layer(layer.bits, x[i * T:(i + 1) * T], "bf16", layer.blobs, k=layer.k, H=layer.H, I=layer.I,
+                         E=layer.E, w_router=layer.w_router, w_dtype="bf16", bias=layer.bias,
+                         shared_blob=layer.shared)
+    for i in range(args.warmup):
+        one(i)
+    t0 = time.perf_counter()
+    for i in range(args.warmup, args.warmup + args.steps):
+        one(i)
+    dt = time.perf_counter() - t0
+    v = args.steps * T / dt
+    return dict(value=v, ms=dt * 1e3, T=T, kind=kind)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default="decode", choices=["decode", "verify", "prefill", "paging"])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--window", type=int, default=16)
+    ap.add_argument("--chunk", type=int, default=8192)
+    ap.add_argument("--layers", type=int, default=0)
+    ap.add_argument("--e2e-steps", type=int, default=500)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    pk = peaks()
+
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        r = bench_reference(args, world, rank)
+        if r is None:
+            return
+        line = {"metric": METRIC, "value": round(r["value"], 4), "unit": "tokens/s", "n_gpus": args.gpus,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(r["ms"] / args.steps, 3),
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic (seeded)", "impl": "reference",
+                "config": {"workload": f"{r['kind']} (oracle: {r['T']} token(s) per step)"},
+                "cpu_baseline": {"value": round(r["value"], 4), "unit": "tokens/s", "cores": host_cores(),
+                                 "kind": "oracle", "sample": f"{args.steps} steps of {r['T']} token(s)"},
+                "e2e": {"value": round(r["value"], 4), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+
+    import torch
+    world, rank, local = dist_setup(args.gpus)
+    if args.workload == "paging":
+        r = bench_paging(args, world, rank, pk)
+    else:
+        r = bench_layer(args, world, rank, pk)
+    if rank == 0:
+        line = {"metric": METRIC, "value": round(r["value"], 2), "unit": "tokens/s", "n_gpus": world,
+                "steps": r["steps"], "warmup": args.warmup, "ms_per_step": round(r["ms"] / r["steps"], 5),
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": r["dtype"],
+                "data": "synthetic (seeded generators; no weights or datasets)", "config": r["config"],
+                "roofline": r["roofline"], "cpu_baseline": r["cpu"], "e2e": r["e2e"],
+                "gpu_launches": int(r["launches"]), "clocks": r["clocks"]}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,254 @@
+/*
+ * moe.h -- C ABI of libmoe: the per-layer quantized Mixture-of-Experts step
+ * (route -> permute -> block-quantized SwiGLU experts -> combine) and the
+ * frequency-driven expert cache, for NVIDIA B200 (sm_100a).
+ *
+ * Sources (web pages on running large MoE models on small GPUs):
+ *  - Strata article (tech.hub77a.com), 30-second summary and section 2
+ *    items 1-3: 10 of 24,576 experts active per token; hot experts resident
+ *    in VRAM, all experts in RAM; a routed expert that is resident is
+ *    computed at once, the others must first be moved in; verify passes of
+ *    drafted tokens; prompt chunks of up to 8,192 tokens.
+ *  - Strata code review (qaqmin.com), sections 1, 3, 4: CUDA MoE and
+ *    dequantisation kernels, an expert cache, a page-locked stage buffer,
+ *    512 experts per layer.
+ *  - 27B dense report (trawling.dev), model-file paragraph: a Q4_0 value
+ *    costs 0.5625 B (32 four-bit codes + one fp16 scale); Strata article,
+ *    summary table: the Q2_0 size.
+ *  - Janas-LLM page (onedev.kr): a RAM expert cache keeps experts that are
+ *    used again.
+ *
+ * Conventions shared by every call
+ *  - Pointers named "device" are CUDA device pointers; "host" are CPU
+ *    pointers.  The caller owns all memory; the library allocates only
+ *    host-side handle state (expert cache) and never calls cudaMalloc.
+ *  - Compute calls are asynchronous on the caller's cudaStream_t (0 = the
+ *    legacy default stream).  They validate arguments on the host before
+ *    launching anything and return a status; nothing throws or aborts.
+ *  - Device buffers must be 16-byte aligned unless stated otherwise.
+ *  - Status: MOE_OK (0) on success; on failure one of the positive codes
+ *    below and a message readable with moe_last_error() (thread-local, valid
+ *    until the next call on the same thread).
+ *  - Kernels never trap.  Problems found on the device (an expert id out of
+ *    range, a missing expert blob, a non-finite selected logit) set a
+ *    per-device error word that moe_device_error() reads.
+ *
+ * Expert blob (one contiguous buffer per expert, "b" = 4 or 2 bits):
+ *    codes Wg [I][H/32][4b B], codes Wu [I][H/32][4b B], codes Wd [H][I/32][4b B],
+ *    scales Wg [I][H/32], Wu [I][H/32], Wd [H][I/32] as IEEE fp16.
+ *  A weight is d * (q - 2^(b-1)).  4-bit block: element i in byte i%16, low
+ *  nibble for i < 16, high nibble otherwise.  2-bit block: element i in byte
+ *  i%8 at bit 2*(i/8).  Wg, Wu map hidden H -> intermediate I, Wd maps back.
+ *  Blob pointers must be 16-byte aligned.  Shapes: H and I multiples of 128.
+ */
+#ifndef MOE_H_
+#define MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *moe_stream_t;   /* same type as cudaStream_t */
+
+/* status codes */
+#define MOE_OK 0
+#define MOE_EINVAL 1      /* bad argument (shape, pointer, alignment, workspace size) */
+#define MOE_ENOMEM 2      /* host allocation failed */
+#define MOE_ECUDA 3       /* a CUDA runtime call failed */
+#define MOE_EBUSY 4       /* expert cache: not enough evictable slots */
+#define MOE_ETIMEDOUT 5   /* expert cache: wait ran out of time */
+#define MOE_EIO 6         /* expert cache: a staging copy failed */
+#define MOE_EDEVICE 7     /* the device error word was set */
+
+/* activation / router dtypes */
+#define MOE_F32 0
+#define MOE_BF16 1
+
+/* expert FFN modes */
+#define MOE_MODE_AUTO 0   /* GEMV when T <= 16, else GEMM */
+#define MOE_MODE_GEMV 1   /* CUDA-core kernels, fp32 math, any T (slow for large T) */
+#define MOE_MODE_GEMM 2   /* tcgen05 tensor-core grouped GEMM, fp16 operands */
+
+/* device error word bits (moe_device_error) */
+#define MOE_DEVERR_BAD_EXPERT 1u     /* expert id outside [0, E) */
+#define MOE_DEVERR_NULL_BLOB 2u      /* an active expert had no blob pointer */
+#define MOE_DEVERR_NONFINITE 4u      /* a selected logit was NaN or +inf */
+#define MOE_DEVERR_BAD_ROW 8u        /* offsets/perm_src inconsistent */
+
+/* Thread-local message of the last failing call ("" if none). */
+const char *moe_last_error(void);
+
+/* Library version (major * 10000 + minor * 100 + patch). */
+int moe_version(void);
+
+/* Number of kernel launches this library has issued in this process (host-side
+ * count; launches recorded into a CUDA graph are counted once, at capture). */
+uint64_t moe_kernel_launches(void);
+
+/* Reads the calling device's error word after synchronizing `s`; clears it if
+ * `clear` != 0.  *bits_out receives MOE_DEVERR_* bits.  Returns MOE_OK, or
+ * MOE_EDEVICE if any bit was set, or MOE_ECUDA. */
+int moe_device_error(uint32_t *bits_out, int clear, moe_stream_t s);
+
+/* Bytes of one expert blob (see layout above). */
+size_t moe_expert_blob_bytes(int bits, int H, int I);
+
+/* ------------------------------------------------------------------ route
+ * Router logits and top-k gate (Strata article, summary table and section 2
+ * item 2: 10 of 24,576 experts per token; the router's choice decides the
+ * compute path).
+ *   l[t,e]  = sum_h x[t,h] * w_router[e,h] (+ bias[e]), fp32 accumulation;
+ *             or, when w_router == NULL, l = logits_in [T,E] fp32 (device).
+ *   ids[t,:] = the k experts first in the order (l descending, id ascending);
+ *             NaN ranks below -inf.
+ *   w[t,j]  = exp(l_j - l_0) / sum_i exp(l_i - l_0) over the k selected.
+ *  x        device [T,H], dtype x_dtype (MOE_F32 | MOE_BF16), row-major.
+ *  w_router device [E,H], dtype w_dtype, row-major; NULL -> use logits_in.
+ *  bias     device [E] fp32 or NULL (added to logits from x, not to logits_in).
+ *  topk_ids device [T,k] int32 out.  topk_w device [T,k] fp32 out.
+ *  logits_out device [T,E] fp32 out, or NULL.
+ *  ws       device workspace of at least moe_route_ws_size(T,E,k) bytes.
+ * Limits: 1 <= k <= min(E, 32), 1 <= E <= 32768, T >= 0.  T = 0 is a no-op.
+ * A selected NaN/+inf logit sets MOE_DEVERR_NONFINITE and yields NaN gates. */
+size_t moe_route_ws_size(int T, int E, int k);
+int moe_route_topk(const void *x, int x_dtype, const void *w_router, int w_dtype,
+                   const float *logits_in, const float *bias, int T, int H, int E, int k,
+                   int32_t *topk_ids, float *topk_w, float *logits_out,
+                   void *ws, size_t ws_bytes, moe_stream_t s);
+
+/* ---------------------------------------------------------------- permute
+ * Token-to-expert permute: a stable counting sort of the T*k (token, slot)
+ * pairs by expert id, so each expert's rows are contiguous and in ascending
+ * token order.
+ *  expert_offsets device [E+1] out: exclusive prefix sum of per-expert counts.
+ *  perm_src device [T*k] out: row -> token index.
+ *  perm_dst device [T*k] out: (t*k + j) -> row.
+ *  active   device [1 + min(E, T*k)] out or NULL: number of experts with rows,
+ *           then those expert ids ascending.
+ * An id outside [0, E) sets MOE_DEVERR_BAD_EXPERT; the outputs are then
+ * unspecified.  ws: at least moe_permute_ws_size(T,k,E) bytes. */
+size_t moe_permute_ws_size(int T, int k, int E);
+int moe_permute(const int32_t *topk_ids, int T, int k, int E, int32_t *expert_offsets,
+                int32_t *perm_src, int32_t *perm_dst, int32_t *active,
+                void *ws, size_t ws_bytes, moe_stream_t s);
+
+/* ------------------------------------------------------------- expert FFN
+ * Block-quantized SwiGLU experts over the permuted rows:
+ *   y_perm[r] = Wd_e (silu(Wg_e x_t) * (Wu_e x_t)),  t = perm_src[r],
+ *   for every row r of every expert e listed in `active` (offsets give the
+ *   rows), and, if shared_blob != NULL, y_shared[t] = the same FFN of the
+ *   shared expert for every token t (Strata code review, section 1: CUDA MoE
+ *   and dequantisation kernels; the shared expert is a reading).
+ * Weights are dequantised on the fly from the blobs (never materialised in
+ * HBM).  GEMV mode: fp32 arithmetic throughout.  GEMM mode: weights and
+ * activations as fp16 tensor-core operands with fp32 accumulation; the
+ * intermediate h is rounded to fp16.
+ *  expert_blobs device array [E] of device blob pointers (expert id -> blob);
+ *           entries of experts that are not active are not read.
+ *  expert_offsets, active, perm_src: as produced by moe_permute.  Rows of
+ *           experts absent from `active` are left untouched in y_perm.
+ *  x        device [T,H] dtype x_dtype.
+ *  y_perm   device [T*k, H] fp32 out.  y_shared device [T,H] fp32 out (or
+ *           NULL when shared_blob is NULL).
+ *  mode     MOE_MODE_AUTO | _GEMV | _GEMM.
+ *  ws       at least moe_expert_ffn_ws_size(bits,T,k,H,I,E,mode) bytes.
+ * _q4 reads 4-bit blobs, _q2 2-bit blobs. */
+size_t moe_expert_ffn_ws_size(int bits, int T, int k, int H, int I, int E, int mode);
+int moe_expert_ffn_q4(const void *const *expert_blobs, const int32_t *expert_offsets,
+                      const int32_t *active, const int32_t *perm_src, const void *x,
+                      int x_dtype, int T, int k, int H, int I, int E,
+                      const void *shared_blob, float *y_perm, float *y_shared, int mode,
+                      void *ws, size_t ws_bytes, moe_stream_t s);
+int moe_expert_ffn_q2(const void *const *expert_blobs, const int32_t *expert_offsets,
+                      const int32_t *active, const int32_t *perm_src, const void *x,
+                      int x_dtype, int T, int k, int H, int I, int E,
+                      const void *shared_blob, float *y_perm, float *y_shared, int mode,
+                      void *ws, size_t ws_bytes, moe_stream_t s);
+
+/* ---------------------------------------------------------------- combine
+ *   y[t] = sum_{j=0}^{k-1} topk_w[t,j] * y_perm[perm_dst[t,j]] (+ y_shared[t]),
+ *   summed in slot order, fp32.  y_shared may be NULL.  y device [T,H] out. */
+int moe_combine(const float *y_perm, const int32_t *perm_dst, const float *topk_w,
+                const float *y_shared, int T, int k, int H, float *y, moe_stream_t s);
+
+/* ----------------------------------------------------------- expert cache
+ * Frequency-driven residency of expert blobs in an HBM slab, paged in from a
+ * page-locked host pool (Strata article, section 2 item 2 and section 3:
+ * hot experts resident in VRAM, everything in RAM, part of the RAM pinned
+ * for the GPU; Strata code review, section 3: the stage buffer; Janas-LLM:
+ * repeated experts stay cached).
+ * Policy, per step (one call of expcache_stage with the step's distinct ids):
+ *  - at the start of step s > 0 with s % decay_period == 0, all counters halve;
+ *  - each id: counter += 1, last use = s; resident -> hit; otherwise miss:
+ *    the lowest free slot, else evict the resident expert not among this
+ *    step's ids with the smallest (counter, last use, id); misses always enter.
+ * Copies run on the cache's own stream (cudaMemcpyAsync from the pinned pool,
+ * one per miss) after the work already queued on the compute stream, then a
+ * tiny kernel patches the device table; expcache_join makes a stream wait for
+ * all of it.  Expert blobs of hits may be used at once.
+ */
+typedef struct moe_expcache moe_expcache;
+
+typedef struct {
+    int32_t n_experts;      /* experts in the host pool */
+    int32_t capacity;       /* HBM slots */
+    int64_t blob_bytes;     /* bytes per expert (multiple of 16) */
+    int64_t slot_stride;    /* bytes between slots and pool entries (>= blob_bytes, multiple of 256) */
+    void *host_pool;        /* host [n_experts * slot_stride], caller-owned; page-locked unless use_staging */
+    void *hbm_slab;         /* device [capacity * slot_stride], caller-owned */
+    void *dev_table;        /* device [n_experts] pointers, caller-owned; set to NULL at create */
+    void *stage_buffer;     /* host, page-locked, >= 2 * slot_stride bytes; used only with use_staging */
+    int32_t decay_period;   /* steps between halvings; 0 = never */
+    int32_t use_staging;    /* 1: pool may be pageable; copies bounce through stage_buffer (double-buffered) */
+} moe_expcache_desc;
+
+typedef struct {
+    int64_t steps, hits, misses, evictions, bytes_staged;
+    int32_t resident;
+} moe_expcache_stats;
+
+/* Creates the cache (empty).  Returns MOE_EINVAL on bad descriptors. */
+int expcache_create(const moe_expcache_desc *d, moe_expcache **out);
+void expcache_destroy(moe_expcache *c);
+
+/* Query only, no state change: slots_out[i] = slot of ids_host[i] or -1. */
+int expcache_lookup(moe_expcache *c, const int32_t *ids_host, int n, int32_t *slots_out, int *n_miss);
+
+/* One step: policy bookkeeping for the n distinct ids (host array), then the
+ * copies of the misses.  Outputs (host, optional, n entries each): hit[i]
+ * 1/0, slot[i], victim[i] (-1 = none).  The compute stream's work queued so
+ * far is ordered before any slot is overwritten.  Returns MOE_EBUSY if
+ * n > capacity, MOE_EINVAL for bad or repeated ids, MOE_EIO/MOE_ECUDA if
+ * issuing a copy failed (the step's bookkeeping is then rolled back). */
+int expcache_stage(moe_expcache *c, const int32_t *ids_host, int n, moe_stream_t compute,
+                   int32_t *hit_out, int32_t *slot_out, int32_t *victim_out);
+
+/* Makes `s` wait (cudaStreamWaitEvent) for every copy and table update issued so far. */
+int expcache_join(moe_expcache *c, moe_stream_t s);
+
+/* Host wait for the staged copies with a time limit; MOE_ETIMEDOUT if not done. */
+int expcache_wait(moe_expcache *c, int64_t timeout_us);
+
+/* Evicts the given resident ids (NULL/0 = nothing).  Non-resident ids are ignored. */
+int expcache_evict(moe_expcache *c, const int32_t *ids_host, int n);
+
+/* The descriptor's dev_table: device [n_experts] blob pointers (NULL = not
+ * resident), for the FFN calls. */
+const void *const *expcache_device_table(moe_expcache *c);
+
+int expcache_stats(moe_expcache *c, moe_expcache_stats *out);
+
+/* Host copy of the per-expert counters and slots (n_experts entries each; either may be NULL). */
+int expcache_snapshot(moe_expcache *c, int64_t *counts_out, int32_t *slot_of_out);
+
+/* Test hook: the next `n` copies report failure before being issued (MOE_EIO). */
+int expcache_inject_copy_failures(moe_expcache *c, int n);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_H_ */

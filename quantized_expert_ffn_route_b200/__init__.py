@@ -1,0 +1,268 @@
+"""Python binding of libmoe, the B200 quantized MoE expert step.
+
+Argument marshalling only: every function below forwards to the C ABI
+declared in include/moe.h with the same name; all arithmetic runs in the
+CUDA kernels of libmoe.so.  There is no CPU fallback: if the shared library
+is missing, the first call raises.
+
+Device buffers are passed as torch CUDA tensors (or raw integer pointers);
+torch is used only for device memory and streams.
+"""
+from __future__ import annotations
+
+import ctypes as C
+from pathlib import Path
+
+from .layer import MoELayer, alloc_step_buffers  # noqa: F401
+
+_PKG = Path(__file__).resolve().parent
+LIB_PATH = _PKG / "_build" / "libmoe.so"
+HEADER = _PKG.parent / "include" / "moe.h"
+
+MOE_OK, MOE_EINVAL, MOE_ENOMEM, MOE_ECUDA, MOE_EBUSY, MOE_ETIMEDOUT, MOE_EIO, MOE_EDEVICE = range(8)
+MOE_F32, MOE_BF16 = 0, 1
+MOE_MODE_AUTO, MOE_MODE_GEMV, MOE_MODE_GEMM = 0, 1, 2
+DEVERR_BAD_EXPERT, DEVERR_NULL_BLOB, DEVERR_NONFINITE, DEVERR_BAD_ROW = 1, 2, 4, 8
+
+_STATUS = {1: "MOE_EINVAL", 2: "MOE_ENOMEM", 3: "MOE_ECUDA", 4: "MOE_EBUSY", 5: "MOE_ETIMEDOUT",
+           6: "MOE_EIO", 7: "MOE_EDEVICE"}
+
+
+class MoEError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{_STATUS.get(status, status)}: {msg}")
+        self.status = status
+
+
+class ExpCacheDesc(C.Structure):
+    _fields_ = [("n_experts", C.c_int32), ("capacity", C.c_int32), ("blob_bytes", C.c_int64),
+                ("slot_stride", C.c_int64), ("host_pool", C.c_void_p), ("hbm_slab", C.c_void_p),
+                ("dev_table", C.c_void_p), ("stage_buffer", C.c_void_p), ("decay_period", C.c_int32),
+                ("use_staging", C.c_int32)]
+
+
+class ExpCacheStats(C.Structure):
+    _fields_ = [("steps", C.c_int64), ("hits", C.c_int64), ("misses", C.c_int64),
+                ("evictions", C.c_int64), ("bytes_staged", C.c_int64), ("resident", C.c_int32)]
+
+
+_lib = None
+
+
+def lib():
+    """Loads libmoe.so (built in-tree by build()); raises if it is missing."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not LIB_PATH.exists():
+        raise RuntimeError(f"libmoe.so not found at {LIB_PATH}; build it with "
+                           "`python -m quantized_expert_ffn_route_b200.build`")
+    import torch  # noqa: F401  (loads the CUDA runtime libmoe shares with torch)
+    L = C.CDLL(str(LIB_PATH))
+    P, I, Z, S = C.c_void_p, C.c_int, C.c_size_t, C.c_void_p
+    sig = {
+        "moe_last_error": (C.c_char_p, []),
+        "moe_version": (I, []),
+        "moe_kernel_launches": (C.c_uint64, []),
+        "moe_device_error": (I, [P, I, S]),
+        "moe_expert_blob_bytes": (Z, [I, I, I]),
+        "moe_route_ws_size": (Z, [I, I, I]),
+        "moe_route_topk": (I, [P, I, P, I, P, P, I, I, I, I, P, P, P, P, Z, S]),
+        "moe_permute_ws_size": (Z, [I, I, I]),
+        "moe_permute": (I, [P, I, I, I, P, P, P, P, P, Z, S]),
+        "moe_expert_ffn_ws_size": (Z, [I, I, I, I, I, I, I]),
+        "moe_expert_ffn_q4": (I, [P, P, P, P, P, I, I, I, I, I, I, P, P, P, I, P, Z, S]),
+        "moe_expert_ffn_q2": (I, [P, P, P, P, P, I, I, I, I, I, I, P, P, P, I, P, Z, S]),
+        "moe_combine": (I, [P, P, P, P, I, I, I, P, S]),
+        "expcache_create": (I, [C.POINTER(ExpCacheDesc), C.POINTER(P)]),
+        "expcache_destroy": (None, [P]),
+        "expcache_lookup": (I, [P, P, I, P, P]),
+        "expcache_stage": (I, [P, P, I, S, P, P, P]),
+        "expcache_join": (I, [P, S]),
+        "expcache_wait": (I, [P, C.c_int64]),
+        "expcache_evict": (I, [P, P, I]),
+        "expcache_device_table": (P, [P]),
+        "expcache_stats": (I, [P, C.POINTER(ExpCacheStats)]),
+        "expcache_snapshot": (I, [P, P, P]),
+        "expcache_inject_copy_failures": (I, [P, I]),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(L, name)
+        f.restype = res
+        f.argtypes = args
+    _lib = L
+    return L
+
+
+def _p(t):
+    """Pointer of a tensor / numpy array / int / None."""
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    if hasattr(t, "data_ptr"):
+        return t.data_ptr()
+    if hasattr(t, "ctypes"):
+        return t.ctypes.data
+    raise TypeError(f"cannot take a pointer of {type(t)}")
+
+
+def _stream(s):
+    if s is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(s, int):
+        return s
+    return s.cuda_stream
+
+
+def _check(rc: int):
+    if rc != MOE_OK:
+        raise MoEError(rc, lib().moe_last_error().decode())
+    return rc
+
+
+# ----------------------------------------------------------------- the ABI
+def moe_version() -> int:
+    return lib().moe_version()
+
+
+def moe_kernel_launches() -> int:
+    return lib().moe_kernel_launches()
+
+
+def moe_last_error() -> str:
+    return lib().moe_last_error().decode()
+
+
+def moe_device_error(clear: bool = True, stream=None) -> int:
+    """Returns the device error bits (0 if none); raises only on CUDA failure."""
+    bits = C.c_uint32(0)
+    rc = lib().moe_device_error(C.byref(bits), int(clear), _stream(stream))
+    if rc not in (MOE_OK, MOE_EDEVICE):
+        _check(rc)
+    return bits.value
+
+
+def moe_expert_blob_bytes(bits: int, H: int, I: int) -> int:
+    return lib().moe_expert_blob_bytes(bits, H, I)
+
+
+def moe_route_ws_size(T, E, k):
+    return lib().moe_route_ws_size(T, E, k)
+
+
+def moe_route_topk(x, x_dtype, w_router, w_dtype, logits_in, bias, T, H, E, k, topk_ids, topk_w,
+                   logits_out=None, ws=None, ws_bytes=0, stream=None):
+    return _check(lib().moe_route_topk(_p(x), x_dtype, _p(w_router), w_dtype, _p(logits_in), _p(bias), T, H, E,
+                                       k, _p(topk_ids), _p(topk_w), _p(logits_out), _p(ws), ws_bytes,
+                                       _stream(stream)))
+
+
+def moe_permute_ws_size(T, k, E):
+    return lib().moe_permute_ws_size(T, k, E)
+
+
+def moe_permute(topk_ids, T, k, E, expert_offsets, perm_src, perm_dst, active=None, ws=None, ws_bytes=0,
+                stream=None):
+    return _check(lib().moe_permute(_p(topk_ids), T, k, E, _p(expert_offsets), _p(perm_src), _p(perm_dst),
+                                    _p(active), _p(ws), ws_bytes, _stream(stream)))
+
+
+def moe_expert_ffn_ws_size(bits, T, k, H, I, E, mode=MOE_MODE_AUTO):
+    return lib().moe_expert_ffn_ws_size(bits, T, k, H, I, E, mode)
+
+
+def _ffn(name, expert_blobs, expert_offsets, active, perm_src, x, x_dtype, T, k, H, I, E, shared_blob, y_perm,
+         y_shared, mode, ws, ws_bytes, stream):
+    f = getattr(lib(), name)
+    return _check(f(_p(expert_blobs), _p(expert_offsets), _p(active), _p(perm_src), _p(x), x_dtype, T, k, H, I, E,
+                    _p(shared_blob), _p(y_perm), _p(y_shared), mode, _p(ws), ws_bytes, _stream(stream)))
+
+
+def moe_expert_ffn_q4(expert_blobs, expert_offsets, active, perm_src, x, x_dtype, T, k, H, I, E, shared_blob,
+                      y_perm, y_shared, mode=MOE_MODE_AUTO, ws=None, ws_bytes=0, stream=None):
+    return _ffn("moe_expert_ffn_q4", expert_blobs, expert_offsets, active, perm_src, x, x_dtype, T, k, H, I, E,
+                shared_blob, y_perm, y_shared, mode, ws, ws_bytes, stream)
+
+
+def moe_expert_ffn_q2(expert_blobs, expert_offsets, active, perm_src, x, x_dtype, T, k, H, I, E, shared_blob,
+                      y_perm, y_shared, mode=MOE_MODE_AUTO, ws=None, ws_bytes=0, stream=None):
+    return _ffn("moe_expert_ffn_q2", expert_blobs, expert_offsets, active, perm_src, x, x_dtype, T, k, H, I, E,
+                shared_blob, y_perm, y_shared, mode, ws, ws_bytes, stream)
+
+
+def moe_combine(y_perm, perm_dst, topk_w, y_shared, T, k, H, y, stream=None):
+    return _check(lib().moe_combine(_p(y_perm), _p(perm_dst), _p(topk_w), _p(y_shared), T, k, H, _p(y),
+                                    _stream(stream)))
+
+
+class ExpCache:
+    """Handle around the expcache_* calls (the caller owns pool, slab and table)."""
+
+    def __init__(self, n_experts, capacity, blob_bytes, slot_stride, host_pool, hbm_slab, dev_table,
+                 decay_period=256, stage_buffer=None):
+        d = ExpCacheDesc(n_experts, capacity, blob_bytes, slot_stride, _p(host_pool), _p(hbm_slab),
+                         _p(dev_table), _p(stage_buffer), decay_period, 1 if stage_buffer is not None else 0)
+        h = C.c_void_p()
+        _check(lib().expcache_create(C.byref(d), C.byref(h)))
+        self.h = h
+        self.n_experts = n_experts
+
+    def close(self):
+        if self.h:
+            lib().expcache_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def lookup(self, ids):
+        import numpy as np
+        ids = np.ascontiguousarray(ids, dtype=np.int32)
+        slots = np.empty(ids.size, np.int32)
+        nm = C.c_int(0)
+        _check(lib().expcache_lookup(self.h, _p(ids), ids.size, _p(slots), C.byref(nm)))
+        return slots, nm.value
+
+    def stage(self, ids, stream=None):
+        """One step; returns (hit, slot, victim) numpy arrays."""
+        import numpy as np
+        ids = np.ascontiguousarray(ids, dtype=np.int32)
+        hit = np.empty(ids.size, np.int32)
+        slot = np.empty(ids.size, np.int32)
+        victim = np.empty(ids.size, np.int32)
+        _check(lib().expcache_stage(self.h, _p(ids), ids.size, _stream(stream), _p(hit), _p(slot), _p(victim)))
+        return hit, slot, victim
+
+    def join(self, stream=None):
+        _check(lib().expcache_join(self.h, _stream(stream)))
+
+    def wait(self, timeout_us: int):
+        return lib().expcache_wait(self.h, int(timeout_us))
+
+    def evict(self, ids):
+        import numpy as np
+        ids = np.ascontiguousarray(ids, dtype=np.int32)
+        _check(lib().expcache_evict(self.h, _p(ids), ids.size))
+
+    def device_table(self) -> int:
+        return lib().expcache_device_table(self.h)
+
+    def stats(self) -> dict:
+        s = ExpCacheStats()
+        _check(lib().expcache_stats(self.h, C.byref(s)))
+        return {f: getattr(s, f) for f, _ in ExpCacheStats._fields_}
+
+    def snapshot(self):
+        import numpy as np
+        cnt = np.empty(self.n_experts, np.int64)
+        slot = np.empty(self.n_experts, np.int32)
+        _check(lib().expcache_snapshot(self.h, _p(cnt), _p(slot)))
+        return cnt, slot
+
+    def inject_copy_failures(self, n: int):
+        _check(lib().expcache_inject_copy_failures(self.h, n))

@@ -1,0 +1,74 @@
+// Shared device/host helpers of libmoe (not shared with the oracle).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "moe.h"
+
+namespace moe {
+
+// ---------------------------------------------------------------- host side
+void set_error(const char *fmt, ...);
+int cuda_status(cudaError_t e, const char *what);   // MOE_OK or MOE_ECUDA (+ message)
+unsigned *device_error_word();                       // this device's error word, or nullptr
+int num_sms();                                       // SMs of the current device (cached)
+void count_launches(int n);                          // adds to the library's launch counter
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// -------------------------------------------------------------- device side
+__device__ __forceinline__ void report(unsigned *err, unsigned bits) {
+    if (err) atomicOr(err, bits);
+}
+
+__device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
+    return __uint_as_float(static_cast<uint32_t>(b) << 16);
+}
+
+template <typename T> __device__ __forceinline__ float to_f32(T v);
+template <> __device__ __forceinline__ float to_f32<float>(float v) { return v; }
+template <> __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 v) {
+    return __bfloat162float(v);
+}
+
+// Four consecutive activations as floats (16-byte aligned f32 or 8-byte aligned bf16).
+__device__ __forceinline__ float4 load4(const float *p) { return *reinterpret_cast<const float4 *>(p); }
+__device__ __forceinline__ float4 load4(const __nv_bfloat16 *p) {
+    uint2 u = *reinterpret_cast<const uint2 *>(p);
+    return make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xffff0000u),
+                       __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xffff0000u));
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// Byte offsets inside an expert blob (codes Wg, Wu, Wd, then fp16 scales).
+struct BlobView {
+    const uint8_t *cg, *cu, *cd;
+    const __half *sg, *su, *sd;
+};
+
+__device__ __forceinline__ BlobView blob_view(const uint8_t *b, int bits, int H, int I) {
+    size_t cb = static_cast<size_t>(I) * H * bits / 8;      // code bytes per matrix
+    size_t sb = static_cast<size_t>(I) * H / 32;            // scales per matrix
+    BlobView v;
+    v.cg = b;
+    v.cu = b + cb;
+    v.cd = b + 2 * cb;
+    v.sg = reinterpret_cast<const __half *>(b + 3 * cb);
+    v.su = v.sg + sb;
+    v.sd = v.su + sb;
+    return v;
+}
+
+inline size_t blob_bytes_host(int bits, int H, int I) {
+    return 3 * static_cast<size_t>(I) * H * bits / 8 + 3 * static_cast<size_t>(I) * H / 32 * 2;
+}
+
+}  // namespace moe

@@ -1,0 +1,359 @@
+// Expert cache: frequency-driven residency of expert blobs in an HBM slab,
+// paged in from a page-locked host pool.
+//
+// Strata article, section 2 item 2: the most-called experts live in VRAM,
+// all experts in RAM; an expert the router picks is computed at once when
+// resident, otherwise it is first moved in.  Section 3: part of the RAM is
+// page-locked for the GPU.  Strata code review, section 3: a stage buffer
+// whose page-locking became optional.  Janas-LLM page: experts used again
+// stay in the cache.
+//
+// Host bookkeeping is O(log capacity) per access (an ordered set keyed by
+// (counter, last use, id) over the resident experts); each miss is one
+// cudaMemcpyAsync on the cache's own stream, after which one small kernel
+// patches the device table of blob pointers.
+#include <chrono>
+#include <cstring>
+#include <new>
+#include <set>
+#include <thread>
+#include <tuple>
+#include <vector>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+
+__global__ void k_table_patch(const void **table, TablePatch p) {
+    const int i = threadIdx.x;
+    if (i < p.n) table[p.ids[i]] = p.ptrs[i];
+}
+
+int launch_table_patch(const void **table, const TablePatch &p, cudaStream_t s) {
+    if (p.n <= 0) return MOE_OK;
+    k_table_patch<<<1, 64, 0, s>>>(table, p); count_launches(1);
+    return cuda_status(cudaGetLastError(), "table patch launch");
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+struct moe_expcache {
+    moe_expcache_desc d;
+    int device = 0;
+    cudaStream_t copy = nullptr;
+    cudaEvent_t ev_compute = nullptr;     // compute stream position at the last stage call
+    cudaEvent_t ev_done = nullptr;        // all copies + table patch issued so far
+    cudaEvent_t ev_stage[2] = {nullptr, nullptr};   // staging halves free again
+    int stage_next = 0;
+    std::vector<int32_t> slot_of, expert_in;
+    std::vector<int64_t> cnt, last;
+    std::set<std::tuple<int64_t, int64_t, int32_t>> order;   // resident experts by (cnt, last, id)
+    std::set<int32_t> free_slots;
+    int64_t step = 0;
+    moe_expcache_stats st{};
+    int inject_fail = 0;
+};
+
+#define REQUIRE(cond, ...)            \
+    do {                              \
+        if (!(cond)) {                \
+            set_error(__VA_ARGS__);   \
+            return MOE_EINVAL;        \
+        }                             \
+    } while (0)
+
+// Makes the cache's device current for the scope and restores the caller's.
+struct DeviceGuard {
+    int prev = -1;
+    explicit DeviceGuard(int dev) {
+        if (cudaGetDevice(&prev) == cudaSuccess && prev != dev) cudaSetDevice(dev);
+    }
+    ~DeviceGuard() {
+        int cur = -1;
+        if (prev >= 0 && cudaGetDevice(&cur) == cudaSuccess && cur != prev) cudaSetDevice(prev);
+    }
+};
+
+static void destroy_events(moe_expcache *c) {
+    if (c->ev_compute) cudaEventDestroy(c->ev_compute);
+    if (c->ev_done) cudaEventDestroy(c->ev_done);
+    for (auto &e : c->ev_stage)
+        if (e) cudaEventDestroy(e);
+    if (c->copy) cudaStreamDestroy(c->copy);
+}
+
+extern "C" {
+
+int expcache_create(const moe_expcache_desc *d, moe_expcache **out) {
+    REQUIRE(d && out, "desc/out are NULL");
+    *out = nullptr;
+    REQUIRE(d->n_experts >= 1, "n_experts must be >= 1");
+    REQUIRE(d->capacity >= 1, "capacity must be >= 1");
+    REQUIRE(d->blob_bytes > 0 && d->blob_bytes % 16 == 0, "blob_bytes must be a positive multiple of 16");
+    REQUIRE(d->slot_stride >= d->blob_bytes && d->slot_stride % 256 == 0,
+            "slot_stride must be >= blob_bytes and a multiple of 256");
+    REQUIRE(d->host_pool && d->hbm_slab && d->dev_table, "host_pool/hbm_slab/dev_table must not be NULL");
+    REQUIRE(aligned16(d->host_pool) && aligned16(d->hbm_slab) && aligned16(d->dev_table),
+            "host_pool/hbm_slab/dev_table must be 16-byte aligned");
+    REQUIRE(d->decay_period >= 0, "decay_period must be >= 0");
+    REQUIRE(!d->use_staging || d->stage_buffer, "use_staging needs a stage_buffer");
+    moe_expcache *c = new (std::nothrow) moe_expcache();
+    if (!c) {
+        set_error("out of host memory");
+        return MOE_ENOMEM;
+    }
+    c->d = *d;
+    cudaGetDevice(&c->device);
+    int rc = cuda_status(cudaStreamCreateWithFlags(&c->copy, cudaStreamNonBlocking), "copy stream");
+    if (!rc) rc = cuda_status(cudaEventCreateWithFlags(&c->ev_compute, cudaEventDisableTiming), "event");
+    if (!rc) rc = cuda_status(cudaEventCreateWithFlags(&c->ev_done, cudaEventDisableTiming), "event");
+    for (int i = 0; i < 2 && !rc; ++i)
+        rc = cuda_status(cudaEventCreateWithFlags(&c->ev_stage[i], cudaEventDisableTiming), "event");
+    if (!rc)
+        rc = cuda_status(cudaMemsetAsync(d->dev_table, 0, sizeof(void *) * static_cast<size_t>(d->n_experts), c->copy),
+                         "table clear");
+    if (!rc) rc = cuda_status(cudaEventRecord(c->ev_done, c->copy), "event record");
+    for (int i = 0; i < 2 && !rc; ++i) rc = cuda_status(cudaEventRecord(c->ev_stage[i], c->copy), "event record");
+    if (rc) {
+        destroy_events(c);
+        delete c;
+        return rc;
+    }
+    try {
+        c->slot_of.assign(d->n_experts, -1);
+        c->expert_in.assign(d->capacity, -1);
+        c->cnt.assign(d->n_experts, 0);
+        c->last.assign(d->n_experts, -1);
+        for (int s = 0; s < d->capacity; ++s) c->free_slots.insert(s);
+    } catch (...) {
+        destroy_events(c);
+        delete c;
+        set_error("out of host memory");
+        return MOE_ENOMEM;
+    }
+    *out = c;
+    return MOE_OK;
+}
+
+void expcache_destroy(moe_expcache *c) {
+    if (!c) return;
+    DeviceGuard g(c->device);
+    cudaStreamSynchronize(c->copy);
+    destroy_events(c);
+    delete c;
+}
+
+int expcache_lookup(moe_expcache *c, const int32_t *ids_host, int n, int32_t *slots_out, int *n_miss) {
+    REQUIRE(c && (n == 0 || ids_host), "cache/ids are NULL");
+    REQUIRE(n >= 0, "n must be >= 0");
+    int miss = 0;
+    for (int i = 0; i < n; ++i) {
+        const int e = ids_host[i];
+        REQUIRE(e >= 0 && e < c->d.n_experts, "expert id %d out of range", e);
+        const int s = c->slot_of[e];
+        if (slots_out) slots_out[i] = s;
+        miss += s < 0;
+    }
+    if (n_miss) *n_miss = miss;
+    return MOE_OK;
+}
+
+int expcache_stage(moe_expcache *c, const int32_t *ids_host, int n, moe_stream_t compute, int32_t *hit_out,
+                   int32_t *slot_out, int32_t *victim_out) {
+    REQUIRE(c && (n == 0 || ids_host), "cache/ids are NULL");
+    REQUIRE(n >= 0 && n <= 32, "n must be in [0, 32]");
+    if (n > c->d.capacity) {
+        set_error("step needs %d experts but the cache holds %d", n, c->d.capacity);
+        return MOE_EBUSY;
+    }
+    for (int i = 0; i < n; ++i) {
+        REQUIRE(ids_host[i] >= 0 && ids_host[i] < c->d.n_experts, "expert id %d out of range", ids_host[i]);
+        for (int j = 0; j < i; ++j) REQUIRE(ids_host[j] != ids_host[i], "expert id %d repeated in a step", ids_host[i]);
+    }
+    int n_miss = 0;
+    for (int i = 0; i < n; ++i) n_miss += c->slot_of[ids_host[i]] < 0;
+    if (n_miss > 0 && c->inject_fail > 0) {   // test hook: fail before any state changes
+        c->inject_fail--;
+        set_error("injected staging-copy failure");
+        return MOE_EIO;
+    }
+    DeviceGuard guard(c->device);
+    const int64_t s = c->step;
+    // halving decay at the start of every decay_period-th step
+    if (c->d.decay_period > 0 && s > 0 && s % c->d.decay_period == 0) {
+        for (auto &v : c->cnt) v /= 2;
+        c->order.clear();
+        for (int e = 0; e < c->d.n_experts; ++e)
+            if (c->slot_of[e] >= 0) c->order.emplace(c->cnt[e], c->last[e], e);
+    }
+    TablePatch patch{};
+    struct Copy { int32_t id, slot; };
+    Copy copies[32];
+    int nc = 0;
+    for (int i = 0; i < n; ++i) {
+        const int e = ids_host[i];
+        const bool resident = c->slot_of[e] >= 0;
+        if (resident) c->order.erase(std::make_tuple(c->cnt[e], c->last[e], e));
+        c->cnt[e] += 1;
+        c->last[e] = s;
+        int victim = -1;
+        if (resident) {
+            c->order.emplace(c->cnt[e], c->last[e], e);
+            c->st.hits++;
+        } else {
+            int slot;
+            if (!c->free_slots.empty()) {
+                slot = *c->free_slots.begin();
+                c->free_slots.erase(c->free_slots.begin());
+            } else {
+                auto it = c->order.begin();
+                for (; it != c->order.end(); ++it) {
+                    const int v = std::get<2>(*it);
+                    bool in_step = false;
+                    for (int j = 0; j < n; ++j) in_step |= ids_host[j] == v;
+                    if (!in_step) break;
+                }
+                victim = std::get<2>(*it);   // exists: capacity >= n and e is not resident
+                c->order.erase(it);
+                slot = c->slot_of[victim];
+                c->slot_of[victim] = -1;
+                c->st.evictions++;
+                patch.ids[patch.n] = victim;
+                patch.ptrs[patch.n] = nullptr;
+                patch.n++;
+            }
+            c->slot_of[e] = slot;
+            c->expert_in[slot] = e;
+            c->order.emplace(c->cnt[e], c->last[e], e);
+            copies[nc++] = Copy{e, slot};
+            c->st.misses++;
+        }
+        if (hit_out) hit_out[i] = resident ? 1 : 0;
+        if (slot_out) slot_out[i] = c->slot_of[e];
+        if (victim_out) victim_out[i] = victim;
+    }
+    c->step++;
+    c->st.steps++;
+    if (nc == 0) return MOE_OK;
+    // copies start after the compute work queued so far (it may still read victims' slots)
+    int rc = cuda_status(cudaEventRecord(c->ev_compute, reinterpret_cast<cudaStream_t>(compute)), "event record");
+    if (!rc) rc = cuda_status(cudaStreamWaitEvent(c->copy, c->ev_compute, 0), "stream wait");
+    const size_t B = static_cast<size_t>(c->d.blob_bytes), S = static_cast<size_t>(c->d.slot_stride);
+    auto *slab = static_cast<uint8_t *>(c->d.hbm_slab);
+    auto *pool = static_cast<const uint8_t *>(c->d.host_pool);
+    for (int i = 0; i < nc && !rc; ++i) {
+        uint8_t *dst = slab + static_cast<size_t>(copies[i].slot) * S;
+        const uint8_t *src = pool + static_cast<size_t>(copies[i].id) * S;
+        if (c->d.use_staging) {
+            const int h = c->stage_next;
+            c->stage_next ^= 1;
+            rc = cuda_status(cudaEventSynchronize(c->ev_stage[h]), "stage wait");
+            uint8_t *buf = static_cast<uint8_t *>(c->d.stage_buffer) + static_cast<size_t>(h) * S;
+            if (!rc) std::memcpy(buf, src, B);
+            if (!rc) rc = cuda_status(cudaMemcpyAsync(dst, buf, B, cudaMemcpyHostToDevice, c->copy), "stage copy");
+            if (!rc) rc = cuda_status(cudaEventRecord(c->ev_stage[h], c->copy), "event record");
+        } else {
+            rc = cuda_status(cudaMemcpyAsync(dst, src, B, cudaMemcpyHostToDevice, c->copy), "expert copy");
+        }
+        if (rc) rc = MOE_EIO;
+        else {
+            patch.ids[patch.n] = copies[i].id;
+            patch.ptrs[patch.n] = dst;
+            patch.n++;
+            c->st.bytes_staged += static_cast<int64_t>(B);
+        }
+    }
+    if (rc) {
+        // copies that could not be issued leave their experts out of the cache
+        for (int i = 0; i < nc; ++i) {
+            bool issued = false;
+            for (int j = 0; j < patch.n; ++j) issued |= patch.ids[j] == copies[i].id && patch.ptrs[j] != nullptr;
+            if (!issued) {
+                const int e = copies[i].id;
+                c->order.erase(std::make_tuple(c->cnt[e], c->last[e], e));
+                c->expert_in[copies[i].slot] = -1;
+                c->slot_of[e] = -1;
+                c->free_slots.insert(copies[i].slot);
+            }
+        }
+    }
+    int rc2 = launch_table_patch(reinterpret_cast<const void **>(c->d.dev_table), patch, c->copy);
+    if (!rc2) rc2 = cuda_status(cudaEventRecord(c->ev_done, c->copy), "event record");
+    return rc ? rc : rc2;
+}
+
+int expcache_join(moe_expcache *c, moe_stream_t s) {
+    REQUIRE(c != nullptr, "cache is NULL");
+    return cuda_status(cudaStreamWaitEvent(reinterpret_cast<cudaStream_t>(s), c->ev_done, 0), "stream wait");
+}
+
+int expcache_wait(moe_expcache *c, int64_t timeout_us) {
+    REQUIRE(c != nullptr, "cache is NULL");
+    const auto t0 = std::chrono::steady_clock::now();
+    for (;;) {
+        const cudaError_t e = cudaEventQuery(c->ev_done);
+        if (e == cudaSuccess) return MOE_OK;
+        if (e != cudaErrorNotReady) return cuda_status(e, "event query");
+        const auto us =
+            std::chrono::duration_cast<std::chrono::microseconds>(std::chrono::steady_clock::now() - t0).count();
+        if (us >= timeout_us) {
+            set_error("staged copies not done after %lld us", static_cast<long long>(timeout_us));
+            return MOE_ETIMEDOUT;
+        }
+        std::this_thread::sleep_for(std::chrono::microseconds(20));
+    }
+}
+
+int expcache_evict(moe_expcache *c, const int32_t *ids_host, int n) {
+    REQUIRE(c && (n == 0 || ids_host), "cache/ids are NULL");
+    REQUIRE(n >= 0 && n <= 64, "n must be in [0, 64]");
+    TablePatch patch{};
+    for (int i = 0; i < n; ++i) {
+        const int e = ids_host[i];
+        REQUIRE(e >= 0 && e < c->d.n_experts, "expert id %d out of range", e);
+        const int s = c->slot_of[e];
+        if (s < 0) continue;
+        c->order.erase(std::make_tuple(c->cnt[e], c->last[e], e));
+        c->slot_of[e] = -1;
+        c->expert_in[s] = -1;
+        c->free_slots.insert(s);
+        c->st.evictions++;
+        patch.ids[patch.n] = e;
+        patch.ptrs[patch.n] = nullptr;
+        patch.n++;
+    }
+    if (patch.n == 0) return MOE_OK;
+    DeviceGuard guard(c->device);
+    int rc = launch_table_patch(reinterpret_cast<const void **>(c->d.dev_table), patch, c->copy);
+    if (!rc) rc = cuda_status(cudaEventRecord(c->ev_done, c->copy), "event record");
+    return rc;
+}
+
+const void *const *expcache_device_table(moe_expcache *c) {
+    return c ? static_cast<const void *const *>(c->d.dev_table) : nullptr;
+}
+
+int expcache_stats(moe_expcache *c, moe_expcache_stats *out) {
+    REQUIRE(c && out, "cache/out are NULL");
+    *out = c->st;
+    out->resident = c->d.capacity - static_cast<int32_t>(c->free_slots.size());
+    return MOE_OK;
+}
+
+int expcache_snapshot(moe_expcache *c, int64_t *counts_out, int32_t *slot_of_out) {
+    REQUIRE(c != nullptr, "cache is NULL");
+    if (counts_out) std::memcpy(counts_out, c->cnt.data(), sizeof(int64_t) * c->cnt.size());
+    if (slot_of_out) std::memcpy(slot_of_out, c->slot_of.data(), sizeof(int32_t) * c->slot_of.size());
+    return MOE_OK;
+}
+
+int expcache_inject_copy_failures(moe_expcache *c, int n) {
+    REQUIRE(c && n >= 0, "bad arguments");
+    c->inject_fail = n;
+    return MOE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,105 @@
+"""C-ABI checks that need no GPU: the library loads, exports every function
+that include/moe.h declares, sizes workspaces, and rejects bad arguments on
+the host before touching the device."""
+import ctypes as C
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+import quantized_expert_ffn_route_b200 as M
+
+
+def _declared():
+    src = M.HEADER.read_text()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"\b((?:moe|expcache)_[a-z0-9_]+)\s*\(", src)
+    return sorted(set(names))
+
+
+def test_library_exports_every_declared_symbol():
+    names = _declared()
+    assert len(names) >= 20
+    L = M.lib()
+    for n in names:
+        assert hasattr(L, n), n
+    out = subprocess.run(["nm", "-D", "--defined-only", str(M.LIB_PATH)], capture_output=True, text=True).stdout
+    exported = set(re.findall(r" T ((?:moe|expcache)_\w+)$", out, flags=re.M))
+    assert set(names) <= exported
+    assert M.moe_version() == 100
+
+
+def test_blob_and_workspace_sizes():
+    assert M.moe_expert_blob_bytes(4, 2048, 512) == 1_769_472
+    assert M.moe_expert_blob_bytes(2, 2048, 512) == 983_040
+    assert M.moe_expert_blob_bytes(3, 2048, 512) == 0
+    assert M.moe_route_ws_size(8, 512, 10) == 8 * 512 * 4
+    assert M.moe_permute_ws_size(1, 10, 512) == 0            # one-block path needs no workspace
+    assert M.moe_permute_ws_size(8192, 10, 512) > 0
+    assert M.moe_expert_ffn_ws_size(4, 1, 10, 2048, 512, 512, M.MOE_MODE_GEMV) == 11 * 512 * 4
+    assert M.moe_expert_ffn_ws_size(4, 0, 10, 2048, 512, 512, 0) == 0
+
+
+def _rc(fn, *a):
+    return getattr(M.lib(), fn)(*a)
+
+
+def test_route_rejects_bad_arguments_on_host():
+    buf = np.zeros(64, np.float32)
+    p = buf.ctypes.data
+    # k > E, k = 0, E too large, T negative
+    assert _rc("moe_route_topk", p, 0, p, 0, None, None, 1, 8, 4, 5, p, p, None, p, 1024, None) == M.MOE_EINVAL
+    assert "k must be" in M.moe_last_error()
+    assert _rc("moe_route_topk", p, 0, p, 0, None, None, 1, 8, 4, 0, p, p, None, p, 1024, None) == M.MOE_EINVAL
+    assert _rc("moe_route_topk", p, 0, p, 0, None, None, 1, 8, 40000, 4, p, p, None, p, 1024, None) == M.MOE_EINVAL
+    assert _rc("moe_route_topk", p, 0, p, 0, None, None, -1, 8, 4, 2, p, p, None, p, 1024, None) == M.MOE_EINVAL
+    # bad dtype, misaligned pointer, missing workspace, no logits source
+    assert _rc("moe_route_topk", p, 7, p, 0, None, None, 1, 8, 4, 2, p, p, None, p, 1024, None) == M.MOE_EINVAL
+    assert _rc("moe_route_topk", p + 4, 0, p, 0, None, None, 1, 8, 4, 2, p, p, None, p, 1024, None) == M.MOE_EINVAL
+    assert _rc("moe_route_topk", p, 0, p, 0, None, None, 1, 8, 4, 2, p, p, None, p, 8, None) == M.MOE_EINVAL
+    assert "workspace" in M.moe_last_error()
+    assert _rc("moe_route_topk", None, 0, None, 0, None, None, 1, 8, 4, 2, p, p, None, None, 0, None) == M.MOE_EINVAL
+    # T = 0 is a no-op
+    assert _rc("moe_route_topk", None, 0, None, 0, None, None, 0, 8, 4, 2, None, None, None, None, 0, None) == 0
+
+
+def test_permute_and_ffn_reject_bad_arguments_on_host():
+    buf = np.zeros(1024, np.int32)
+    p = buf.ctypes.data
+    assert _rc("moe_permute", p, 1, 0, 16, p, p, p, p, None, 0, None) == M.MOE_EINVAL
+    assert _rc("moe_permute", p, 1, 4, 0, p, p, p, p, None, 0, None) == M.MOE_EINVAL
+    assert _rc("moe_permute", p, 1, 4, 16, p + 4, p, p, p, None, 0, None) == M.MOE_EINVAL
+    assert _rc("moe_permute", p, 8192, 10, 512, p, p, p, p, None, 0, None) == M.MOE_EINVAL   # workspace
+    f = M.lib().moe_expert_ffn_q4
+    # H not a multiple of 128, I too large, bad mode, NULL pointers, missing workspace
+    assert f(p, p, p, p, p, 1, 1, 2, 200, 512, 16, None, p, None, 0, p, 1 << 20, None) == M.MOE_EINVAL
+    assert f(p, p, p, p, p, 1, 1, 2, 256, 8192, 16, None, p, None, 0, p, 1 << 20, None) == M.MOE_EINVAL
+    assert f(p, p, p, p, p, 1, 1, 2, 256, 128, 16, None, p, None, 9, p, 1 << 20, None) == M.MOE_EINVAL
+    assert f(None, p, p, p, p, 1, 1, 2, 256, 128, 16, None, p, None, 0, p, 1 << 20, None) == M.MOE_EINVAL
+    assert f(p, p, p, p, p, 1, 1, 2, 256, 128, 16, None, p, None, 0, p, 16, None) == M.MOE_EINVAL
+    assert f(p, p, p, p, p, 1, 1, 2, 256, 128, 16, p, p, None, 0, p, 1 << 20, None) == M.MOE_EINVAL  # y_shared
+    assert _rc("moe_combine", p, p, p, None, 1, 0, 64, p, None) == M.MOE_EINVAL
+    assert _rc("moe_combine", p, p, p, None, 1, 2, 62, p, None) == M.MOE_EINVAL
+
+
+def test_expcache_rejects_bad_descriptors_on_host():
+    pool = np.zeros(4096, np.uint8)
+    d = M.ExpCacheDesc(4, 2, 256, 256, pool.ctypes.data, pool.ctypes.data, pool.ctypes.data, None, 8, 0)
+    h = C.c_void_p()
+    bad = [dict(n_experts=0), dict(capacity=0), dict(blob_bytes=100), dict(slot_stride=128),
+           dict(host_pool=None), dict(decay_period=-1), dict(use_staging=1)]
+    for b in bad:
+        dd = M.ExpCacheDesc.from_buffer_copy(d)
+        for k, v in b.items():
+            setattr(dd, k, v)
+        assert M.lib().expcache_create(C.byref(dd), C.byref(h)) == M.MOE_EINVAL, b
+    assert M.lib().expcache_stage(None, None, 0, None, None, None, None) == M.MOE_EINVAL
+
+
+def test_product_path_has_no_fallback(monkeypatch, tmp_path):
+    """Without the shared library the binding raises instead of computing elsewhere."""
+    monkeypatch.setattr(M, "_lib", None)
+    monkeypatch.setattr(M, "LIB_PATH", tmp_path / "missing.so")
+    with pytest.raises(RuntimeError, match="libmoe.so not found"):
+        M.lib()

@@ -1,0 +1,287 @@
+"""GPU parity: every kernel of the step against the fp64 oracle on the same
+seeded inputs.  Integer results (expert ids, permutation, cache events) must
+be bit-exact; floating outputs within 2e-3 x RMS of the oracle (the bar the
+task sets, with fp32 accumulation).  All calls go through the C ABI."""
+import numpy as np
+import pytest
+
+import oracle
+import workloads as W
+from tests.gpu_util import TOL, decisive_tokens, dev_x, logit_bound, rel_err, run_gpu, xd
+
+pytestmark = pytest.mark.gpu
+
+# The CUDA-core path computes sum_i (q_i - half) x_i as 128 * sum_i f_i x_i -
+# (128 + half) * sum_i x_i with f_i = 1 + q_i/128 (a float built from the code
+# bits).  The subtraction cancels the leading bits, so each 32-weight block
+# carries an absolute error of about (128 + half) * 2^-24 * sqrt(32) * |x|;
+# relative to RMS(y) that measures 1e-5 (4-bit) to 2e-4 (2-bit), ten times
+# below the acceptance bar.  GEMV_TOL bounds it.
+GEMV_TOL = 5e-4
+
+torch = pytest.importorskip("torch")
+import quantized_expert_ffn_route_b200 as M  # noqa: E402
+
+
+def _t(a, dtype=None):
+    return torch.from_numpy(np.ascontiguousarray(a if dtype is None else a.astype(dtype))).cuda()
+
+
+def _layer_gpu(layer):
+    return M.MoELayer(layer.bits, layer.H, layer.I, layer.E, layer.k, layer.blobs, layer.shared,
+                      layer.w_router, layer.w_dtype, layer.bias)
+
+
+# ------------------------------------------------------------------ top-k
+def _logits_case(seed, T, E, kind):
+    rng = np.random.default_rng(seed)
+    if kind == "gauss":
+        return rng.standard_normal((T, E)).astype(np.float32)
+    if kind == "ints":          # many exact ties
+        return rng.integers(-3, 4, size=(T, E)).astype(np.float32)
+    if kind == "special":
+        l = rng.standard_normal((T, E)).astype(np.float32)
+        l[:, ::7] = np.nan
+        l[:, 1::11] = -np.inf
+        l[:, 2::13] = 0.0
+        l[:, 3::13] = -0.0
+        return l
+    raise ValueError(kind)
+
+
+@pytest.mark.parametrize("E,k", [(16, 2), (64, 10), (512, 10), (1000, 32), (24576, 10), (3000, 1)])
+@pytest.mark.parametrize("kind", ["gauss", "ints", "special"])
+def test_topk_bit_exact(E, k, kind):
+    T = 33 if E <= 1024 else 5
+    l = _logits_case(E * 7 + k, T, E, kind)
+    ids_ref, w_ref, st = oracle.topk(l, k)
+    ids = torch.empty(T * k, dtype=torch.int32, device="cuda")
+    w = torch.empty(T * k, dtype=torch.float32, device="cuda")
+    M.moe_route_topk(None, 0, None, 0, _t(l), None, T, 0, E, k, ids, w)
+    err = M.moe_device_error(clear=True)
+    assert np.array_equal(ids.cpu().numpy().reshape(T, k), ids_ref)
+    if st == 0:
+        assert err == 0
+        assert np.allclose(w.cpu().numpy().reshape(T, k), w_ref, rtol=4e-6, atol=1e-7)
+    else:
+        assert err & M.DEVERR_NONFINITE
+
+
+def test_topk_nan_selected_sets_error():
+    l = np.full((2, 40), np.nan, np.float32)
+    l[0, 3] = 1.0
+    ids = torch.empty(8, dtype=torch.int32, device="cuda")
+    w = torch.empty(8, dtype=torch.float32, device="cuda")
+    M.moe_route_topk(None, 0, None, 0, _t(l), None, 2, 0, 40, 4, ids, w)
+    assert M.moe_device_error(clear=True) & M.DEVERR_NONFINITE
+    assert ids.cpu().numpy()[:4].tolist() == [3, 0, 1, 2]
+    assert np.all(np.isnan(w.cpu().numpy()))
+
+
+# ----------------------------------------------------------------- logits
+@pytest.mark.parametrize("dt", ["bf16", "f32"])
+def test_router_logits_within_bound(dt):
+    layer = W.make_layer(31, 4, 256, 128, 48, 4, shared=False, w_dtype=dt, sigma_r=0.1,
+                         bias=np.linspace(-0.5, 0.5, 48).astype(np.float32))
+    x = W.make_tokens(32, 21, 256, dt)
+    ref = oracle.router_logits(x, dt, layer.w_router, dt, layer.bias)
+    g = _layer_gpu(layer)
+    out = run_gpu(g, x, dt)
+    eps = logit_bound(layer, x, dt)
+    assert np.all(np.abs(out["logits"] - ref) <= eps)
+
+
+def test_router_ties_from_duplicate_rows():
+    """Duplicated router rows give bit-identical logits, so the lower id must win."""
+    layer = W.make_layer(41, 4, 256, 128, 16, 3, shared=False, w_dtype="bf16")
+    wr = layer.w_router.copy()
+    wr[9] = wr[2]
+    wr[12] = wr[5]
+    layer.w_router = wr
+    x = W.make_tokens(42, 40, 256, "bf16")
+    out = run_gpu(_layer_gpu(layer), x, "bf16")
+    l = out["logits"]
+    assert np.array_equal(l[:, 9], l[:, 2]) and np.array_equal(l[:, 12], l[:, 5])
+    for t in range(40):
+        ids = out["ids"][t].tolist()
+        assert 9 not in ids or 2 in ids
+        if 2 in ids and 9 in ids:
+            assert ids.index(2) < ids.index(9)
+
+
+# ---------------------------------------------------------------- permute
+@pytest.mark.parametrize("T,k,E", [(1, 10, 512), (37, 10, 512), (500, 10, 512), (8192, 10, 512),
+                                   (3, 10, 24576), (2000, 3, 7), (1, 1, 1), (4096, 1, 32768)])
+def test_permute_bit_exact(T, k, E):
+    rng = np.random.default_rng(T + 13 * k + E)
+    ids = np.stack([rng.choice(E, size=k, replace=False) for _ in range(T)]).astype(np.int32)
+    ref = oracle.permute(ids, E)
+    n = T * k
+    offsets = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    ps = torch.empty(n, dtype=torch.int32, device="cuda")
+    pd = torch.empty(n, dtype=torch.int32, device="cuda")
+    act = torch.empty(1 + min(n, E) + 3, dtype=torch.int32, device="cuda")
+    wsb = M.moe_permute_ws_size(T, k, E)
+    ws = torch.empty(max(16, wsb), dtype=torch.uint8, device="cuda")
+    M.moe_permute(_t(ids), T, k, E, offsets, ps, pd, act, ws, wsb)
+    assert M.moe_device_error(clear=True) == 0
+    assert np.array_equal(offsets.cpu().numpy(), ref["offsets"])
+    assert np.array_equal(ps.cpu().numpy(), ref["perm_src"])
+    assert np.array_equal(pd.cpu().numpy().reshape(T, k), ref["perm_dst"])
+    a = act.cpu().numpy()
+    assert np.array_equal(a[:1 + a[0]], ref["active"])
+
+
+def test_permute_empty_and_bad_id():
+    offsets = torch.full((17,), 7, dtype=torch.int32, device="cuda")
+    act = torch.full((4,), 7, dtype=torch.int32, device="cuda")
+    M.moe_permute(None, 0, 2, 16, offsets, None, None, act)
+    assert offsets.cpu().numpy().tolist() == [0] * 17 and act[0].item() == 0
+    ids = _t(np.array([[1, 16]], np.int32))
+    ps = torch.empty(2, dtype=torch.int32, device="cuda")
+    pd = torch.empty(2, dtype=torch.int32, device="cuda")
+    M.moe_permute(ids, 1, 2, 16, offsets, ps, pd, act)
+    assert M.moe_device_error(clear=True) & M.DEVERR_BAD_EXPERT
+
+
+# ---------------------------------------------------------------- combine
+def test_combine_against_oracle():
+    rng = np.random.default_rng(5)
+    T, k, H = 37, 10, 512
+    yp = rng.standard_normal((T * k, H)).astype(np.float32)
+    pd = rng.permutation(T * k).astype(np.int32).reshape(T, k)
+    w = rng.random((T, k)).astype(np.float32)
+    ys = rng.standard_normal((T, H)).astype(np.float32)
+    ref = oracle.combine(yp.astype(np.float64), pd, w.astype(np.float64), ys.astype(np.float64))
+    y = torch.empty(T * H, dtype=torch.float32, device="cuda")
+    M.moe_combine(_t(yp), _t(pd), _t(w), _t(ys), T, k, H, y)
+    assert rel_err(y.cpu().numpy().reshape(T, H), ref) < 1e-6
+
+
+# ------------------------------------------------------------ whole layer
+def _check_layer(out, ref, layer, x, x_dtype, tol=TOL):
+    """ids/permutation bit-exact where the routing margin is decisive; y within tol."""
+    eps = logit_bound(layer, x, x_dtype) if layer.w_router is not None else np.zeros_like(ref["logits"])
+    dec = decisive_tokens(ref["logits"], eps, layer.k)
+    assert out["err"] == 0
+    assert np.array_equal(out["ids"][dec], ref["ids"][dec])
+    if dec.all():
+        assert np.array_equal(out["offsets"], ref["offsets"])
+        assert np.array_equal(out["perm_src"], ref["perm_src"])
+        assert np.array_equal(out["perm_dst"], ref["perm_dst"])
+    e = rel_err(out["y"][dec], ref["y"][dec])
+    assert e <= tol, f"max|y - y_oracle| = {e:.3e} x RMS"
+    return e, int((~dec).sum())
+
+
+def test_layer_tiny_gemv():
+    layer, x = W.tiny_case()
+    ref = oracle.moe_layer(4, x, "f32", layer.blobs, k=2, H=256, I=128, E=16, w_router=layer.w_router,
+                           w_dtype="f32", want_yperm=True)
+    out = run_gpu(_layer_gpu(layer), x, "f32", mode=M.MOE_MODE_GEMV)
+    e, _ = _check_layer(out, ref, layer, x, "f32")
+    assert e < GEMV_TOL
+    assert rel_err(out["y_perm"], ref["y_perm"]) < GEMV_TOL
+
+
+@pytest.mark.parametrize("bits", [4, 2])
+@pytest.mark.parametrize("T", [1, 3, 16, 40])
+def test_layer_small_gemv(bits, T):
+    layer = W.make_layer(50 + bits, bits, 256, 128, 24, 4, shared=True, w_dtype="bf16")
+    x = W.make_tokens(60 + T, T, 256, "bf16")
+    ref = oracle.moe_layer(bits, x, "bf16", layer.blobs, k=4, H=256, I=128, E=24, w_router=layer.w_router,
+                           w_dtype="bf16", shared_blob=layer.shared, want_yperm=True)
+    out = run_gpu(_layer_gpu(layer), x, "bf16", mode=M.MOE_MODE_GEMV)
+    e, _ = _check_layer(out, ref, layer, x, "bf16")
+    assert e < GEMV_TOL
+    assert rel_err(out["y_shared"], ref["y_shared"]) < GEMV_TOL
+
+
+@pytest.mark.parametrize("mode", [M.MOE_MODE_GEMM, M.MOE_MODE_AUTO])
+@pytest.mark.parametrize("bits,T", [(4, 300), (2, 300), (4, 17), (4, 1000)])
+def test_layer_ragged_gemm(mode, bits, T):
+    """Several tiles per expert with ragged tails (uneven per-expert counts)."""
+    layer = W.make_layer(70 + bits, bits, 256, 256, 8, 2, shared=True, w_dtype="bf16")
+    x = W.make_tokens(71 + T, T, 256, "bf16")
+    ref = oracle.moe_layer(bits, x, "bf16", layer.blobs, k=2, H=256, I=256, E=8, w_router=layer.w_router,
+                           w_dtype="bf16", shared_blob=layer.shared)
+    out = run_gpu(_layer_gpu(layer), x, "bf16", mode=mode)
+    _check_layer(out, ref, layer, x, "bf16")
+
+
+# ------------------------------------------------------ full-size layers
+@pytest.fixture(scope="module")
+def decode_layer():
+    c = W.DECODE
+    layer = W.make_layer(W.SEED["decode"], 4, c["H"], c["I"], c["E"], c["k"], shared=True, w_dtype="bf16")
+    return layer, _layer_gpu(layer)
+
+
+def _sampled_ref(layer, x, rows):
+    return oracle.moe_layer(layer.bits, x[rows], "bf16", layer.blobs, k=layer.k, H=layer.H, I=layer.I, E=layer.E,
+                            w_router=layer.w_router, w_dtype="bf16", bias=layer.bias, shared_blob=layer.shared)
+
+
+@pytest.mark.parametrize("T", [1, 4])
+def test_decode_full_size(decode_layer, T):
+    layer, g = decode_layer
+    x = W.make_tokens(W.SEED["decode"] + 100 + T, T, layer.H, "bf16")
+    out = run_gpu(g, x, "bf16")
+    ref = _sampled_ref(layer, x, np.arange(T))
+    e, _ = _check_layer(out, ref, layer, x, "bf16")
+    assert e < GEMV_TOL
+
+
+@pytest.mark.parametrize("T", [512, 2048])
+def test_prefill_full_size_sampled(decode_layer, T):
+    """Prefill chunk in GEMM mode at full layer size; oracle on sampled tokens."""
+    layer, g = decode_layer
+    x = W.make_tokens(W.SEED["prefill"] + T, T, layer.H, "bf16")
+    out = run_gpu(g, x, "bf16", mode=M.MOE_MODE_AUTO)
+    assert out["err"] == 0
+    rows = np.unique(np.concatenate([[0, T - 1], np.random.default_rng(T).choice(T, 6, replace=False)]))
+    ref = _sampled_ref(layer, x, rows)
+    eps = logit_bound(layer, x[rows], "bf16")
+    dec = decisive_tokens(ref["logits"], eps, layer.k)
+    assert np.array_equal(out["ids"][rows][dec], ref["ids"][dec])
+    e = rel_err(out["y"][rows][dec], ref["y"][dec])
+    assert e <= TOL, e
+    # whole-chunk invariants: every row of the permutation is used once
+    assert sorted(out["perm_dst"].ravel().tolist()) == list(range(T * layer.k))
+    assert out["offsets"][-1] == T * layer.k
+
+
+@pytest.fixture(scope="module")
+def verify_layer():
+    layer = W.verify_layer()
+    return layer, _layer_gpu(layer)
+
+
+@pytest.mark.parametrize("T", [2, 3, 5, 9, 16])
+def test_verify_windows_q2(verify_layer, T):
+    layer, g = verify_layer
+    x = W.make_tokens(W.SEED["verify"] + T, T, layer.H, "bf16")
+    out = run_gpu(g, x, "bf16")
+    ref = _sampled_ref(layer, x, np.arange(T))
+    e, _ = _check_layer(out, ref, layer, x, "bf16")
+    assert e < GEMV_TOL
+    # the window gives the rows of T single-token steps (Strata article, section 2 item 3)
+    for t in range(T):
+        one = run_gpu(g, x[t:t + 1], "bf16")
+        assert np.array_equal(one["ids"][0], out["ids"][t])
+        assert rel_err(one["y"][0], out["y"][t]) < 1e-6
+
+
+def test_null_blob_sets_error(decode_layer):
+    layer, g = decode_layer
+    x = W.make_tokens(5, 1, layer.H, "bf16")
+    out = run_gpu(g, x, "bf16")
+    e = int(out["ids"][0, 0])
+    saved = g.table[e].item()
+    g.table[e] = 0
+    try:
+        out = run_gpu(g, x, "bf16")
+        assert out["err"] & M.DEVERR_NULL_BLOB
+    finally:
+        g.table[e] = saved
+    assert run_gpu(g, x, "bf16")["err"] == 0

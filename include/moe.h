@@ -168,6 +168,33 @@ int moe_expert_ffn_q2(const void *const *expert_blobs, const int32_t *expert_off
                       const void *shared_blob, float *y_perm, float *y_shared, int mode,
                       void *ws, size_t ws_bytes, moe_stream_t s);
 
+/* ------------------------------------------------- allocation-free FFN
+ * The pages have no counterpart of this call; it serves callers that cannot
+ * allocate device memory when they run the step: code running while a
+ * stream is captured into a CUDA graph (an allocation there breaks the
+ * capture), engines held to a memory budget fixed at start-up, and C hosts
+ * with no device allocator to hand out a workspace.
+ * Same computation and arguments as moe_expert_ffn_q4/q2 in MOE_MODE_GEMV
+ * (bits = 4 or 2 selects the blob format), but without ws/ws_bytes: the
+ * scratch (the fp32 intermediate h, T*(k+1)*I*4 bytes) comes from one array
+ * built into the library of moe_expert_ffn_noalloc_max_bytes() bytes (8 MiB),
+ * which every GPU that loads the library holds until the process exits.
+ *  - Calls needing more scratch than that, or H/I outside [128, 2048], are
+ *    rejected with MOE_EINVAL before anything is launched.
+ *  - It never calls cudaMalloc, cudaFree or any allocating routine.
+ *  - The first call on a device looks up the array's device address (once per
+ *    device, with that device current); make that first call before any stream
+ *    capture.  MOE_ECUDA if the lookup fails.
+ *  - All calls on a device share the one array and it keeps the last call's
+ *    contents (nothing in it needs to start at zero).  Calls whose kernels
+ *    overlap on the GPU (other streams, other threads) race on it: serialise
+ *    them. */
+size_t moe_expert_ffn_noalloc_max_bytes(void);
+int moe_expert_ffn_noalloc(int bits, const void *const *expert_blobs, const int32_t *expert_offsets,
+                           const int32_t *active, const int32_t *perm_src, const void *x, int x_dtype,
+                           int T, int k, int H, int I, int E, const void *shared_blob,
+                           float *y_perm, float *y_shared, moe_stream_t s);
+
 /* ---------------------------------------------------------------- combine
  *   y[t] = sum_{j=0}^{k-1} topk_w[t,j] * y_perm[perm_dst[t,j]] (+ y_shared[t]),
  *   summed in slot order, fp32.  y_shared may be NULL.  y device [T,H] out. */

@@ -74,6 +74,8 @@ def lib():
         "moe_expert_ffn_q4": (I, [P, P, P, P, P, I, I, I, I, I, I, P, P, P, I, P, Z, S]),
         "moe_expert_ffn_q2": (I, [P, P, P, P, P, I, I, I, I, I, I, P, P, P, I, P, Z, S]),
         "moe_combine": (I, [P, P, P, P, I, I, I, P, S]),
+        "moe_expert_ffn_noalloc_max_bytes": (Z, []),
+        "moe_expert_ffn_noalloc": (I, [I, P, P, P, P, P, I, I, I, I, I, I, P, P, P, S]),
         "expcache_create": (I, [C.POINTER(ExpCacheDesc), C.POINTER(P)]),
         "expcache_destroy": (None, [P]),
         "expcache_lookup": (I, [P, P, I, P, P]),
@@ -190,6 +192,17 @@ def moe_expert_ffn_q2(expert_blobs, expert_offsets, active, perm_src, x, x_dtype
                       y_perm, y_shared, mode=MOE_MODE_AUTO, ws=None, ws_bytes=0, stream=None):
     return _ffn("moe_expert_ffn_q2", expert_blobs, expert_offsets, active, perm_src, x, x_dtype, T, k, H, I, E,
                 shared_blob, y_perm, y_shared, mode, ws, ws_bytes, stream)
+
+
+def moe_expert_ffn_noalloc_max_bytes() -> int:
+    return lib().moe_expert_ffn_noalloc_max_bytes()
+
+
+def moe_expert_ffn_noalloc(bits, expert_blobs, expert_offsets, active, perm_src, x, x_dtype, T, k, H, I, E,
+                           shared_blob, y_perm, y_shared, stream=None):
+    return _check(lib().moe_expert_ffn_noalloc(bits, _p(expert_blobs), _p(expert_offsets), _p(active),
+                                               _p(perm_src), _p(x), x_dtype, T, k, H, I, E, _p(shared_blob),
+                                               _p(y_perm), _p(y_shared), _stream(stream)))
 
 
 def moe_combine(y_perm, perm_dst, topk_w, y_shared, T, k, H, y, stream=None):

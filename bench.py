@@ -256,8 +256,18 @@ def bench_layer(args, world, rank, pk):
             return xs[j * T:(j + 1) * T]
         return xs[i * T:(i + 1) * T]
 
+    fused = kind == "decode" and not args.unfused
+    dbuf = copies[0].decode_buffers() if fused else None
+
     def step(i, e0=None, e1=None):
         L = copies[i % n_layers]
+        if fused:                                      # the whole step in one kernel
+            if e0 is not None:
+                e0.record()
+            L.forward_decode(x_of(i), M.MOE_BF16, bufs=dbuf)
+            if e1 is not None:
+                e1.record()
+            return
         b = bufs
         x = x_of(i)
         M.moe_route_topk(x, M.MOE_BF16, L.w_router, L.w_dtype, None, L.bias, T, H, E, k, b.ids, b.w, b.logits,
@@ -274,6 +284,9 @@ def bench_layer(args, world, rank, pk):
 
     def ffn_only(i):
         L = copies[i % n_layers]
+        if fused:
+            L.forward_decode(x_of(i), M.MOE_BF16, bufs=dbuf)
+            return
         b = bufs
         ffn = M.moe_expert_ffn_q4 if bits == 4 else M.moe_expert_ffn_q2
         ffn(L.table, b.offsets, b.active, b.perm_src, x_of(i), M.MOE_BF16, T, k, H, I, E, L.shared, b.y_perm,
@@ -326,7 +339,7 @@ def bench_layer(args, world, rank, pk):
     assert M.moe_device_error() == 0
 
     # distinct experts actually touched in the last timed step (all routed + shared)
-    n_act = int(bufs.active[0].item())
+    n_act = k if fused else int(bufs.active[0].item())
     tokens_total = sum_over_ranks(args.steps * T, world)
     value = tokens_total / (ms_max / 1e3)
 
@@ -346,13 +359,17 @@ def bench_layer(args, world, rank, pk):
     else:
         # per-window distinct experts differ; average over the timed steps is not tracked on device,
         # so credit the experts of the last window (decode: always k routed + 1 shared)
-        bytes_ffn = (n_act + 1) * blob + T * H * 2 + T * (k + 1) * H * 4
+        if fused:   # one kernel: router rows + k routed + shared expert blobs + x + logits + y
+            bytes_ffn = (k + 1) * blob + E * H * 2 + H * 2 + E * 4 + H * 4
+        else:
+            bytes_ffn = (n_act + 1) * blob + T * H * 2 + T * (k + 1) * H * 4
         gbs = bytes_ffn / (ffn_avg_ms / 1e3) / 1e9
         roof = {"bound": "hbm", "achieved": round(gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
                 "frac": round(gbs / pk["hbm_gbs"], 4)}
-    sha = src_hash("gemv.cu") if kind != "prefill" else src_hash("gemm_tc.cu")
-    roof["traffic"] = traffic_from_profiles(f"expert_ffn_{kind}", sha)
-    roof["kernel"] = "moe_expert_ffn (gate/up + down kernels)"
+    sha = src_hash("decode.cu" if fused else ("gemv.cu" if kind != "prefill" else "gemm_tc.cu"))
+    roof["traffic"] = traffic_from_profiles("k_decode" if fused else f"expert_ffn_{kind}", sha)
+    roof["kernel"] = ("k_decode (moe_layer_decode: route + top-k + experts + combine, one launch)" if fused
+                      else "moe_expert_ffn (gate/up + down kernels)")
     roof["ms_per_launch"] = round(ffn_avg_ms, 5)
     roof["timing"] = ffn_timing
     roof["algorithmic_bytes_per_launch"] = int(bytes_ffn)
@@ -369,8 +386,12 @@ def bench_layer(args, world, rank, pk):
         s = torch.cuda.current_stream()
         for i in range(3):
             xd.copy_(xh[:T], non_blocking=True)
-            copies[i % n_layers].forward(xd, M.MOE_BF16, T=T, mode=mode, bufs=bufs)
-            yh.copy_(bufs.y[:T * H], non_blocking=True)
+            if fused:
+                copies[i % n_layers].forward_decode(xd, M.MOE_BF16, bufs=dbuf)
+                yh.copy_(dbuf["y"][:H], non_blocking=True)
+            else:
+                copies[i % n_layers].forward(xd, M.MOE_BF16, T=T, mode=mode, bufs=bufs)
+                yh.copy_(bufs.y[:T * H], non_blocking=True)
             s.synchronize()
         barrier(world)
         a, b2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -378,15 +399,20 @@ def bench_layer(args, world, rank, pk):
         for i in range(n_e2e):
             j = i * T if kind != "prefill" else 0
             xd.copy_(xh[j:j + T], non_blocking=True)
-            copies[i % n_layers].forward(xd, M.MOE_BF16, T=T, mode=mode, bufs=bufs)
-            yh.copy_(bufs.y[:T * H], non_blocking=True)
+            if fused:
+                copies[i % n_layers].forward_decode(xd, M.MOE_BF16, bufs=dbuf)
+                yh.copy_(dbuf["y"][:H], non_blocking=True)
+            else:
+                copies[i % n_layers].forward(xd, M.MOE_BF16, T=T, mode=mode, bufs=bufs)
+                yh.copy_(bufs.y[:T * H], non_blocking=True)
             s.synchronize()
         b2.record()
         torch.cuda.synchronize()
         e_ms = max_over_ranks(a.elapsed_time(b2), world)
         e2e = {"value": round(sum_over_ranks(n_e2e * T, world) / (e_ms / 1e3), 1), "unit": "tokens/s",
                "h2d_bytes_per_step": T * H * 2, "d2h_bytes_per_step": T * H * 4, "steps": n_e2e,
-               "note": "MoELayer.forward via the C ABI; pinned host x in, fp32 y out, stream sync every step"}
+               "note": ("MoELayer.forward_decode" if fused else "MoELayer.forward") +
+                       " via the C ABI; pinned host x in, fp32 y out, stream sync every step"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -400,7 +426,8 @@ def bench_layer(args, world, rank, pk):
                        f"{bits}-bit blocks of 32 + fp16 scale, {T} token(s)/step",
            "tokens_per_step": T, "layer_copies": n_layers,
            "l2": f"inputs larger than L2: {n_layers} layer copies x {E + 1} experts x {blob} B rotate per step",
-           "mode": {0: "auto", 1: "gemv", 2: "gemm"}[mode], "parallelism": f"replicas x{world}"}
+           "mode": "fused decode kernel" if fused else {0: "auto", 1: "gemv", 2: "gemm"}[mode],
+           "parallelism": f"replicas x{world}"}
     return dict(value=value, ms=ms_max, steps=args.steps, roofline=roof, e2e=e2e, cpu=cpu, clocks=clk,
                 launches=launches, config=cfg, dtype="fp32 (CUDA-core FMA on 4-bit codes)" if kind == "decode"
                 else ("fp32 (CUDA-core FMA on 2-bit codes)" if kind == "verify" else "fp16 tensor cores, fp32 accum"))
@@ -582,6 +609,7 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=500)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--unfused", action="store_true", help="decode through the four separate calls")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:

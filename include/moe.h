@@ -77,6 +77,7 @@ typedef struct CUstream_st *moe_stream_t;   /* same type as cudaStream_t */
 #define MOE_DEVERR_NULL_BLOB 2u      /* an active expert had no blob pointer */
 #define MOE_DEVERR_NONFINITE 4u      /* a selected logit was NaN or +inf */
 #define MOE_DEVERR_BAD_ROW 8u        /* offsets/perm_src inconsistent */
+#define MOE_DEVERR_TIMEOUT 16u       /* a bounded in-kernel wait ran out */
 
 /* Thread-local message of the last failing call ("" if none). */
 const char *moe_last_error(void);
@@ -167,6 +168,31 @@ int moe_expert_ffn_q2(const void *const *expert_blobs, const int32_t *expert_off
                       int x_dtype, int T, int k, int H, int I, int E,
                       const void *shared_blob, float *y_perm, float *y_shared, int mode,
                       void *ws, size_t ws_bytes, moe_stream_t s);
+
+/* ------------------------------------------------------- fused decode step
+ * The whole step for ONE token: router logits (or logits_in), top-k + gates,
+ * the k routed experts and the shared expert, and the combine
+ *   y = sum_{j<k} w_j * FFN_{ids_j}(x) + FFN_shared(x)    (fp32, slot order),
+ * with the same definitions as moe_route_topk -> moe_permute ->
+ * moe_expert_ffn_q4/q2 (GEMV mode) -> moe_combine (Strata article, section 2
+ * item 2: only the experts the router picks are computed; at one token the
+ * step is bound by streaming those experts' weights).  Three kernels chained
+ * with programmatic dependent launch (route in one thread-block cluster, then
+ * gate/up, then down + combine); no in-kernel waits spin.
+ *  x [H] (x_dtype), w_router [E,H] (w_dtype) or NULL with logits_in [E];
+ *  expert_blobs device [E] blob pointers; shared_blob or NULL;
+ *  topk_ids [k] int32 out, topk_w [k] fp32 out, logits_out [E] or NULL
+ *  (written only when the logits are computed here), y [H] fp32 out.
+ *  ws: moe_layer_decode_ws_size() bytes of scratch (no initialisation needed).
+ * Supported shapes (else MOE_EINVAL: use the separate calls): E <= 1024,
+ * k <= 32, H <= 2048, I a multiple of 128 with I/32 (4-bit) or I/64 (2-bit)
+ * a power of two <= 32, and k + 1 <= 8 * 32 / (that number). */
+size_t moe_layer_decode_ws_size(int E, int k, int I);
+int moe_layer_decode(int bits, const void *x, int x_dtype, const void *w_router, int w_dtype,
+                     const float *bias, const float *logits_in, const void *const *expert_blobs,
+                     const void *shared_blob, int H, int I, int E, int k, int32_t *topk_ids,
+                     float *topk_w, float *logits_out, float *y, void *ws, size_t ws_bytes,
+                     moe_stream_t s);
 
 /* ------------------------------------------------- allocation-free FFN
  * The pages have no counterpart of this call; it serves callers that cannot

@@ -74,6 +74,8 @@ def lib():
         "moe_expert_ffn_q4": (I, [P, P, P, P, P, I, I, I, I, I, I, P, P, P, I, P, Z, S]),
         "moe_expert_ffn_q2": (I, [P, P, P, P, P, I, I, I, I, I, I, P, P, P, I, P, Z, S]),
         "moe_combine": (I, [P, P, P, P, I, I, I, P, S]),
+        "moe_layer_decode_ws_size": (Z, [I, I, I]),
+        "moe_layer_decode": (I, [I, P, I, P, I, P, P, P, P, I, I, I, I, P, P, P, P, P, Z, S]),
         "moe_expert_ffn_noalloc_max_bytes": (Z, []),
         "moe_expert_ffn_noalloc": (I, [I, P, P, P, P, P, I, I, I, I, I, I, P, P, P, S]),
         "expcache_create": (I, [C.POINTER(ExpCacheDesc), C.POINTER(P)]),
@@ -192,6 +194,17 @@ def moe_expert_ffn_q2(expert_blobs, expert_offsets, active, perm_src, x, x_dtype
                       y_perm, y_shared, mode=MOE_MODE_AUTO, ws=None, ws_bytes=0, stream=None):
     return _ffn("moe_expert_ffn_q2", expert_blobs, expert_offsets, active, perm_src, x, x_dtype, T, k, H, I, E,
                 shared_blob, y_perm, y_shared, mode, ws, ws_bytes, stream)
+
+
+def moe_layer_decode_ws_size(E, k, I):
+    return lib().moe_layer_decode_ws_size(E, k, I)
+
+
+def moe_layer_decode(bits, x, x_dtype, w_router, w_dtype, bias, logits_in, expert_blobs, shared_blob, H, I, E, k,
+                     topk_ids, topk_w, logits_out, y, ws, ws_bytes, stream=None):
+    return _check(lib().moe_layer_decode(bits, _p(x), x_dtype, _p(w_router), w_dtype, _p(bias), _p(logits_in),
+                                         _p(expert_blobs), _p(shared_blob), H, I, E, k, _p(topk_ids), _p(topk_w),
+                                         _p(logits_out), _p(y), _p(ws), ws_bytes, _stream(stream)))
 
 
 def moe_expert_ffn_noalloc_max_bytes() -> int:

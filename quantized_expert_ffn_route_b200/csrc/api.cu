@@ -230,6 +230,8 @@ static int expert_ffn(int bits, const void *const *expert_blobs, const int32_t *
     mode = resolve_mode(mode, T);
     if (mode == MOE_MODE_GEMV) {
         REQUIRE(H <= 2048 && I <= 2048, "GEMV mode supports H, I <= 2048 (got H=%d, I=%d)", H, I);
+    } else {
+        REQUIRE(gemm_supported(T, k, E), "GEMM mode supports at most 2047 active experts (min(E, T*k))");
     }
     const size_t need = moe_expert_ffn_ws_size(bits, T, k, H, I, E, mode);
     REQUIRE(ws && ws_bytes >= need && aligned16(ws), "workspace too small: need %zu bytes", need);
@@ -259,6 +261,41 @@ int moe_expert_ffn_q2(const void *const *expert_blobs, const int32_t *expert_off
                       moe_stream_t s) {
     return expert_ffn(2, expert_blobs, expert_offsets, active, perm_src, x, x_dtype, T, k, H, I, E, shared_blob,
                       y_perm, y_shared, mode, ws, ws_bytes, s);
+}
+
+// ------------------------------------------------------- fused decode step
+size_t moe_layer_decode_ws_size(int E, int k, int I) {
+    if (E <= 0 || k <= 0 || I <= 0) return 0;
+    return decode_ws_bytes(E, k, I);
+}
+
+int moe_layer_decode(int bits, const void *x, int x_dtype, const void *w_router, int w_dtype, const float *bias,
+                     const float *logits_in, const void *const *expert_blobs, const void *shared_blob, int H, int I,
+                     int E, int k, int32_t *topk_ids, float *topk_w, float *logits_out, float *y, void *ws,
+                     size_t ws_bytes, moe_stream_t s) {
+    t_err.clear();
+    REQUIRE(bits == 4 || bits == 2, "bits must be 4 or 2 (got %d)", bits);
+    REQUIRE(E >= 1 && k >= 1 && k <= E, "need 1 <= k <= E (got k=%d, E=%d)", k, E);
+    REQUIRE(H >= 128 && H % 128 == 0 && I >= 128 && I % 128 == 0, "H and I must be multiples of 128");
+    REQUIRE(decode_supported(bits, H, I, E, k),
+            "fused decode supports E <= 1024, k <= 32, H, I <= 2048, I %% 256 == 0 (got H=%d I=%d E=%d k=%d)", H, I,
+            E, k);
+    REQUIRE(check_dtype(x_dtype), "x_dtype must be MOE_F32 or MOE_BF16");
+    REQUIRE(x && expert_blobs && topk_ids && topk_w && y, "x/expert_blobs/topk_ids/topk_w/y must not be NULL");
+    REQUIRE(w_router || logits_in, "w_router and logits_in are both NULL");
+    REQUIRE(!w_router || check_dtype(w_dtype), "w_dtype must be MOE_F32 or MOE_BF16");
+    REQUIRE(aligned16(x) && aligned16(y) && aligned16(expert_blobs) && (!w_router || aligned16(w_router)) &&
+                (!logits_in || aligned16(logits_in)) && (!logits_out || aligned16(logits_out)) &&
+                (!shared_blob || aligned16(shared_blob)),
+            "x/y/expert_blobs/w_router/logits/shared_blob must be 16-byte aligned");
+    REQUIRE(ws && ws_bytes >= decode_ws_bytes(E, k, I) && aligned16(ws), "workspace too small: need %zu bytes",
+            decode_ws_bytes(E, k, I));
+    unsigned *err = device_error_word();
+    if (!err) return cuda_status(cudaErrorInvalidDevice, "device error word");
+    return launch_decode(bits, x, x_dtype, w_router, w_dtype, bias, logits_in,
+                         reinterpret_cast<const uint8_t *const *>(expert_blobs),
+                         static_cast<const uint8_t *>(shared_blob), H, I, E, k, topk_ids, topk_w, logits_out, y, ws,
+                         err, reinterpret_cast<cudaStream_t>(s));
 }
 
 // ---------------------------------------------------------------- combine

@@ -21,9 +21,17 @@ int launch_gemv(int bits, const uint8_t *const *blobs, const int32_t *offsets, c
                 const uint8_t *shared_blob, float *y_perm, float *y_shared, void *ws, unsigned *err, cudaStream_t s);
 
 size_t gemm_ws_bytes(int bits, int T, int k, int H, int I, int E);
+bool gemm_supported(int T, int k, int E);
 int launch_gemm(int bits, const uint8_t *const *blobs, const int32_t *offsets, const int32_t *active,
                 const int32_t *perm_src, const void *x, int x_dtype, int T, int k, int H, int I, int E,
                 const uint8_t *shared_blob, float *y_perm, float *y_shared, void *ws, unsigned *err, cudaStream_t s);
+
+size_t decode_ws_bytes(int E, int k, int I);
+bool decode_supported(int bits, int H, int I, int E, int k);
+int launch_decode(int bits, const void *x, int x_dtype, const void *w_router, int w_dtype, const float *bias,
+                  const float *logits_in, const uint8_t *const *blobs, const uint8_t *shared, int H, int I, int E,
+                  int k, int32_t *ids, float *w, float *logits_out, float *y, void *ws, unsigned *err,
+                  cudaStream_t s);
 
 int launch_combine(const float *y_perm, const int32_t *perm_dst, const float *w, const float *y_shared, int T, int k,
                    int H, float *y, unsigned *err, cudaStream_t s);

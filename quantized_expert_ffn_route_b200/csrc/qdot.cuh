@@ -1,0 +1,148 @@
+// Packed-code dot products shared by the CUDA-core expert kernels.
+//
+// Dequantisation without int->float conversions: a byte 0x80|q placed in bits
+// 16..23 of 0x3F000000 is the float 1 + q/128, so
+//   sum_i (q_i - half) x_i = 128 * sum_i f_i x_i - (128 + half) * sum_i x_i,
+// where the per-block activation sums are computed once per token when the
+// activations are staged in shared memory.  All arithmetic is fp32.
+#pragma once
+
+#include "common.cuh"
+
+namespace moe {
+
+template <int BITS> struct QT;
+template <> struct QT<4> {
+    static constexpr int EPC = 32;    // elements per 16-byte code chunk
+    static constexpr int BPC = 1;     // quant blocks (scales) per chunk
+    static constexpr int PPC = 8;     // float4 pieces per chunk
+    static constexpr int HALF = 8;
+};
+template <> struct QT<2> {
+    static constexpr int EPC = 64;
+    static constexpr int BPC = 2;
+    static constexpr int PPC = 16;
+    static constexpr int HALF = 2;
+};
+
+__device__ __forceinline__ float magic(uint32_t bytes, int b) {
+    // bytes hold 0x80|q in every byte; select byte b into bits 16..23 of 0x3F000000
+    return __uint_as_float(__byte_perm(bytes, 0x3F000000u, 0x7054u | (static_cast<unsigned>(b) << 8)));
+}
+
+__device__ __forceinline__ uint4 ldg_stream(const void *p) {
+    uint4 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p));
+    return r;
+}
+
+// Accumulates one 16-byte code chunk against NT staged activation rows.
+// xs: float4 [NT][PPC][nch]; cs: float [NT][nch*BPC] (pre-scaled block sums).
+template <int BITS, int NT>
+__device__ __forceinline__ void chunk_dot(const uint4 &code, const float (&d)[QT<BITS>::BPC], const float4 *xs,
+                                          const float *cs, int nch, int c, float (&dot)[NT]) {
+    using Q = QT<BITS>;
+    float A[NT][2];
+#pragma unroll
+    for (int t = 0; t < NT; ++t) A[t][0] = A[t][1] = 0.f;
+    const uint32_t words[4] = {code.x, code.y, code.z, code.w};
+    if constexpr (BITS == 4) {
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            const uint32_t L = (words[m] & 0x0F0F0F0Fu) | 0x80808080u;
+            const uint32_t Hh = ((words[m] >> 4) & 0x0F0F0F0Fu) | 0x80808080u;
+            const float l0 = magic(L, 0), l1 = magic(L, 1), l2 = magic(L, 2), l3 = magic(L, 3);
+            const float h0 = magic(Hh, 0), h1 = magic(Hh, 1), h2 = magic(Hh, 2), h3 = magic(Hh, 3);
+#pragma unroll
+            for (int t = 0; t < NT; ++t) {
+                const float4 a = xs[(t * Q::PPC + m) * nch + c];
+                const float4 b = xs[(t * Q::PPC + 4 + m) * nch + c];
+                float s0 = A[t][0], s1 = A[t][1];
+                s0 = fmaf(l0, a.x, s0); s1 = fmaf(h0, b.x, s1);
+                s0 = fmaf(l1, a.y, s0); s1 = fmaf(h1, b.y, s1);
+                s0 = fmaf(l2, a.z, s0); s1 = fmaf(h2, b.z, s1);
+                s0 = fmaf(l3, a.w, s0); s1 = fmaf(h3, b.w, s1);
+                A[t][0] = s0; A[t][1] = s1;
+            }
+        }
+#pragma unroll
+        for (int t = 0; t < NT; ++t)
+            dot[t] = fmaf(d[0], fmaf(128.f, A[t][0] + A[t][1], -cs[t * nch + c]), dot[t]);
+    } else {
+#pragma unroll
+        for (int wi = 0; wi < 4; ++wi) {
+            const int beta = wi >> 1, m = wi & 1;
+#pragma unroll
+            for (int s = 0; s < 4; ++s) {
+                const uint32_t Ls = ((words[wi] >> (2 * s)) & 0x03030303u) | 0x80808080u;
+                const float f0 = magic(Ls, 0), f1 = magic(Ls, 1), f2 = magic(Ls, 2), f3 = magic(Ls, 3);
+                const int piece = 8 * beta + 2 * s + m;
+#pragma unroll
+                for (int t = 0; t < NT; ++t) {
+                    const float4 a = xs[(t * Q::PPC + piece) * nch + c];
+                    float v = A[t][beta];
+                    v = fmaf(f0, a.x, v); v = fmaf(f1, a.y, v); v = fmaf(f2, a.z, v); v = fmaf(f3, a.w, v);
+                    A[t][beta] = v;
+                }
+            }
+        }
+#pragma unroll
+        for (int t = 0; t < NT; ++t) {
+            float r = dot[t];
+            r = fmaf(d[0], fmaf(128.f, A[t][0], -cs[(t * nch + c) * 2 + 0]), r);
+            r = fmaf(d[1], fmaf(128.f, A[t][1], -cs[(t * nch + c) * 2 + 1]), r);
+            dot[t] = r;
+        }
+    }
+}
+
+template <int BITS>
+__device__ __forceinline__ void load_scales(const __half *row_scales, int c, bool valid, float (&d)[QT<BITS>::BPC]) {
+    if constexpr (BITS == 4) {
+        d[0] = valid ? __half2float(row_scales[c]) : 0.f;
+    } else {
+        if (valid) {
+            const __half2 s2 = *reinterpret_cast<const __half2 *>(row_scales + 2 * c);
+            d[0] = __low2float(s2);
+            d[1] = __high2float(s2);
+        } else {
+            d[0] = d[1] = 0.f;
+        }
+    }
+}
+
+// Stages nt activation rows (fp32 or bf16, rows[t] -> row t) as fp32 pieces
+// plus the pre-scaled block sums; rows nt..NTS-1 are zero.
+template <int BITS>
+__device__ void stage_rows(float4 *xs, float *cs, int NTS, int nt, int K, const void *const *rows, int bf16) {
+    using Q = QT<BITS>;
+    const int nch = K / Q::EPC;
+    const int g4n = K / 4;
+    for (int idx = threadIdx.x; idx < NTS * g4n; idx += blockDim.x) {
+        const int t = idx / g4n, g4 = idx % g4n;
+        const int c = (4 * g4) / Q::EPC, q = ((4 * g4) % Q::EPC) / 4;
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (t < nt)
+            v = bf16 ? load4(static_cast<const __nv_bfloat16 *>(rows[t]) + 4 * g4)
+                     : load4(static_cast<const float *>(rows[t]) + 4 * g4);
+        xs[(t * Q::PPC + q) * nch + c] = v;
+    }
+    __syncthreads();
+    const int nblk = K / 32;
+    for (int idx = threadIdx.x; idx < NTS * nblk; idx += blockDim.x) {
+        const int t = idx / nblk, b = idx % nblk;
+        const int c = b / Q::BPC, beta = b % Q::BPC;
+        float s = 0.f;
+#pragma unroll
+        for (int p = 0; p < 8; ++p) {
+            const float4 v = xs[(t * Q::PPC + 8 * beta + p) * nch + c];
+            s += v.x; s += v.y; s += v.z; s += v.w;
+        }
+        cs[t * nblk + b] = static_cast<float>(128 + Q::HALF) * s;
+    }
+    __syncthreads();
+}
+
+}  // namespace moe

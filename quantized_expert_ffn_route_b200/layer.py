@@ -123,6 +123,30 @@ class MoELayer:
                                                  self.shared is not None)
         return self._bufs[key]
 
+    def decode_buffers(self):
+        """Buffers of the fused one-token step (the workspace starts zeroed, as it must)."""
+        import torch
+        from . import moe_layer_decode_ws_size
+        if "decode" not in self._bufs:
+            n = moe_layer_decode_ws_size(self.E, self.k, self.I)
+            d = self.device
+            self._bufs["decode"] = dict(
+                ws=torch.zeros(n, dtype=torch.uint8, device=d), ws_bytes=n,
+                ids=torch.empty(_round_up(self.k, 4), dtype=torch.int32, device=d),
+                w=torch.empty(_round_up(self.k, 4), dtype=torch.float32, device=d),
+                logits=torch.empty(self.E, dtype=torch.float32, device=d),
+                y=torch.empty(self.H, dtype=torch.float32, device=d))
+        return self._bufs["decode"]
+
+    def forward_decode(self, x, x_dtype, logits_in=None, stream=None, bufs=None):
+        """One token [1, H] through the fused decode step; returns the buffer dict (y in ["y"])."""
+        from . import moe_layer_decode
+        b = bufs or self.decode_buffers()
+        moe_layer_decode(self.bits, x, x_dtype, None if logits_in is not None else self.w_router, self.w_dtype,
+                         self.bias, logits_in, self.table, self.shared, self.H, self.I, self.E, self.k, b["ids"],
+                         b["w"], b["logits"], b["y"], b["ws"], b["ws_bytes"], stream)
+        return b
+
     def forward(self, x, x_dtype, T=None, mode=0, logits_in=None, stream=None, bufs=None):
         """x: device tensor [T, H] (float32 or bfloat16); returns the StepBuffers (y in bufs.y)."""
         from . import moe_combine, moe_expert_ffn_q2, moe_expert_ffn_q4, moe_permute, moe_route_topk

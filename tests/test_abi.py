@@ -103,3 +103,20 @@ def test_product_path_has_no_fallback(monkeypatch, tmp_path):
     monkeypatch.setattr(M, "LIB_PATH", tmp_path / "missing.so")
     with pytest.raises(RuntimeError, match="libmoe.so not found"):
         M.lib()
+
+
+def test_fused_decode_shape_checks_on_host():
+    """Supported shapes pass host validation (they fail later only for lack of a GPU here)."""
+    buf = np.zeros(4096, np.float32)
+    p = buf.ctypes.data
+    L = M.lib()
+    for bits, H, I, E, k in [(4, 2048, 512, 512, 10), (2, 2048, 512, 512, 10), (4, 256, 256, 24, 4)]:
+        rc = L.moe_layer_decode(bits, p, M.MOE_BF16, p, M.MOE_BF16, None, None, p, p, H, I, E, k, p, p, None, p,
+                                p, M.moe_layer_decode_ws_size(E, k, I), None)
+        assert rc != M.MOE_EINVAL, M.moe_last_error()
+    # I/32 = 64 chunks per row (more than one per lane), H > 2048, E > 1024, too many groups
+    for bits, H, I, E, k in [(4, 2048, 2048, 512, 10), (4, 4096, 512, 512, 10), (4, 2048, 512, 2048, 10),
+                             (4, 2048, 1024, 512, 32)]:
+        rc = L.moe_layer_decode(bits, p, M.MOE_BF16, p, M.MOE_BF16, None, None, p, p, H, I, E, k, p, p, None, p,
+                                p, M.moe_layer_decode_ws_size(E, k, I), None)
+        assert rc == M.MOE_EINVAL

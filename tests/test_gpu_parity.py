@@ -285,3 +285,80 @@ def test_null_blob_sets_error(decode_layer):
     finally:
         g.table[e] = saved
     assert run_gpu(g, x, "bf16")["err"] == 0
+
+
+# ------------------------------------------------------ fused decode step
+def _run_fused(g, x, x_dtype, logits_in=None):
+    import quantized_expert_ffn_route_b200 as MM
+    xdev = dev_x(x, x_dtype)
+    li = None if logits_in is None else torch.from_numpy(np.ascontiguousarray(logits_in, np.float32)).cuda()
+    b = g.forward_decode(xdev, MM.MOE_BF16 if x_dtype == "bf16" else MM.MOE_F32, logits_in=li)
+    torch.cuda.synchronize()
+    return dict(err=MM.moe_device_error(clear=True), ids=b["ids"][:g.k].cpu().numpy(),
+                w=b["w"][:g.k].cpu().numpy(), logits=b["logits"].cpu().numpy(), y=b["y"].cpu().numpy())
+
+
+def test_fused_decode_full_size(decode_layer):
+    layer, g = decode_layer
+    x = W.make_tokens(W.SEED["decode"] + 500, 6, layer.H, "bf16")
+    ref = _sampled_ref(layer, x, np.arange(6))
+    eps = logit_bound(layer, x, "bf16")
+    dec = decisive_tokens(ref["logits"], eps, layer.k)
+    for t in range(6):
+        f = _run_fused(g, x[t:t + 1], "bf16")
+        assert f["err"] == 0
+        assert np.all(np.abs(f["logits"] - ref["logits"][t]) <= eps[t])
+        if dec[t]:
+            assert np.array_equal(f["ids"], ref["ids"][t])
+            assert rel_err(f["y"], ref["y"][t]) < GEMV_TOL
+        # same routing and outputs as the separate calls
+        m = run_gpu(g, x[t:t + 1], "bf16", mode=M.MOE_MODE_GEMV)
+        assert np.array_equal(f["ids"], m["ids"][0])
+        assert np.allclose(f["w"], m["w"][0], rtol=1e-6, atol=1e-7)
+        assert rel_err(f["y"], m["y"][0]) < 1e-5
+
+
+def test_fused_decode_q2_bias(verify_layer):
+    layer, g = verify_layer
+    x = W.make_tokens(W.SEED["verify"] + 900, 3, layer.H, "bf16")
+    ref = _sampled_ref(layer, x, np.arange(3))
+    eps = logit_bound(layer, x, "bf16")
+    dec = decisive_tokens(ref["logits"], eps, layer.k)
+    for t in range(3):
+        f = _run_fused(g, x[t:t + 1], "bf16")
+        assert f["err"] == 0
+        if dec[t]:
+            assert np.array_equal(f["ids"], ref["ids"][t])
+            assert rel_err(f["y"], ref["y"][t]) < GEMV_TOL
+
+
+@pytest.mark.parametrize("bits,dt,shared", [(4, "f32", False), (2, "bf16", True), (4, "bf16", True)])
+def test_fused_decode_small(bits, dt, shared):
+    layer = W.make_layer(400 + bits, bits, 256, 256, 24, 4, shared=shared, w_dtype=dt)
+    x = W.make_tokens(401 + bits, 3, 256, dt)
+    ref = oracle.moe_layer(bits, x, dt, layer.blobs, k=4, H=256, I=256, E=24, w_router=layer.w_router,
+                           w_dtype=dt, shared_blob=layer.shared)
+    g = _layer_gpu(layer)
+    eps = logit_bound(layer, x, dt)
+    dec = decisive_tokens(ref["logits"], eps, 4)
+    for t in range(3):
+        f = _run_fused(g, x[t:t + 1], dt)
+        assert f["err"] == 0
+        if dec[t]:
+            assert np.array_equal(f["ids"], ref["ids"][t])
+            assert rel_err(f["y"], ref["y"][t]) < GEMV_TOL
+
+
+def test_fused_decode_logits_in():
+    """Router logits given directly (the paging path), with exact ties."""
+    layer = W.make_layer(410, 2, 256, 256, 64, 6, shared=False, w_dtype="bf16")
+    x = W.make_tokens(411, 2, 256, "bf16")
+    rng = np.random.default_rng(412)
+    li = rng.integers(-2, 3, size=(2, 64)).astype(np.float32)
+    ref = oracle.moe_layer(2, x, "bf16", layer.blobs, k=6, H=256, I=256, E=64, logits_in=li)
+    g = _layer_gpu(layer)
+    for t in range(2):
+        f = _run_fused(g, x[t:t + 1], "bf16", logits_in=li[t:t + 1])
+        assert f["err"] == 0
+        assert np.array_equal(f["ids"], ref["ids"][t])
+        assert rel_err(f["y"], ref["y"][t]) < GEMV_TOL

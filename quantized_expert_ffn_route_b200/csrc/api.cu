@@ -26,6 +26,7 @@ void set_error(const char *fmt, ...) {
 int cuda_status(cudaError_t e, const char *what) {
     if (e == cudaSuccess) return MOE_OK;
     set_error("%s: %s", what, cudaGetErrorString(e));
+    (void)cudaGetLastError();   // a non-sticky error is reported here, not to the caller's next CUDA call
     return MOE_ECUDA;
 }
 

@@ -2,14 +2,14 @@
 // programmatic dependent launch (each starts while its predecessor runs and
 // waits with griddepcontrol only where it reads the predecessor's results).
 //
-//   1. route  (one cluster of up to 16 CTAs): router logits, rows split over
-//      the cluster and gathered through distributed shared memory; top-k and
-//      gates by one warp.
-//   2. gate/up (all selected experts + the shared expert, one warp per row
-//      pair): h_g[i] = silu(Wg_g[i] . x) * (Wu_g[i] . x).  The shared expert's
-//      CTAs do not wait for the route kernel at all.
-//   3. down + combine (one warp per output row, all groups): the codes of the
-//      row are loaded before h is staged, then
+//   1. logits (one warp per router row, spread over E/4 SMs).
+//   2. gate/up (all selected experts + the shared expert, 16 rows per CTA):
+//      every routed CTA selects the top-k from the logits itself (a block
+//      top-k of a few hundred cycles, cheaper than another kernel boundary),
+//      then h_g[i] = silu(Wg_g[i] . x) * (Wu_g[i] . x); CTA 0 publishes ids
+//      and gates.  The shared expert's CTAs never wait for the logits.
+//   3. down + combine (a few output rows per CTA, all groups; each lane one
+//      chunk of one row): every code load is issued before h is staged, then
 //      y[r] = sum_j w_j (Wd_{e_j}[r] . h_j) + Wd_shared[r] . h_shared, summed
 //      in slot order.
 // At one token the step streams ~20 MB of expert weights with little
@@ -18,14 +18,10 @@
 //
 // Strata article, section 2 item 2: the router's choice decides which
 // experts are computed; only those experts' weights are streamed.
-#include <cooperative_groups.h>
-
 #include "common.cuh"
 #include "kernels.h"
 #include "qdot.cuh"
 #include "topk.cuh"
-
-namespace cg = cooperative_groups;
 
 namespace moe {
 
@@ -54,45 +50,6 @@ __host__ __device__ inline DecodeWs decode_ws(void *ws, int E) {
     return w;
 }
 
-// Top-k of E <= 1024 values in shared memory by one warp (lane l owns experts
-// l, l + 32, ...) with single-instruction warp maxima: first the 32-bit value
-// key, then, among lanes holding that key, the lowest id.  Lane j < k ends
-// with slot j's (value, id).
-__device__ __forceinline__ void warp_topk_smem(const float *vals, int E, int k, int lane, float &my_v, int &my_id) {
-    const int npl = (E - lane + 31) / 32;
-    uint32_t taken = 0u;
-    uint32_t bv = 0u;
-    int bi = -1;
-    auto best = [&]() {
-        bv = 0u;
-        bi = -1;
-        for (int i = 0; i < npl; ++i) {
-            if (taken & (1u << i)) continue;
-            const uint32_t key = float_key(vals[lane + 32 * i]);
-            if (bi < 0 || key > bv) {                   // equal keys keep the lower id (smaller i)
-                bv = key;
-                bi = lane + 32 * i;
-            }
-        }
-    };
-    best();
-    for (int j = 0; j < k; ++j) {
-        // keys are shifted by one so that "no candidate" (0) ranks below every real key
-        const uint32_t hi = __reduce_max_sync(0xffffffffu, bi >= 0 ? bv + 1u : 0u);
-        const unsigned lo_in = (bi >= 0 && bv + 1u == hi) ? 0xffffffffu - static_cast<unsigned>(bi) : 0u;
-        const unsigned lo = __reduce_max_sync(0xffffffffu, lo_in);
-        const int id = static_cast<int>(0xffffffffu - lo);
-        if (lane == j) {
-            my_v = key_float(hi - 1u);
-            my_id = id;
-        }
-        if (bi == id) {                                   // the winner retires its candidate
-            taken |= 1u << ((id - lane) / 32);
-            best();
-        }
-    }
-}
-
 struct DecodeArgs {
     int H, I, E, k;
     const void *x;
@@ -111,103 +68,126 @@ struct DecodeArgs {
     unsigned *err;
 };
 
-// ------------------------------------------------------------ 1. route
-// One cluster; CTA rank r computes logit rows [r*er, (r+1)*er) for the single
-// token, rank 0 gathers them and selects.  (With logits_in, rank 0 selects
-// directly.)  Dynamic smem: x natural [H] + this CTA's logits [er] + all [E].
-__global__ void __launch_bounds__(kDecThreads) k_dec_route(DecodeArgs a) {
-    cg::cluster_group cluster = cg::this_cluster();
-    extern __shared__ __align__(16) float rsm[];
+// ------------------------------------------------------------ 1. logits
+// One warp per router row, kLogitRows rows per CTA, so the E rows are read by
+// E / kLogitRows SMs at once; every lane issues all of its weight loads
+// before it stages x.
+constexpr int kLogitRows = 4;
+
+__global__ void __launch_bounds__(kLogitRows * 32) k_dec_logits(DecodeArgs a) {
+    __shared__ __align__(16) float xs[2048];
     pdl_trigger();                                       // the gate/up kernel may start its prologue
-    const int H = a.H, E = a.E, k = a.k;
-    const int C = static_cast<int>(cluster.num_blocks());
-    const int rank = static_cast<int>(cluster.block_rank());
-    const int er = ceil_div(E, C);
-    float *xnat = rsm;
-    float *lg = rsm + H;
-    float *lall = lg + er;
+    const int H = a.H, E = a.E;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    if (!a.logits_in) {
-        for (int i = threadIdx.x; i < H / 4; i += kDecThreads)
-            reinterpret_cast<float4 *>(xnat)[i] = a.x_bf16 ? load4(static_cast<const __nv_bfloat16 *>(a.x) + 4 * i)
-                                                           : load4(static_cast<const float *>(a.x) + 4 * i);
-        __syncthreads();
-        const int e0 = min(E, rank * er), e1 = min(E, e0 + er);
-        constexpr int RI = 8;                            // H <= 2048: one row's loads all in flight
-        for (int e = e0 + warp; e < e1; e += kDecWarps) {
-            float4 w0[RI], w1[RI];
+    const int e = blockIdx.x * kLogitRows + warp;
+    uint4 w[8];                                          // bf16 rows: 8 x 16 B per lane covers H <= 2048
+    if (a.w_bf16) {
 #pragma unroll
-            for (int j = 0; j < RI; ++j) {
-                const int hh = lane * 8 + 256 * j;
-                w0[j] = w1[j] = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (hh < H) {
-                    if (a.w_bf16) {
-                        const __nv_bfloat16 *wr =
-                            static_cast<const __nv_bfloat16 *>(a.w_router) + static_cast<size_t>(e) * H + hh;
-                        w0[j] = load4(wr);
-                        w1[j] = load4(wr + 4);
-                    } else {
-                        const float *wr = static_cast<const float *>(a.w_router) + static_cast<size_t>(e) * H + hh;
-                        w0[j] = load4(wr);
-                        w1[j] = load4(wr + 4);
-                    }
-                }
-            }
-            float acc = 0.f;
+        for (int j = 0; j < 8; ++j) {
+            const int hh = lane * 8 + 256 * j;
+            w[j] = make_uint4(0, 0, 0, 0);
+            if (e < E && hh < H)
+                w[j] = ldg_stream(static_cast<const __nv_bfloat16 *>(a.w_router) + static_cast<size_t>(e) * H + hh);
+        }
+    }
+    for (int i = threadIdx.x; i < H / 4; i += blockDim.x)
+        reinterpret_cast<float4 *>(xs)[i] = a.x_bf16 ? load4(static_cast<const __nv_bfloat16 *>(a.x) + 4 * i)
+                                                     : load4(static_cast<const float *>(a.x) + 4 * i);
+    __syncthreads();
+    if (e >= E) return;
+    float s = 0.f;
+    if (a.w_bf16) {
 #pragma unroll
-            for (int j = 0; j < RI; ++j) {
-                const int hh = lane * 8 + 256 * j;
-                if (hh < H) {
-                    const float4 x0 = reinterpret_cast<const float4 *>(xnat + hh)[0];
-                    const float4 x1 = reinterpret_cast<const float4 *>(xnat + hh)[1];
-                    acc = fmaf(w0[j].x, x0.x, acc); acc = fmaf(w0[j].y, x0.y, acc);
-                    acc = fmaf(w0[j].z, x0.z, acc); acc = fmaf(w0[j].w, x0.w, acc);
-                    acc = fmaf(w1[j].x, x1.x, acc); acc = fmaf(w1[j].y, x1.y, acc);
-                    acc = fmaf(w1[j].z, x1.z, acc); acc = fmaf(w1[j].w, x1.w, acc);
-                }
-            }
-            acc = warp_sum(acc);
-            if (lane == 0) {
-                const float l = acc + (a.bias ? a.bias[e] : 0.f);
-                lg[e - e0] = l;
-                if (a.logits_out) a.logits_out[e] = l;
+        for (int j = 0; j < 8; ++j) {
+            const int hh = lane * 8 + 256 * j;
+            if (hh < H) {
+                const float4 x0 = reinterpret_cast<const float4 *>(xs + hh)[0];
+                const float4 x1 = reinterpret_cast<const float4 *>(xs + hh)[1];
+                const uint4 u = w[j];
+                s = fmaf(__uint_as_float(u.x << 16), x0.x, s);
+                s = fmaf(__uint_as_float(u.x & 0xffff0000u), x0.y, s);
+                s = fmaf(__uint_as_float(u.y << 16), x0.z, s);
+                s = fmaf(__uint_as_float(u.y & 0xffff0000u), x0.w, s);
+                s = fmaf(__uint_as_float(u.z << 16), x1.x, s);
+                s = fmaf(__uint_as_float(u.z & 0xffff0000u), x1.y, s);
+                s = fmaf(__uint_as_float(u.w << 16), x1.z, s);
+                s = fmaf(__uint_as_float(u.w & 0xffff0000u), x1.w, s);
             }
         }
-        cluster.sync();                                  // logit rows visible cluster-wide
-        if (rank == 0)
-            for (int e = threadIdx.x; e < E; e += kDecThreads) lall[e] = cluster.map_shared_rank(lg, e / er)[e % er];
-        cluster.sync();                                  // no distributed shared memory reads after this
-    } else if (rank == 0) {
-        for (int e = threadIdx.x; e < E; e += kDecThreads) lall[e] = a.logits_in[e];
+    } else {
+        for (int hh = lane * 4; hh < H; hh += 128) {
+            const float4 wv = load4(static_cast<const float *>(a.w_router) + static_cast<size_t>(e) * H + hh);
+            const float4 xv = reinterpret_cast<const float4 *>(xs + hh)[0];
+            s = fmaf(wv.x, xv.x, s); s = fmaf(wv.y, xv.y, s);
+            s = fmaf(wv.z, xv.z, s); s = fmaf(wv.w, xv.w, s);
+        }
     }
-    if (rank != 0) return;
+    s = warp_sum(s);
+    if (lane == 0) {
+        const float l = s + (a.bias ? a.bias[e] : 0.f);
+        a.ws.logits[e] = l;
+        if (a.logits_out) a.logits_out[e] = l;
+    }
+}
+
+// Top-k (k <= 32) of E <= 1024 logits by one block of kDecThreads threads.
+// Each warp first takes the k best of its keys (k rounds of two warp max
+// reductions: the value key, then among equal values the larger low word,
+// i.e. the lower id), then warp 0 takes the k best of those 8k candidates.
+// sel[0..k-1] receives the selection keys in rank order.
+template <int N>
+__device__ __forceinline__ void warp_take(uint64_t (&keys)[N], int k, int lane, uint64_t *dst) {
+    uint64_t best = 0ull;
+#pragma unroll
+    for (int q = 0; q < N; ++q) best = keys[q] > best ? keys[q] : best;
+    for (int r = 0; r < k; ++r) {
+        const uint32_t hi = __reduce_max_sync(0xffffffffu, static_cast<uint32_t>(best >> 32));
+        const uint32_t lo =
+            __reduce_max_sync(0xffffffffu, static_cast<uint32_t>(best >> 32) == hi ? static_cast<uint32_t>(best) : 0u);
+        const uint64_t win = (static_cast<uint64_t>(hi) << 32) | lo;
+        if (lane == 0) dst[r] = win;
+        if (best == win && win != 0ull) {                // keys are distinct: exactly one lane holds it
+            best = 0ull;
+#pragma unroll
+            for (int q = 0; q < N; ++q) {
+                if (keys[q] == win) keys[q] = 0ull;
+                best = keys[q] > best ? keys[q] : best;
+            }
+        }
+    }
+}
+
+__device__ void block_topk(const float *logits, int E, int k, uint64_t *cand, uint64_t *sel) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    {
+        uint64_t keys[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int e = threadIdx.x + kDecThreads * q;
+            keys[q] = e < E ? sel_key(__ldcg(logits + e), e) : 0ull;
+        }
+        warp_take(keys, k, lane, cand + warp * k);
+    }
     __syncthreads();
     if (warp == 0) {
-        float my_v = 0.f;
-        int my_id = 0;
-        warp_topk_smem(lall, E, k, lane, my_v, my_id);
-        const float v0 = __shfl_sync(0xffffffffu, my_v, 0);
-        const bool bad = lane < k && (my_v != my_v || my_v == __int_as_float(0x7f800000));
-        const bool any_bad = __any_sync(0xffffffffu, bad);
-        const float ex = lane < k ? expf(my_v - v0) : 0.f;
-        float s = 0.f;
-        for (int j = 0; j < k; ++j) s += __shfl_sync(0xffffffffu, ex, j);   // slot order
-        if (lane < k) {
-            const float wj = any_bad ? __int_as_float(0x7fc00000) : ex / s;
-            a.ws.ids[lane] = my_id;
-            a.ws.gates[lane] = wj;
-            a.ids_out[lane] = my_id;
-            a.w_out[lane] = wj;
+        uint64_t keys[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            const int i = lane + 32 * q;
+            keys[q] = i < kDecWarps * k ? cand[i] : 0ull;
         }
-        if (lane == 0 && any_bad) report(a.err, MOE_DEVERR_NONFINITE);
+        warp_take(keys, k, lane, sel);
     }
+    __syncthreads();
 }
 
 // ----------------------------------------------------------- 2. gate/up
 // Block = 8 warps x 2 row pairs = 16 rows of one group; grid = groups x I/16.
-// The last group (when present) is the shared expert.
+// The last group (when present) is the shared expert.  Each lane keeps the
+// activation pieces of one chunk in registers and applies them to the four
+// weight rows of its warp (gate and up of two rows).
 template <int BITS>
-__global__ void __launch_bounds__(kDecThreads, 3) k_dec_gateup(DecodeArgs a) {
+__global__ void __launch_bounds__(kDecThreads, BITS == 4 ? 3 : 2) k_dec_gateup(DecodeArgs a) {
     using Q = QT<BITS>;
     extern __shared__ __align__(16) float4 gsm[];
     __shared__ const uint8_t *blob_s;
@@ -220,21 +200,43 @@ __global__ void __launch_bounds__(kDecThreads, 3) k_dec_gateup(DecodeArgs a) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     float4 *xs = gsm;
     float *cs = reinterpret_cast<float *>(gsm + H / 4);
-    // prologue: x pieces + block sums (independent of the routing)
     {
-        const void *rows[1] = {a.x};
-        stage_rows<BITS>(xs, cs, 1, 1, H, rows, a.x_bf16);
+        const void *x = a.x;
+        stage_rows_fn<BITS>(xs, cs, 1, 1, H, [x](int) { return x; }, a.x_bf16);   // independent of the routing
     }
     pdl_trigger();                                       // the down kernel may start
-    if (threadIdx.x == 0) {
-        const uint8_t *b = a.shared;
-        if (!shared_group) {
-            pdl_wait();                                  // the route kernel's ids are needed from here on
-            const int e = a.ws.ids[g];
-            b = (e >= 0 && e < a.E) ? a.blobs[e] : nullptr;
-            if (!b) report(a.err, (e >= 0 && e < a.E) ? MOE_DEVERR_NULL_BLOB : MOE_DEVERR_BAD_EXPERT);
+    if (!shared_group) {
+        pdl_wait();                                      // the logits are final from here on
+        __shared__ uint64_t cand[kDecWarps * 32], sel[32];
+        block_topk(a.logits_in ? a.logits_in : a.ws.logits, a.E, k, cand, sel);
+        if (blockIdx.x == 0 && threadIdx.x < 32) {       // one CTA publishes ids and gates
+            const int lane = threadIdx.x;
+            const uint64_t key = lane < k ? sel[lane] : 0ull;
+            const float my_v = key_float(static_cast<uint32_t>(key >> 32));
+            const int my_id = static_cast<int>(0xffffffffu - static_cast<uint32_t>(key));
+            const float v0 = __shfl_sync(0xffffffffu, my_v, 0);
+            const bool bad = lane < k && (my_v != my_v || my_v == __int_as_float(0x7f800000));
+            const bool any_bad = __any_sync(0xffffffffu, bad);
+            const float ex = lane < k ? expf(my_v - v0) : 0.f;
+            float sum = 0.f;
+            for (int j = 0; j < k; ++j) sum += __shfl_sync(0xffffffffu, ex, j);   // slot order
+            if (lane < k) {
+                const float wj = any_bad ? __int_as_float(0x7fc00000) : ex / sum;
+                a.ws.ids[lane] = my_id;
+                a.ws.gates[lane] = wj;
+                a.ids_out[lane] = my_id;
+                a.w_out[lane] = wj;
+            }
+            if (lane == 0 && any_bad) report(a.err, MOE_DEVERR_NONFINITE);
         }
-        blob_s = b;
+        if (threadIdx.x == 0) {
+            const int e = static_cast<int>(0xffffffffu - static_cast<uint32_t>(sel[g]));
+            const uint8_t *b = (e >= 0 && e < a.E) ? a.blobs[e] : nullptr;
+            if (!b) report(a.err, (e >= 0 && e < a.E) ? MOE_DEVERR_NULL_BLOB : MOE_DEVERR_BAD_EXPERT);
+            blob_s = b;
+        }
+    } else if (threadIdx.x == 0) {
+        blob_s = a.shared;
     }
     __syncthreads();
     const uint8_t *blob = blob_s;
@@ -243,65 +245,77 @@ __global__ void __launch_bounds__(kDecThreads, 3) k_dec_gateup(DecodeArgs a) {
     const int nch = H / Q::EPC;
     const int nscx = H / 32;
     const size_t xrowb = static_cast<size_t>(H) * BITS / 8;
-    uint4 cgv[2][2], cuv[2][2];
-    float sgv[2][2][Q::BPC], suv[2][2][Q::BPC];
+    // all code loads of the warp's four row vectors first
+    constexpr int S = 2048 / Q::EPC / 32;               // chunks per lane (H <= 2048)
+    uint4 code[4][S];
+    float dsc[4][S][Q::BPC];
 #pragma unroll
-    for (int j = 0; j < 2; ++j) {
-        const int i = i0 + warp * 2 + j;
+    for (int v = 0; v < 4; ++v) {
+        const int i = i0 + warp * 2 + (v >> 1);
+        const uint8_t *cbase = (v & 1) ? bv.cu : bv.cg;
+        const __half *sbase = (v & 1) ? bv.su : bv.sg;
 #pragma unroll
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < S; ++s) {
             const int cc = lane + 32 * s;
             const bool valid = cc < nch;
-            cgv[j][s] = cuv[j][s] = make_uint4(0, 0, 0, 0);
-            if (valid) {
-                const size_t off = static_cast<size_t>(i) * xrowb + static_cast<size_t>(cc) * 16;
-                cgv[j][s] = ldg_stream(bv.cg + off);
-                cuv[j][s] = ldg_stream(bv.cu + off);
+            code[v][s] = valid ? ldg_stream(cbase + static_cast<size_t>(i) * xrowb + static_cast<size_t>(cc) * 16)
+                               : make_uint4(0, 0, 0, 0);
+            load_scales<BITS>(sbase + static_cast<size_t>(i) * nscx, cc, valid, dsc[v][s]);
+        }
+    }
+    float dot[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int s = 0; s < S; ++s) {
+        const int cc = lane + 32 * s;
+        if (cc < nch) {
+            float4 xp[Q::PPC];
+#pragma unroll
+            for (int q = 0; q < Q::PPC; ++q) xp[q] = xs[q * nch + cc];
+            float csum[Q::BPC];
+#pragma unroll
+            for (int b = 0; b < Q::BPC; ++b) csum[b] = cs[cc * Q::BPC + b];
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+                float fx[Q::BPC];
+                chunk_fx<BITS>(code[v][s], xp, fx);
+                dot[v] = chunk_finish<BITS>(fx, dsc[v][s], csum, dot[v]);
             }
-            load_scales<BITS>(bv.sg + static_cast<size_t>(i) * nscx, cc, valid, sgv[j][s]);
-            load_scales<BITS>(bv.su + static_cast<size_t>(i) * nscx, cc, valid, suv[j][s]);
         }
     }
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
-        const int i = i0 + warp * 2 + j;
-        float dg[1] = {0.f}, du[1] = {0.f};
-#pragma unroll
-        for (int s = 0; s < 2; ++s) {
-            const int cc = lane + 32 * s;
-            if (cc < nch) {
-                chunk_dot<BITS, 1>(cgv[j][s], sgv[j][s], xs, cs, nch, cc, dg);
-                chunk_dot<BITS, 1>(cuv[j][s], suv[j][s], xs, cs, nch, cc, du);
-            }
-        }
-        const float gv = warp_sum(dg[0]);
-        const float uv = warp_sum(du[0]);
-        if (lane == 0) a.ws.h[static_cast<size_t>(g) * I + i] = gv / (1.0f + expf(-gv)) * uv;
+        const float gv = warp_sum(dot[2 * j]);
+        const float uv = warp_sum(dot[2 * j + 1]);
+        if (lane == 0) a.ws.h[static_cast<size_t>(g) * I + i0 + warp * 2 + j] = gv / (1.0f + expf(-gv)) * uv;
     }
 }
 
 // ------------------------------------------------------ 3. down + combine
-// Warp = RPW output rows x all groups; lanes split a row's chunks (lpr lanes
-// per group row, 32/lpr groups at a time).  Codes are loaded before h is
-// staged (kDownRows x kMaxPass codes per lane in registers).
-constexpr int kDownRows = 2;
-constexpr int kMaxPass = 8;                             // passes of 32/lpr groups each (checked on the host)
+// Block = RB output rows x all groups.  Tasks (group, lane-row group) are
+// spread over the 8 warps; each lane takes one chunk of one row (lpr lanes
+// per row), with every code load of the warp issued before h is staged.
+// Per-group partials meet in shared memory and are summed in slot order.
+constexpr int kDownTasks = 8;                            // tasks per warp (checked on the host)
 
 template <int BITS>
-__global__ void __launch_bounds__(kDecThreads, 2) k_dec_down(DecodeArgs a, int ng, int lpr) {
+__global__ void __launch_bounds__(kDecThreads, 2) k_dec_down(DecodeArgs a, int ng, int RB) {
     using Q = QT<BITS>;
     extern __shared__ __align__(16) float4 dsm[];
     __shared__ const uint8_t *blobs_s[33];
     __shared__ float gates_s[33];
     const int H = a.H, I = a.I, k = a.k;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int r0 = (blockIdx.x * kDecWarps + warp) * kDownRows;
-    const int gpp = 32 / lpr;                            // groups per warp pass
-    const int npass = ceil_div(ng, gpp);
-    const int sub = lane / lpr, seg = lane % lpr;
-    const int nchd = I / Q::EPC;                         // == lpr (checked on the host)
+    const int nchd = I / Q::EPC;                         // chunks per row == lanes per row (power of two)
+    const int lpr = nchd;
+    const int rpp = 32 / lpr;                            // rows per task
+    const int tpg = RB / rpp;                            // tasks per group
+    const int ntasks = ng * tpg;
+    const int r0 = blockIdx.x * RB;
     const size_t drowb = static_cast<size_t>(I) * BITS / 8;
     const int dnsc = I / 32;
+    float4 *hs = dsm;
+    float *hcs = reinterpret_cast<float *>(dsm + static_cast<size_t>(ng) * (I / 4));
+    float *part = hcs + static_cast<size_t>(ng) * (I / 32);
     pdl_wait();                                          // ids (route) and h (gate/up) are final
     if (threadIdx.x < ng) {
         const int g = threadIdx.x;
@@ -316,54 +330,48 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_dec_down(DecodeArgs a, int n
         gates_s[g] = gw;
     }
     __syncthreads();
-    // issue every code load of this warp's rows first
-    uint4 code[kDownRows][kMaxPass];
-    float sc[kDownRows][kMaxPass][Q::BPC];
+    const int seg = lane % lpr, sub = lane / lpr;
+    uint4 code[kDownTasks];
+    float dsc[kDownTasks][Q::BPC];
 #pragma unroll
-    for (int rr = 0; rr < kDownRows; ++rr)
-#pragma unroll
-        for (int p = 0; p < kMaxPass; ++p) {
-            const int g = p * gpp + sub;
-            const int r = r0 + rr;
-            const bool valid = p < npass && g < ng && r < H && blobs_s[g] != nullptr;
-            code[rr][p] = make_uint4(0, 0, 0, 0);
-            sc[rr][p][0] = 0.f;
-            if (Q::BPC > 1) sc[rr][p][Q::BPC - 1] = 0.f;
-            if (valid) {
-                const BlobView bv = blob_view(blobs_s[g], BITS, H, I);
-                code[rr][p] = ldg_stream(bv.cd + static_cast<size_t>(r) * drowb + static_cast<size_t>(seg) * 16);
-                load_scales<BITS>(bv.sd + static_cast<size_t>(r) * dnsc, seg, true, sc[rr][p]);
-            }
-        }
-    // h of every group as pieces + block sums
-    float4 *hs = dsm;
-    float *hcs = reinterpret_cast<float *>(dsm + static_cast<size_t>(ng) * (I / 4));
-    {
-        const void *rows[33];
-        for (int g = 0; g < ng; ++g) rows[g] = a.ws.h + static_cast<size_t>(g) * I;
-        stage_rows<BITS>(hs, hcs, ng, ng, I, rows, 0);
+    for (int t = 0; t < kDownTasks; ++t) {
+        const int task = warp + kDecWarps * t;
+        const int g = task / tpg;
+        const int r = r0 + (task % tpg) * rpp + sub;
+        const bool valid = task < ntasks && r < H && blobs_s[g] != nullptr;
+        code[t] = make_uint4(0, 0, 0, 0);
+        const BlobView bv = blob_view(valid ? blobs_s[g] : a.shared, BITS, H, I);
+        if (valid) code[t] = ldg_stream(bv.cd + static_cast<size_t>(r) * drowb + static_cast<size_t>(seg) * 16);
+        load_scales<BITS>(bv.sd + static_cast<size_t>(valid ? r : 0) * dnsc, seg, valid, dsc[t]);
     }
+    {
+        const float *h = a.ws.h;
+        stage_rows_fn<BITS>(hs, hcs, ng, ng, I,
+                            [h, I](int t) { return static_cast<const void *>(h + static_cast<size_t>(t) * I); }, 0);
+    }                                                    // ends with __syncthreads
 #pragma unroll
-    for (int rr = 0; rr < kDownRows; ++rr) {
-        const int r = r0 + rr;
+    for (int t = 0; t < kDownTasks; ++t) {
+        const int task = warp + kDecWarps * t;
+        if (task >= ntasks) break;                       // uniform over the warp
+        const int g = task / tpg;
+        const int rl = (task % tpg) * rpp + sub;
+        float4 xp[Q::PPC];
+#pragma unroll
+        for (int q = 0; q < Q::PPC; ++q) xp[q] = hs[static_cast<size_t>(g) * (I / 4) + q * nchd + seg];
+        float csum[Q::BPC];
+#pragma unroll
+        for (int b = 0; b < Q::BPC; ++b) csum[b] = hcs[static_cast<size_t>(g) * (I / 32) + seg * Q::BPC + b];
+        float fx[Q::BPC];
+        chunk_fx<BITS>(code[t], xp, fx);
+        float v = blobs_s[g] ? chunk_finish<BITS>(fx, dsc[t], csum, 0.f) : 0.f;
+        for (int o = lpr >> 1; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        if (seg == 0) part[g * RB + rl] = v;
+    }
+    __syncthreads();
+    if (threadIdx.x < RB && r0 + static_cast<int>(threadIdx.x) < H) {
         float acc = 0.f;
-#pragma unroll
-        for (int p = 0; p < kMaxPass; ++p) {
-            if (p >= npass) break;
-            const int g = p * gpp + sub;
-            float dot[1] = {0.f};
-            if (g < ng && blobs_s[g])
-                chunk_dot<BITS, 1>(code[rr][p], sc[rr][p], hs + static_cast<size_t>(g) * (I / 4),
-                                   hcs + static_cast<size_t>(g) * (I / 32), nchd, seg, dot);
-            float v = dot[0];
-            for (int o = lpr >> 1; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-            for (int s2 = 0; s2 < gpp; ++s2) {           // slot order: groups p*gpp + s2
-                const float vs = __shfl_sync(0xffffffffu, v, s2 * lpr);
-                const int gg = p * gpp + s2;
-                if (gg < ng) acc = fmaf(gates_s[gg], vs, acc);
-            }
-        }
-        if (lane == 0 && r < H) a.y[r] = acc;
+        for (int g = 0; g < ng; ++g) acc = fmaf(gates_s[g], part[g * RB + threadIdx.x], acc);   // slot order
+        a.y[r0 + threadIdx.x] = acc;
     }
 }
 
@@ -372,13 +380,16 @@ size_t decode_ws_bytes(int E, int k, int I) {
     return 256 + ((static_cast<size_t>(E) * 4 + 255) / 256) * 256 + static_cast<size_t>(k + 1) * I * 4;
 }
 
+static int down_rows_per_block(int ng) { return ng <= 16 ? 8 : 4; }
+
 bool decode_supported(int bits, int H, int I, int E, int k) {
     if (E > 1024 || k > 32 || H > 2048 || I % 128 != 0) return false;
     const int nchd = I / (bits == 4 ? 32 : 64);
     if (nchd > 32 || (nchd & (nchd - 1)) != 0) return false;    // one chunk per lane, power-of-two lanes per row
-    const int gpp = 32 / nchd;
-    if (ceil_div(k + 1, gpp) > kMaxPass) return false;
-    const size_t smem_down = static_cast<size_t>(k + 1) * I * 4 + static_cast<size_t>(k + 1) * (I / 32) * 4;
+    const int rpp = 32 / nchd, ng = k + 1, RB = down_rows_per_block(ng);
+    if (RB % rpp != 0 || ceil_div(ng * (RB / rpp), kDecWarps) > kDownTasks) return false;
+    const size_t smem_down = static_cast<size_t>(ng) * I * 4 + static_cast<size_t>(ng) * (I / 32) * 4 +
+                             static_cast<size_t>(ng) * RB * 4;
     return smem_down <= 200 * 1024;
 }
 
@@ -388,26 +399,13 @@ static int launch_decode_t(DecodeArgs a, int groups, cudaStream_t s) {
     cudaLaunchAttribute pdl;
     pdl.id = cudaLaunchAttributeProgrammaticStreamSerialization;
     pdl.val.programmaticStreamSerializationAllowed = 1;
-    // 1. route: one cluster (16 CTAs when the router is computed here)
-    {
-        int C = a.logits_in ? 1 : 16;
-        const size_t smem = (static_cast<size_t>(H) + ceil_div(E, C) + E) * 4;
-        int rc = cuda_status(cudaFuncSetAttribute(k_dec_route, cudaFuncAttributeNonPortableClusterSizeAllowed, 1),
-                             "route cluster attribute");
-        if (rc) return rc;
+    // 1. router logits (skipped when the caller supplies them)
+    if (!a.logits_in) {
         cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(C);
-        cfg.blockDim = dim3(kDecThreads);
-        cfg.dynamicSmemBytes = smem;
+        cfg.gridDim = dim3(ceil_div(E, kLogitRows));
+        cfg.blockDim = dim3(kLogitRows * 32);
         cfg.stream = s;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = C;
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        rc = cuda_status(cudaLaunchKernelEx(&cfg, k_dec_route, a), "decode route launch");
+        int rc = cuda_status(cudaLaunchKernelEx(&cfg, k_dec_logits, a), "decode logits launch");
         count_launches(1);
         if (rc) return rc;
     }
@@ -421,28 +419,28 @@ static int launch_decode_t(DecodeArgs a, int groups, cudaStream_t s) {
         cfg.dynamicSmemBytes = smem;
         cfg.stream = s;
         cfg.attrs = &pdl;
-        cfg.numAttrs = 1;
+        cfg.numAttrs = a.logits_in ? 0 : 1;              // x and given logits come from earlier work: no overlap
         int rc = cuda_status(cudaLaunchKernelEx(&cfg, k_dec_gateup<BITS>, a), "decode gate/up launch");
         count_launches(1);
         if (rc) return rc;
     }
     // 3. down + combine
     {
-        const int nchd = I / QT<BITS>::EPC;
-        const int lpr = nchd;
-        const size_t smem = static_cast<size_t>(groups) * I * 4 + static_cast<size_t>(groups) * (I / 32) * 4;
+        const int RB = down_rows_per_block(groups);
+        const size_t smem = static_cast<size_t>(groups) * I * 4 + static_cast<size_t>(groups) * (I / 32) * 4 +
+                            static_cast<size_t>(groups) * RB * 4;
         int rc = cuda_status(cudaFuncSetAttribute(k_dec_down<BITS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                   static_cast<int>(smem)),
                              "down smem attribute");
         if (rc) return rc;
         cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(ceil_div(H, kDecWarps * kDownRows));
+        cfg.gridDim = dim3(ceil_div(H, RB));
         cfg.blockDim = dim3(kDecThreads);
         cfg.dynamicSmemBytes = smem;
         cfg.stream = s;
         cfg.attrs = &pdl;
         cfg.numAttrs = 1;
-        rc = cuda_status(cudaLaunchKernelEx(&cfg, k_dec_down<BITS>, a, groups, lpr), "decode down launch");
+        rc = cuda_status(cudaLaunchKernelEx(&cfg, k_dec_down<BITS>, a, groups, RB), "decode down launch");
         count_launches(1);
         return rc;
     }

@@ -7,12 +7,15 @@
 // Per tile: 128 weight rows (MMA M) x up to 256 of the expert's tokens (MMA N),
 // K in steps of 64.  Weights are the A operand, so small token groups still
 // fill the M = 128 datapath ("swap AB").  Roles of one persistent CTA per SM:
-//   warps 0-3  producers: copy raw codes + scales (cp.async, two steps ahead),
-//              dequantise them to fp16 into the 128-byte-swizzled A tile, and
-//              gather the tile's token rows (fp16) into the B tile;
-//   warp  8    allocates 512 TMEM columns and issues tcgen05.mma (one thread);
-//   warps 4-7  epilogue: tcgen05.ld the fp32 accumulators and write
-//              gate/up -> h = silu(g) * u (fp16) or down -> y rows (fp32).
+//   warps 0-7   copy their raw codes + scales a few k-steps ahead (cp.async
+//               into private slots) and dequantise them to fp16 into the
+//               128-byte-swizzled A stages;
+//   warps 13-14 gather the tile's token rows (fp16) into the B stages with
+//               cp.async, each thread arriving on the stage's barrier when
+//               its copies land (cp.async.mbarrier.arrive.noinc);
+//   warp  12    allocates TMEM and issues tcgen05.mma (one thread);
+//   warps 8-11  epilogue: tcgen05.ld the fp32 accumulators and write
+//               gate/up -> h = silu(g) * u (fp16) or down -> y rows (fp32).
 // Every mbarrier wait is bounded; a timeout sets MOE_DEVERR_TIMEOUT and all
 // roles leave their loops, after which TMEM is freed.
 #include "common.cuh"
@@ -24,31 +27,39 @@ using namespace sm100;
 
 constexpr int kBM = 128;            // weight rows per tile
 constexpr int kBK = 64;             // K per stage: one 128-byte row of fp16
-constexpr int kMaxN = 256;          // tokens per tile
-constexpr int kStA = 2;             // A operand stages
-constexpr int kStB = 3;             // B operand stages = raw-code ring slots
-constexpr int kLook = kStB - 1;     // copies run this many k-steps ahead
-constexpr int kGemmThreads = 288;   // 4 producer warps, 4 epilogue warps, 1 MMA warp
+constexpr int kProd = 256;          // dequantising threads: 128 rows x 2 parts
+constexpr int kLoad = 64;           // token-row loader threads
+constexpr int kGemmThreads = 480;   // 8 dequant warps, 4 epilogue warps, 1 MMA warp, 2 loader warps
 constexpr long kSpin = 1L << 22;    // polls before a wait gives up (about a second)
 constexpr int kMaxGroups = 2048;
 
-template <int BITS, bool GATEUP>
+// MAXN: tokens per tile.  Small tiles (64) leave room for deep rings (the
+// HBM-bound regime: few tokens per expert); large tiles (256) fill the
+// tensor cores when experts hold hundreds of tokens.
+template <int BITS, bool GATEUP, int MAXN>
 struct GemmCfg {
     static constexpr int NA = GATEUP ? 2 : 1;                 // weight matrices per tile (gate, up)
-    static constexpr int RAW_CODE = kBK * BITS / 8;           // code bytes of a row per k-step
-    static constexpr int SEG = (RAW_CODE + 4 + 15) / 16 * 16; // codes + 2 fp16 scales, 16-byte aligned
-    static constexpr int RAW_ROW = NA * SEG;
+    static constexpr int ELEMS = GATEUP ? 64 : 32;            // elements one producer thread dequantises per k-step
+    static constexpr int RAW_CODE = ELEMS * BITS / 8;         // its code bytes per k-step
+    static constexpr int SEG = (RAW_CODE + 4 + 15) / 16 * 16; // codes + two fp16 scales, 16-byte aligned
+    static constexpr int SA = GATEUP ? 3 : 4;                 // A (dequantised weight) stages
+    static constexpr int SB = MAXN > 128 ? (GATEUP ? 3 : 4) : 8;   // B (token row) stages
+    static constexpr int L = MAXN > 128 ? (GATEUP ? 2 : 3) : 4;    // k-steps the code copies run ahead (= slots)
+    static constexpr int ACC = NA * MAXN * 2 <= 512 ? 2 : 1;  // TMEM accumulator buffers
+    static constexpr int TMEM_COLS = ACC * NA * MAXN <= 128 ? 128 : (ACC * NA * MAXN <= 256 ? 256 : 512);
     static constexpr size_t A_STAGE = static_cast<size_t>(NA) * kBM * 128;
-    static constexpr size_t B_STAGE = static_cast<size_t>(kMaxN) * 128;
-    static constexpr size_t RAW_STAGE = static_cast<size_t>(kBM) * RAW_ROW;
-    // shared-memory plan
+    static constexpr size_t B_STAGE = static_cast<size_t>(MAXN) * 128;
+    static constexpr size_t RAW_STAGE = static_cast<size_t>(kProd) * SEG;
     static constexpr size_t OFF_A = 0;
-    static constexpr size_t OFF_B = OFF_A + kStA * A_STAGE;
-    static constexpr size_t OFF_RAW = OFF_B + kStB * B_STAGE;
-    static constexpr size_t OFF_TOK = OFF_RAW + kStB * RAW_STAGE;
-    static constexpr size_t OFF_GS = OFF_TOK + kMaxN * 4;
+    static constexpr size_t OFF_B = OFF_A + SA * A_STAGE;
+    static constexpr size_t OFF_RAW = OFF_B + SB * B_STAGE;
+    static constexpr size_t OFF_TOK = OFF_RAW + L * RAW_STAGE;
+    static constexpr size_t OFF_GS = OFF_TOK + MAXN * 4;
     static constexpr size_t OFF_BAR = (OFF_GS + (kMaxGroups + 1) * 4 + 15) / 16 * 16;
-    static constexpr size_t SMEM = OFF_BAR + 16 * 8 + 16 + 1024;   // + slack for 1024-byte alignment
+    static constexpr size_t SMEM = OFF_BAR + 32 * 8 + 16 + 1024;   // bars, TMEM address, tile count, abort
+                                                                   // flag; + slack for 1024-byte alignment
+    static_assert(2 * SA + 2 * SB + 5 <= 32, "barrier slots");
+    static_assert(SMEM <= 232448, "shared memory per block (no static shared memory is used)");
 };
 
 struct GemmArgs {
@@ -89,95 +100,71 @@ __device__ __forceinline__ GroupInfo group_info(const GemmArgs &a, int g, int n_
     return G;
 }
 
-// fp16 weights of 8 consecutive elements from 4 packed code bytes (q4: the
-// low or high nibbles of 8 bytes) -- returned as 4 half2 words.
-__device__ __forceinline__ uint32_t pair16(uint32_t bytes, uint32_t sel) {
-    // bytes hold one code (0..15) per byte; builds half2 (1024 + q_a, 1024 + q_b)
-    return __byte_perm(bytes, 0x64646464u, sel);
-}
+// One tile of this CTA's sequence: group, first token, first weight row.
+struct TileInfo {
+    GroupInfo G;
+    int n0, m0, nvalid, N;
+};
+
+// bytes hold one code per byte; builds the half2 (1024 + q_a, 1024 + q_b)
+__device__ __forceinline__ uint32_t pair16(uint32_t bytes, uint32_t sel) { return __byte_perm(bytes, 0x64646464u, sel); }
 __device__ __forceinline__ uint32_t dq2(uint32_t magic_pair, __half2 offset, __half2 d2) {
     __half2 h = *reinterpret_cast<__half2 *>(&magic_pair);
     h = __hmul2(__hsub2(h, offset), d2);       // (q - offset) exact, then one rounding of d * (q - offset)
     return *reinterpret_cast<uint32_t *>(&h);
 }
+__device__ __forceinline__ void st_shared16(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
 
-// Dequantises one row's k-step (64 elements) into the swizzled A row.
+// Dequantises one quant block (32 elements) into chunks chunk0..chunk0+3 of a
+// swizzled 128-byte A row (chunk c stored at c ^ (row % 8)).
 template <int BITS>
-__device__ __forceinline__ void dequant_row(const uint8_t *raw_seg, uint32_t a_row_addr, int row) {
-    constexpr int RAW_CODE = kBK * BITS / 8;
-    const uint4 *cw = reinterpret_cast<const uint4 *>(raw_seg);
-    const __half2 *sc = reinterpret_cast<const __half2 *>(raw_seg + RAW_CODE);
-    const __half2 s01 = *sc;
-    const int sw = row & 7;
+__device__ __forceinline__ void dequant_block(const uint8_t *codes, __half2 d2, uint32_t a_row, int chunk0, int sw) {
     if constexpr (BITS == 4) {
         const __half2 off = __float2half2_rn(1032.0f);
+        const uint4 w = *reinterpret_cast<const uint4 *>(codes);
+        // chunk j (8 elements): 0 = low nibbles of bytes 0-7, 1 = low of 8-15,
+        //                       2 = high nibbles of bytes 0-7, 3 = high of 8-15
+        const uint32_t src[4][2] = {{w.x & 0x0F0F0F0Fu, w.y & 0x0F0F0F0Fu},
+                                    {w.z & 0x0F0F0F0Fu, w.w & 0x0F0F0F0Fu},
+                                    {(w.x >> 4) & 0x0F0F0F0Fu, (w.y >> 4) & 0x0F0F0F0Fu},
+                                    {(w.z >> 4) & 0x0F0F0F0Fu, (w.w >> 4) & 0x0F0F0F0Fu}};
 #pragma unroll
-        for (int b = 0; b < 2; ++b) {                              // quant block b: elements 32b..32b+31
-            const uint4 w = cw[b];
-            const __half2 d2 = b == 0 ? __low2half2(s01) : __high2half2(s01);
-            const uint32_t lo0 = w.x & 0x0F0F0F0Fu, lo1 = w.y & 0x0F0F0F0Fu;
-            const uint32_t lo2 = w.z & 0x0F0F0F0Fu, lo3 = w.w & 0x0F0F0F0Fu;
-            const uint32_t hi0 = (w.x >> 4) & 0x0F0F0F0Fu, hi1 = (w.y >> 4) & 0x0F0F0F0Fu;
-            const uint32_t hi2 = (w.z >> 4) & 0x0F0F0F0Fu, hi3 = (w.w >> 4) & 0x0F0F0F0Fu;
-            // chunk j (8 elements): 0 = low nibbles of bytes 0-7, 1 = low of 8-15,
-            //                       2 = high nibbles of bytes 0-7, 3 = high of 8-15
-            const uint32_t src[4][2] = {{lo0, lo1}, {lo2, lo3}, {hi0, hi1}, {hi2, hi3}};
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const uint32_t v0 = dq2(pair16(src[j][0], 0x5140u), off, d2);
-                const uint32_t v1 = dq2(pair16(src[j][0], 0x5342u), off, d2);
-                const uint32_t v2 = dq2(pair16(src[j][1], 0x5140u), off, d2);
-                const uint32_t v3 = dq2(pair16(src[j][1], 0x5342u), off, d2);
-                const int c = 4 * b + j;                               // 16-byte chunk of the 128-byte row
-                const uint32_t dst = a_row_addr + static_cast<uint32_t>(((c ^ sw) << 4));
-                asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(dst), "r"(v0), "r"(v1), "r"(v2),
-                             "r"(v3)
-                             : "memory");
-            }
-        }
+        for (int j = 0; j < 4; ++j)
+            st_shared16(a_row + ((((chunk0 + j) ^ sw)) << 4), dq2(pair16(src[j][0], 0x5140u), off, d2),
+                        dq2(pair16(src[j][0], 0x5342u), off, d2), dq2(pair16(src[j][1], 0x5140u), off, d2),
+                        dq2(pair16(src[j][1], 0x5342u), off, d2));
     } else {
         const __half2 off = __float2half2_rn(1026.0f);
-        const uint4 w = cw[0];
-        const uint32_t words[4] = {w.x, w.y, w.z, w.w};
+        const uint2 w = *reinterpret_cast<const uint2 *>(codes);
 #pragma unroll
-        for (int b = 0; b < 2; ++b) {                              // quant block b: 8 bytes = words 2b, 2b+1
-            const __half2 d2 = b == 0 ? __low2half2(s01) : __high2half2(s01);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {                          // crumb level j: elements 8j..8j+7 of the block
-                const uint32_t c0 = (words[2 * b] >> (2 * j)) & 0x03030303u;
-                const uint32_t c1 = (words[2 * b + 1] >> (2 * j)) & 0x03030303u;
-                const uint32_t v0 = dq2(pair16(c0, 0x5140u), off, d2);
-                const uint32_t v1 = dq2(pair16(c0, 0x5342u), off, d2);
-                const uint32_t v2 = dq2(pair16(c1, 0x5140u), off, d2);
-                const uint32_t v3 = dq2(pair16(c1, 0x5342u), off, d2);
-                const int c = 4 * b + j;
-                const uint32_t dst = a_row_addr + static_cast<uint32_t>(((c ^ sw) << 4));
-                asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(dst), "r"(v0), "r"(v1), "r"(v2),
-                             "r"(v3)
-                             : "memory");
-            }
+        for (int j = 0; j < 4; ++j) {            // crumb level j: elements 8j..8j+7 of the block
+            const uint32_t c0 = (w.x >> (2 * j)) & 0x03030303u, c1 = (w.y >> (2 * j)) & 0x03030303u;
+            st_shared16(a_row + ((((chunk0 + j) ^ sw)) << 4), dq2(pair16(c0, 0x5140u), off, d2),
+                        dq2(pair16(c0, 0x5342u), off, d2), dq2(pair16(c1, 0x5140u), off, d2),
+                        dq2(pair16(c1, 0x5342u), off, d2));
         }
     }
 }
 
-template <int BITS, bool GATEUP>
+template <int BITS, bool GATEUP, int MAXN>
 __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(GemmArgs a) {
-    using Cfg = GemmCfg<BITS, GATEUP>;
+    using Cfg = GemmCfg<BITS, GATEUP, MAXN>;
+    constexpr int SA = Cfg::SA, SB = Cfg::SB, L = Cfg::L, ACC = Cfg::ACC, NA = Cfg::NA;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
-    // 1024-byte alignment of the operand tiles (swizzle atoms)
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sA = smem + Cfg::OFF_A;
     uint8_t *sB = smem + Cfg::OFF_B;
     uint8_t *sRaw = smem + Cfg::OFF_RAW;
-    int32_t *sTok = reinterpret_cast<int32_t *>(smem + Cfg::OFF_TOK);
+    int32_t *tok_s = reinterpret_cast<int32_t *>(smem + Cfg::OFF_TOK);
     int32_t *gstart = reinterpret_cast<int32_t *>(smem + Cfg::OFF_GS);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::OFF_BAR);
-    uint64_t *fullA = bars, *emptyA = bars + 2, *fullB = bars + 4, *emptyB = bars + 7;
-    uint64_t *acc_full = bars + 10, *acc_empty = bars + 11, *drain = bars + 12;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 13);
-    __shared__ int abort_sh;
-    __shared__ int total_tiles_s;
-    volatile int &abort_s = abort_sh;            // read in loop conditions: never cached
+    uint64_t *fullA = bars, *emptyA = bars + SA, *fullB = bars + 2 * SA, *emptyB = bars + 2 * SA + SB;
+    uint64_t *accF = bars + 2 * SA + 2 * SB, *accE = accF + 2, *drain = accF + 4;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 32);
+    int *total_tiles_p = reinterpret_cast<int *>(bars + 32) + 1;
+    volatile int &abort_s = *(reinterpret_cast<int *>(bars + 32) + 2);   // read in loop conditions: never cached
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int K = GATEUP ? a.H : a.I;           // reduction length
@@ -189,16 +176,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(GemmArgs a) {
 
     if (tid == 0) {
         abort_s = 0;
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(fullA + i, 128);
+        for (int i = 0; i < SA; ++i) {
+            mbar_init(fullA + i, kProd);
             mbar_init(emptyA + i, 1);
         }
-        for (int i = 0; i < 3; ++i) {
-            mbar_init(fullB + i, 128);
+        for (int i = 0; i < SB; ++i) {
+            mbar_init(fullB + i, kLoad);
             mbar_init(emptyB + i, 1);
         }
-        mbar_init(acc_full, 1);
-        mbar_init(acc_empty, 128);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(accF + i, 1);
+            mbar_init(accE + i, 128);
+        }
         mbar_init(drain, 1);
         fence_barrier_init();
         fence_proxy_async();
@@ -211,7 +200,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(GemmArgs a) {
             int t = 0;
             if (g < ng) {
                 const GroupInfo G = group_info(a, g, n_act);
-                t = ((G.n + kMaxN - 1) / kMaxN) * MT;
+                t = ((G.n + MAXN - 1) / MAXN) * MT;
             }
             int incl = t;
 #pragma unroll
@@ -224,182 +213,202 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(GemmArgs a) {
         }
         if (lane == 0) {
             gstart[ng] = run;
-            total_tiles_s = run;
+            *total_tiles_p = run;
         }
     }
-    if (warp == 8) {
-        tmem_alloc(tmem_slot, 512);
+    if (warp == 12) {
+        tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
         tmem_relinquish();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const int total = total_tiles_s;
+    const int total = *total_tiles_p;
+    const int n_my = blockIdx.x < total ? (total - 1 - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x) + 1 : 0;
+    const long J = static_cast<long>(n_my) * nk;   // k-steps of this CTA
 
-    auto decode_tile = [&](int t, int &g, int &n0, int &m0) {
-        int lo = 0, hi = ng;                      // largest g with gstart[g] <= t
+    auto tile_of = [&](int i) {                  // i-th tile of this CTA
+        const int t = blockIdx.x + i * gridDim.x;
+        int lo = 0, hi = ng;                     // largest g with gstart[g] <= t
         while (hi - lo > 1) {
             const int mid = (lo + hi) >> 1;
             if (gstart[mid] <= t) lo = mid;
             else hi = mid;
         }
-        g = lo;
-        const int local = t - gstart[g];
-        n0 = (local / MT) * kMaxN;
-        m0 = (local % MT) * kBM;
+        TileInfo ti;
+        ti.G = group_info(a, lo, n_act);
+        const int local = t - gstart[lo];
+        ti.n0 = (local / MT) * MAXN;
+        ti.m0 = (local % MT) * kBM;
+        ti.nvalid = min(MAXN, ti.G.n - ti.n0);
+        ti.N = (ti.nvalid + 15) & ~15;
+        return ti;
+    };
+    auto fail = [&]() {
+        report(a.err, MOE_DEVERR_TIMEOUT);
+        abort_s = 1;
     };
 
-    if (warp < 4) {
-        // ------------------------------------------------------- producers
-        long it = 0;                              // global k-step counter of this CTA
-        const int row = tid;                      // weight row within the tile
-        for (int t = blockIdx.x; t < total && !abort_s; t += gridDim.x) {
-            int g, n0, m0;
-            decode_tile(t, g, n0, m0);
-            const GroupInfo G = group_info(a, g, n_act);
-            const int nvalid = min(kMaxN, G.n - n0);
-            const int N = (nvalid + 15) & ~15;
-            const BlobView bv = blob_view(G.blob, BITS, a.H, a.I);
-            // token rows (gate/up: x16 rows; down: h16 rows) of this tile
-            asm volatile("bar.sync 1, 128;" ::: "memory");
-            for (int n = tid; n < N; n += 128) {
-                int r = 0;
-                if (n < nvalid) {
-                    if (GATEUP) r = min(max(G.row0 >= 0 ? a.perm_src[G.row0 + n0 + n] : n0 + n, 0), a.T - 1);
-                    else r = (G.row0 >= 0 ? G.row0 : a.T * a.k) + n0 + n;
-                }
-                sTok[n] = r;
+    if (warp < 8) {
+        // ------------------------------------------------- dequantisation
+        const int row = tid & 127, part = tid >> 7;
+        const size_t rowbytes = static_cast<size_t>(K) * BITS / 8;
+        const int nsc = K / 32;
+        int raw_tile = -1;
+        TileInfo rt{};
+        // copies of this thread's codes + scales of k-step jr into its slot jr % L
+        auto issue_raw = [&](long jr) {
+            if (jr >= J) return;
+            const int i = static_cast<int>(jr / nk), s = static_cast<int>(jr % nk);
+            if (i != raw_tile) {
+                rt = tile_of(i);
+                raw_tile = i;
             }
-            asm volatile("bar.sync 1, 128;" ::: "memory");
-            const uint8_t *codes[2];
-            const __half *scl[2];
-            codes[0] = GATEUP ? bv.cg : bv.cd;
-            codes[1] = bv.cu;
-            scl[0] = GATEUP ? bv.sg : bv.sd;
-            scl[1] = bv.su;
-            const size_t rowbytes = static_cast<size_t>(K) * BITS / 8;
-            const int nsc = K / 32;
-            const uint8_t *bsrc = GATEUP ? reinterpret_cast<const uint8_t *>(a.x16)
-                                         : reinterpret_cast<const uint8_t *>(a.h16);
-            const size_t brow = static_cast<size_t>(K) * 2;
-            auto issue = [&](int s, long j) {
-                const int sb = static_cast<int>(j % kStB);
-                if (!mbar_wait(emptyB + sb, static_cast<uint32_t>(((j / kStB) & 1) ^ 1), kSpin)) {
-                    report(a.err, MOE_DEVERR_TIMEOUT);
-                    abort_s = 1;
-                }
-                // raw codes + scales of this thread's row
-                const uint32_t raw = smem_addr(sRaw + sb * Cfg::RAW_STAGE + static_cast<size_t>(row) * Cfg::RAW_ROW);
+            const BlobView bv = blob_view(rt.G.blob, BITS, a.H, a.I);
+            const uint8_t *codes = GATEUP ? (part ? bv.cu : bv.cg) : bv.cd;
+            const __half *scl = GATEUP ? (part ? bv.su : bv.sg) : bv.sd;
+            const size_t m = static_cast<size_t>(rt.m0 + row);
+            const uint8_t *src = codes + m * rowbytes + static_cast<size_t>(s) * (kBK * BITS / 8) +
+                                 (GATEUP ? 0 : part * Cfg::RAW_CODE);
+            const uint32_t dst = smem_addr(sRaw + (jr % L) * Cfg::RAW_STAGE + static_cast<size_t>(tid) * Cfg::SEG);
+            if constexpr (Cfg::RAW_CODE >= 16) {
 #pragma unroll
-                for (int mat = 0; mat < Cfg::NA; ++mat) {
-                    const uint8_t *src = codes[mat] + static_cast<size_t>(m0 + row) * rowbytes +
-                                         static_cast<size_t>(s) * Cfg::RAW_CODE;
-#pragma unroll
-                    for (int q = 0; q < Cfg::RAW_CODE / 16; ++q)
-                        cp_async16(raw + mat * Cfg::SEG + q * 16, src + q * 16, 16);
-                    cp_async4(raw + mat * Cfg::SEG + Cfg::RAW_CODE,
-                              scl[mat] + static_cast<size_t>(m0 + row) * nsc + 2 * s);
-                }
-                // token rows of the B tile, 16 bytes per copy, swizzled
-                const uint32_t bdst = smem_addr(sB + sb * Cfg::B_STAGE);
-                for (int idx = tid; idx < N * 8; idx += 128) {
-                    const int n = idx >> 3, c = idx & 7;
-                    const uint8_t *src = bsrc + static_cast<size_t>(sTok[n]) * brow + static_cast<size_t>(s) * 128 + c * 16;
-                    cp_async16(bdst + n * 128 + ((c ^ (n & 7)) << 4), src, n < nvalid ? 16u : 0u);
-                }
-                cp_async_commit();
-            };
-            const long j0 = it;
-            for (int s = 0; s < kLook && s < nk; ++s) issue(s, j0 + s);
-            for (int s = 0; s < nk && !abort_s; ++s) {
-                const long j = j0 + s;
-                if (s + 1 < nk) cp_async_wait<1>();
-                else cp_async_wait<0>();
-                const int sa = static_cast<int>(j % kStA), sb = static_cast<int>(j % kStB);
-                if (!mbar_wait(emptyA + sa, static_cast<uint32_t>(((j / kStA) & 1) ^ 1), kSpin)) {
-                    report(a.err, MOE_DEVERR_TIMEOUT);
-                    abort_s = 1;
-                    break;
-                }
-                const uint8_t *raw = sRaw + sb * Cfg::RAW_STAGE + static_cast<size_t>(row) * Cfg::RAW_ROW;
-#pragma unroll
-                for (int mat = 0; mat < Cfg::NA; ++mat)
-                    dequant_row<BITS>(raw + mat * Cfg::SEG,
-                                      smem_addr(sA + sa * Cfg::A_STAGE + static_cast<size_t>(mat) * kBM * 128 +
-                                                static_cast<size_t>(row) * 128),
-                                      row);
-                fence_proxy_async();
-                mbar_arrive(fullA + sa);
-                mbar_arrive(fullB + sb);
-                if (s + kLook < nk) issue(s + kLook, j + kLook);
+                for (int q = 0; q < Cfg::RAW_CODE / 16; ++q) cp_async16(dst + q * 16, src + q * 16, 16);
+            } else {
+                asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dst), "l"(src) : "memory");
             }
-            it = j0 + nk;
+            cp_async4(dst + Cfg::RAW_CODE, scl + m * nsc + 2 * s);
+        };
+        for (int p = 0; p < L; ++p) {             // prologue: one commit group per k-step
+            issue_raw(p);
+            cp_async_commit();
+        }
+        for (long j = 0; j < J && !abort_s; ++j) {
+            cp_async_wait<L - 1>();              // this thread's codes of k-step j have landed
+            const int sa = static_cast<int>(j % SA);
+            if (!mbar_wait(emptyA + sa, static_cast<uint32_t>(((j / SA) & 1) ^ 1), kSpin)) {
+                fail();
+                break;
+            }
+            const uint8_t *raw = sRaw + (j % L) * Cfg::RAW_STAGE + static_cast<size_t>(tid) * Cfg::SEG;
+            const __half2 s01 = *reinterpret_cast<const __half2 *>(raw + Cfg::RAW_CODE);
+            const uint32_t a_row = smem_addr(sA + sa * Cfg::A_STAGE +
+                                             static_cast<size_t>(GATEUP ? part : 0) * kBM * 128 +
+                                             static_cast<size_t>(row) * 128);
+            if (GATEUP) {
+                dequant_block<BITS>(raw, __low2half2(s01), a_row, 0, row & 7);
+                dequant_block<BITS>(raw + 4 * BITS, __high2half2(s01), a_row, 4, row & 7);
+            } else {
+                dequant_block<BITS>(raw, part ? __high2half2(s01) : __low2half2(s01), a_row, 4 * part, row & 7);
+            }
+            fence_proxy_async();
+            mbar_arrive(fullA + sa);
+            issue_raw(j + L);                    // into the slot just read
+            cp_async_commit();
         }
         cp_async_wait<0>();
-    } else if (warp < 8) {
+    } else if (warp >= 13) {
+        // --------------------------------------------------- token rows
+        // Loader warp lw copies rows lw*MAXN/2 .. of each tile: lane = 8 x row
+        // + 16-byte chunk.  Its token indices live in a warp-private table.
+        const int lw = warp - 13;
+        constexpr int HALF = MAXN / 2;
+        int32_t *tok = tok_s + lw * HALF;
+        const uint8_t *bsrc = GATEUP ? reinterpret_cast<const uint8_t *>(a.x16)
+                                     : reinterpret_cast<const uint8_t *>(a.h16);
+        const size_t brow = static_cast<size_t>(K) * 2;
+        const int c = lane & 7;
+        int cur = -1;
+        TileInfo bt{};
+        for (long j = 0; j < J && !abort_s; ++j) {
+            const int i = static_cast<int>(j / nk), s = static_cast<int>(j % nk);
+            if (i != cur) {
+                bt = tile_of(i);
+                cur = i;
+                __syncwarp();
+                for (int nl = lane; nl < HALF; nl += 32) {
+                    const int n = lw * HALF + nl;
+                    int v = 0;
+                    if (n < bt.nvalid) {
+                        if (GATEUP)
+                            v = min(max(bt.G.row0 >= 0 ? a.perm_src[bt.G.row0 + bt.n0 + n] : bt.n0 + n, 0), a.T - 1);
+                        else
+                            v = (bt.G.row0 >= 0 ? bt.G.row0 : a.T * a.k) + bt.n0 + n;
+                    }
+                    tok[nl] = v;
+                }
+                __syncwarp();
+            }
+            const int sb = static_cast<int>(j % SB);
+            if (!mbar_wait(emptyB + sb, static_cast<uint32_t>(((j / SB) & 1) ^ 1), kSpin)) {
+                fail();
+                break;
+            }
+            const uint32_t bdst = smem_addr(sB + sb * Cfg::B_STAGE);
+#pragma unroll 4
+            for (int nl = lane >> 3; nl < HALF; nl += 4) {
+                const int n = lw * HALF + nl;
+                if (n < bt.N) {
+                    const uint8_t *src = bsrc + static_cast<size_t>(tok[nl]) * brow + static_cast<size_t>(s) * 128 + c * 16;
+                    cp_async16(bdst + n * 128 + ((c ^ (n & 7)) << 4), src, n < bt.nvalid ? 16u : 0u);
+                }
+            }
+            asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_addr(fullB + sb))
+                         : "memory");
+        }
+        cp_async_wait<0>();
+    } else if (warp < 12) {
         // -------------------------------------------------------- epilogue
         const int q = warp & 3;                   // TMEM lanes 32q .. 32q+31
         const int m = 32 * q + lane;              // weight row within the tile
-        long tile_it = 0;
-        for (int t = blockIdx.x; t < total && !abort_s; t += gridDim.x, ++tile_it) {
-            int g, n0, m0;
-            decode_tile(t, g, n0, m0);
-            const GroupInfo G = group_info(a, g, n_act);
-            const int nvalid = min(kMaxN, G.n - n0);
-            if (!mbar_wait(acc_full, static_cast<uint32_t>(tile_it & 1), kSpin)) {
-                report(a.err, MOE_DEVERR_TIMEOUT);
-                abort_s = 1;
+        for (int i = 0; i < n_my && !abort_s; ++i) {
+            const TileInfo ti = tile_of(i);
+            const int b = i % ACC;
+            if (!mbar_wait(accF + b, static_cast<uint32_t>((i / ACC) & 1), kSpin)) {
+                fail();
                 break;
             }
             tc_fence_after();
-            const uint32_t lane_base = tmem + (static_cast<uint32_t>(32 * q) << 16);
-            for (int c0 = 0; c0 < nvalid; c0 += 16) {
+            const uint32_t base = tmem + (static_cast<uint32_t>(32 * q) << 16) + b * NA * MAXN;
+            for (int c0 = 0; c0 < ti.nvalid; c0 += 16) {
                 float gv[16], uv[16];
-                tmem_ld16(lane_base + c0, gv);
-                if (GATEUP) tmem_ld16(lane_base + 256 + c0, uv);
+                tmem_ld16(base + c0, gv);
+                if (GATEUP) tmem_ld16(base + MAXN + c0, uv);
                 tmem_ld_wait();
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const int n = c0 + i;
-                    if (n >= nvalid) break;
+                for (int e = 0; e < 16; ++e) {
+                    const int n = c0 + e;
+                    if (n >= ti.nvalid) break;
                     if (GATEUP) {
-                        const float h = gv[i] / (1.0f + expf(-gv[i])) * uv[i];
-                        const size_t r = static_cast<size_t>(G.row0 >= 0 ? G.row0 : a.T * a.k) + n0 + n;
-                        a.h16[r * a.I + m0 + m] = __float2half_rn(h);
+                        const float h = gv[e] / (1.0f + expf(-gv[e])) * uv[e];
+                        const size_t r = static_cast<size_t>(ti.G.row0 >= 0 ? ti.G.row0 : a.T * a.k) + ti.n0 + n;
+                        a.h16[r * a.I + ti.m0 + m] = __float2half_rn(h);
                     } else {
-                        float *dst = G.row0 >= 0 ? a.y_perm + (static_cast<size_t>(G.row0) + n0 + n) * a.H
-                                                 : a.y_shared + (static_cast<size_t>(n0) + n) * a.H;
-                        dst[m0 + m] = gv[i];
+                        float *dst = ti.G.row0 >= 0 ? a.y_perm + (static_cast<size_t>(ti.G.row0) + ti.n0 + n) * a.H
+                                                    : a.y_shared + (static_cast<size_t>(ti.n0) + n) * a.H;
+                        dst[ti.m0 + m] = gv[e];
                     }
                 }
             }
             tc_fence_before();
-            mbar_arrive(acc_empty);
+            mbar_arrive(accE + b);
         }
     } else {
         // ------------------------------------------------------ MMA issuer
-        long it = 0, tile_it = 0;
-        for (int t = blockIdx.x; t < total && !abort_s; t += gridDim.x, ++tile_it) {
-            int g, n0, m0;
-            decode_tile(t, g, n0, m0);
-            const GroupInfo G = group_info(a, g, n_act);
-            const int nvalid = min(kMaxN, G.n - n0);
-            const int N = (nvalid + 15) & ~15;
-            const uint32_t idesc = idesc_f16_f32(kBM, N);
+        for (int i = 0; i < n_my && !abort_s; ++i) {
+            const TileInfo ti = tile_of(i);
+            const uint32_t idesc = idesc_f16_f32(kBM, ti.N);
+            const int b = i % ACC;
             if (lane == 0) {
-                if (!mbar_wait(acc_empty, static_cast<uint32_t>((tile_it & 1) ^ 1), kSpin)) {
-                    report(a.err, MOE_DEVERR_TIMEOUT);
-                    abort_s = 1;
-                }
+                if (!mbar_wait(accE + b, static_cast<uint32_t>(((i / ACC) & 1) ^ 1), kSpin)) fail();
                 tc_fence_after();
                 for (int s = 0; s < nk && !abort_s; ++s) {
-                    const long j = it + s;
-                    const int sa = static_cast<int>(j % kStA), sb = static_cast<int>(j % kStB);
-                    if (!mbar_wait(fullA + sa, static_cast<uint32_t>((j / kStA) & 1), kSpin) ||
-                        !mbar_wait(fullB + sb, static_cast<uint32_t>((j / kStB) & 1), kSpin)) {
-                        report(a.err, MOE_DEVERR_TIMEOUT);
-                        abort_s = 1;
+                    const long j = static_cast<long>(i) * nk + s;
+                    const int sa = static_cast<int>(j % SA), sb = static_cast<int>(j % SB);
+                    if (!mbar_wait(fullA + sa, static_cast<uint32_t>((j / SA) & 1), kSpin) ||
+                        !mbar_wait(fullB + sb, static_cast<uint32_t>((j / SB) & 1), kSpin)) {
+                        fail();
                         break;
                     }
                     tc_fence_after();
@@ -408,19 +417,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(GemmArgs a) {
                     for (int kk = 0; kk < kBK / 16; ++kk) {
                         const uint64_t bdesc = desc_sw128(b_addr + kk * 32);
 #pragma unroll
-                        for (int mat = 0; mat < Cfg::NA; ++mat) {
+                        for (int mat = 0; mat < NA; ++mat) {
                             const uint32_t a_addr =
                                 smem_addr(sA + sa * Cfg::A_STAGE + static_cast<size_t>(mat) * kBM * 128) + kk * 32;
-                            mma_f16(tmem + mat * 256, desc_sw128(a_addr), bdesc, idesc, (s | kk) != 0);
+                            mma_f16(tmem + b * NA * MAXN + mat * MAXN, desc_sw128(a_addr), bdesc, idesc,
+                                    (s | kk) != 0);
                         }
                     }
                     mma_commit(emptyA + sa);
                     mma_commit(emptyB + sb);
                 }
-                mma_commit(acc_full);
+                mma_commit(accF + b);
             }
             __syncwarp();
-            it += nk;
         }
         // every MMA issued has completed before TMEM is released
         if (lane == 0) {
@@ -431,9 +440,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(GemmArgs a) {
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 8) {
+    if (warp == 12) {
         tc_fence_after();
-        tmem_dealloc(tmem, 512);
+        tmem_dealloc(tmem, Cfg::TMEM_COLS);
     }
 }
 
@@ -462,16 +471,23 @@ size_t gemm_ws_bytes(int bits, int T, int k, int H, int I, int E) {
 
 bool gemm_supported(int T, int k, int E) { return (T * k < E ? T * k : E) + 1 <= kMaxGroups; }
 
-template <int BITS, bool GATEUP>
+template <int BITS, bool GATEUP, int MAXN>
 static int launch_k_gemm(const GemmArgs &a, cudaStream_t s) {
-    using Cfg = GemmCfg<BITS, GATEUP>;
-    int rc = cuda_status(cudaFuncSetAttribute(k_gemm<BITS, GATEUP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    using Cfg = GemmCfg<BITS, GATEUP, MAXN>;
+    int rc = cuda_status(cudaFuncSetAttribute(k_gemm<BITS, GATEUP, MAXN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                               static_cast<int>(Cfg::SMEM)),
                          "gemm smem attribute");
     if (rc) return rc;
-    k_gemm<BITS, GATEUP><<<num_sms(), kGemmThreads, Cfg::SMEM, s>>>(a);
+    k_gemm<BITS, GATEUP, MAXN><<<num_sms(), kGemmThreads, Cfg::SMEM, s>>>(a);
     count_launches(1);
     return cuda_status(cudaGetLastError(), "gemm launch");
+}
+
+template <int BITS>
+static int launch_pair(const GemmArgs &a, bool large, cudaStream_t s) {
+    int rc = large ? launch_k_gemm<BITS, true, 256>(a, s) : launch_k_gemm<BITS, true, 64>(a, s);
+    if (rc) return rc;
+    return large ? launch_k_gemm<BITS, false, 256>(a, s) : launch_k_gemm<BITS, false, 64>(a, s);
 }
 
 int launch_gemm(int bits, const uint8_t *const *blobs, const int32_t *offsets, const int32_t *active,
@@ -501,9 +517,10 @@ int launch_gemm(int bits, const uint8_t *const *blobs, const int32_t *offsets, c
         k_to_half<<<blocks, 256, 0, s>>>(x, x_dtype == MOE_BF16, n, const_cast<__half *>(a.x16));
         count_launches(1);
     }
-    int rc = bits == 4 ? launch_k_gemm<4, true>(a, s) : launch_k_gemm<2, true>(a, s);
-    if (rc) return rc;
-    return bits == 4 ? launch_k_gemm<4, false>(a, s) : launch_k_gemm<2, false>(a, s);
+    // tiles of 256 tokens once experts hold more than ~48 tokens on average, else 64
+    const int groups = T * k < E ? T * k : E;
+    const bool large = static_cast<long>(T) * k > 48L * (groups > 0 ? groups : 1);
+    return bits == 4 ? launch_pair<4>(a, large, s) : launch_pair<2>(a, large, s);
 }
 
 }  // namespace moe

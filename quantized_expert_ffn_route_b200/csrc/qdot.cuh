@@ -113,10 +113,10 @@ __device__ __forceinline__ void load_scales(const __half *row_scales, int c, boo
     }
 }
 
-// Stages nt activation rows (fp32 or bf16, rows[t] -> row t) as fp32 pieces
-// plus the pre-scaled block sums; rows nt..NTS-1 are zero.
-template <int BITS>
-__device__ void stage_rows(float4 *xs, float *cs, int NTS, int nt, int K, const void *const *rows, int bf16) {
+// Stages nt activation rows (fp32 or bf16, row_of(t) -> row t) as fp32
+// pieces plus the pre-scaled block sums; rows nt..NTS-1 are zero.
+template <int BITS, class RowOf>
+__device__ void stage_rows_fn(float4 *xs, float *cs, int NTS, int nt, int K, RowOf row_of, int bf16) {
     using Q = QT<BITS>;
     const int nch = K / Q::EPC;
     const int g4n = K / 4;
@@ -125,8 +125,8 @@ __device__ void stage_rows(float4 *xs, float *cs, int NTS, int nt, int K, const 
         const int c = (4 * g4) / Q::EPC, q = ((4 * g4) % Q::EPC) / 4;
         float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
         if (t < nt)
-            v = bf16 ? load4(static_cast<const __nv_bfloat16 *>(rows[t]) + 4 * g4)
-                     : load4(static_cast<const float *>(rows[t]) + 4 * g4);
+            v = bf16 ? load4(static_cast<const __nv_bfloat16 *>(row_of(t)) + 4 * g4)
+                     : load4(static_cast<const float *>(row_of(t)) + 4 * g4);
         xs[(t * Q::PPC + q) * nch + c] = v;
     }
     __syncthreads();
@@ -143,6 +143,69 @@ __device__ void stage_rows(float4 *xs, float *cs, int NTS, int nt, int K, const 
         cs[t * nblk + b] = static_cast<float>(128 + Q::HALF) * s;
     }
     __syncthreads();
+}
+
+template <int BITS>
+__device__ void stage_rows(float4 *xs, float *cs, int NTS, int nt, int K, const void *const *rows, int bf16) {
+    stage_rows_fn<BITS>(xs, cs, NTS, nt, K, [rows](int t) { return rows[t]; }, bf16);
+}
+
+}  // namespace moe
+
+namespace moe {
+
+// ---------------------------------------------------------------------------
+// Single-token variant with the activation pieces of one chunk in registers,
+// so several weight rows can reuse them: returns, per quant block of the
+// chunk, sum_i f_i x_i with f_i = 1 + q_i/128, accumulated with packed fp32
+// FMAs (two lanes of a float2 per instruction).
+template <int BITS>
+__device__ __forceinline__ void chunk_fx(const uint4 &code, const float4 (&xp)[QT<BITS>::PPC],
+                                         float (&out)[QT<BITS>::BPC]) {
+    const uint32_t words[4] = {code.x, code.y, code.z, code.w};
+    if constexpr (BITS == 4) {
+        float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            const uint32_t L = (words[m] & 0x0F0F0F0Fu) | 0x80808080u;
+            const uint32_t Hh = ((words[m] >> 4) & 0x0F0F0F0Fu) | 0x80808080u;
+            const float4 a = xp[m], b = xp[4 + m];   // elements 4m..4m+3 (low nibbles), 16+4m.. (high)
+            acc = __ffma2_rn(make_float2(magic(L, 0), magic(Hh, 0)), make_float2(a.x, b.x), acc);
+            acc = __ffma2_rn(make_float2(magic(L, 1), magic(Hh, 1)), make_float2(a.y, b.y), acc);
+            acc = __ffma2_rn(make_float2(magic(L, 2), magic(Hh, 2)), make_float2(a.z, b.z), acc);
+            acc = __ffma2_rn(make_float2(magic(L, 3), magic(Hh, 3)), make_float2(a.w, b.w), acc);
+        }
+        out[0] = acc.x + acc.y;
+    } else {
+        float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+        for (int wi = 0; wi < 4; ++wi) {
+            const int beta = wi >> 1, m = wi & 1;
+#pragma unroll
+            for (int s = 0; s < 4; s += 2) {
+                const uint32_t L0 = ((words[wi] >> (2 * s)) & 0x03030303u) | 0x80808080u;
+                const uint32_t L1 = ((words[wi] >> (2 * s + 2)) & 0x03030303u) | 0x80808080u;
+                const float4 a = xp[8 * beta + 2 * s + m], b = xp[8 * beta + 2 * (s + 1) + m];
+                float2 v = acc[beta];
+                v = __ffma2_rn(make_float2(magic(L0, 0), magic(L1, 0)), make_float2(a.x, b.x), v);
+                v = __ffma2_rn(make_float2(magic(L0, 1), magic(L1, 1)), make_float2(a.y, b.y), v);
+                v = __ffma2_rn(make_float2(magic(L0, 2), magic(L1, 2)), make_float2(a.z, b.z), v);
+                v = __ffma2_rn(make_float2(magic(L0, 3), magic(L1, 3)), make_float2(a.w, b.w), v);
+                acc[beta] = v;
+            }
+        }
+        out[0] = acc[0].x + acc[0].y;
+        out[1] = acc[1].x + acc[1].y;
+    }
+}
+
+// dot += sum over the chunk's blocks of d_b * (128 * fx_b - cs_b)
+template <int BITS>
+__device__ __forceinline__ float chunk_finish(const float (&fx)[QT<BITS>::BPC], const float (&d)[QT<BITS>::BPC],
+                                              const float (&cs)[QT<BITS>::BPC], float dot) {
+#pragma unroll
+    for (int b = 0; b < QT<BITS>::BPC; ++b) dot = fmaf(d[b], fmaf(128.f, fx[b], -cs[b]), dot);
+    return dot;
 }
 
 }  // namespace moe

@@ -443,7 +443,7 @@ def bench_layer(args, world, rank, pk):
 def host_link_gbs(nbytes=1 << 30):
     """Pinned host -> device copy bandwidth (best of 3)."""
     import torch
-    h = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
+    h = torch.empty(nbytes, dtype=torch.uint8, pin_memory=True)
     d = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
     best = 0.0
     for _ in range(3):
@@ -469,7 +469,16 @@ def bench_paging(args, world, rank, pk):
     stride = (nb + 255) // 256 * 256
     link = host_link_gbs()
     # page-locked pool of all experts (512 distinct blobs repeated: only bytes moved matter here)
-    pool = torch.empty(E * stride, dtype=torch.uint8).pin_memory()
+    need = E * stride
+    try:
+        import psutil
+        avail = psutil.virtual_memory().available
+    except Exception:
+        avail = None
+    if avail is not None and avail < need + (16 << 30):
+        raise SystemExit(f"paging: {need / 2**30:.1f} GiB of page-locked host memory needed, "
+                         f"{avail / 2**30:.1f} GiB available")
+    pool = torch.empty(need, dtype=torch.uint8, pin_memory=True)
     pv = pool.view(E, stride)
     bt = torch.from_numpy(base.blobs)
     for e0 in range(0, E, 512):

@@ -68,7 +68,7 @@ typedef struct CUstream_st *moe_stream_t;   /* same type as cudaStream_t */
 #define MOE_BF16 1
 
 /* expert FFN modes */
-#define MOE_MODE_AUTO 0   /* GEMV when T <= 16, else GEMM */
+#define MOE_MODE_AUTO 0   /* GEMV when T <= 16 and the shape suits it, else GEMM */
 #define MOE_MODE_GEMV 1   /* CUDA-core kernels, fp32 math, any T (slow for large T) */
 #define MOE_MODE_GEMM 2   /* tcgen05 tensor-core grouped GEMM, fp16 operands */
 
@@ -78,6 +78,7 @@ typedef struct CUstream_st *moe_stream_t;   /* same type as cudaStream_t */
 #define MOE_DEVERR_NONFINITE 4u      /* a selected logit was NaN or +inf */
 #define MOE_DEVERR_BAD_ROW 8u        /* offsets/perm_src inconsistent */
 #define MOE_DEVERR_TIMEOUT 16u       /* a bounded in-kernel wait ran out */
+#define MOE_DEVERR_WORKSPACE 32u     /* moe_layer_decode: the workspace ticket counter was not zero */
 
 /* Thread-local message of the last failing call ("" if none). */
 const char *moe_last_error(void);
@@ -154,7 +155,9 @@ int moe_permute(const int32_t *topk_ids, int T, int k, int E, int32_t *expert_of
  *  x        device [T,H] dtype x_dtype.
  *  y_perm   device [T*k, H] fp32 out.  y_shared device [T,H] fp32 out (or
  *           NULL when shared_blob is NULL).
- *  mode     MOE_MODE_AUTO | _GEMV | _GEMM.
+ *  mode     MOE_MODE_AUTO | _GEMV | _GEMM.  GEMV needs H <= 2048 and I/32
+ *           (4-bit) or I/64 (2-bit) in {2, 4, 8, 16, 32}; GEMM needs at most
+ *           4095 groups (min(E, T*k) + shared).  Else MOE_EINVAL.
  *  ws       at least moe_expert_ffn_ws_size(bits,T,k,H,I,E,mode) bytes.
  * _q4 reads 4-bit blobs, _q2 2-bit blobs. */
 size_t moe_expert_ffn_ws_size(int bits, int T, int k, int H, int I, int E, int mode);
@@ -177,16 +180,23 @@ int moe_expert_ffn_q2(const void *const *expert_blobs, const int32_t *expert_off
  * moe_expert_ffn_q4/q2 (GEMV mode) -> moe_combine (Strata article, section 2
  * item 2: only the experts the router picks are computed; at one token the
  * step is bound by streaming those experts' weights).  Three kernels chained
- * with programmatic dependent launch (route in one thread-block cluster, then
- * gate/up, then down + combine); no in-kernel waits spin.
+ * with programmatic dependent launch (route: logits over E/4 CTAs, the last
+ * CTA to finish selects; then gate/up; then down + combine); no in-kernel
+ * waits spin.
  *  x [H] (x_dtype), w_router [E,H] (w_dtype) or NULL with logits_in [E];
  *  expert_blobs device [E] blob pointers; shared_blob or NULL;
  *  topk_ids [k] int32 out, topk_w [k] fp32 out, logits_out [E] or NULL
  *  (written only when the logits are computed here), y [H] fp32 out.
- *  ws: moe_layer_decode_ws_size() bytes of scratch (no initialisation needed).
+ *  ws: moe_layer_decode_ws_size() bytes of scratch, zero-filled before its
+ *  first use with this call (e.g. one cudaMemsetAsync after allocation); it
+ *  holds a ticket counter that every completed call leaves at zero.  A
+ *  counter found non-zero sets MOE_DEVERR_WORKSPACE (the outputs of that
+ *  call are then not valid).  Calls sharing one ws must not overlap.
  * Supported shapes (else MOE_EINVAL: use the separate calls): E <= 1024,
- * k <= 32, H <= 2048, I a multiple of 128 with I/32 (4-bit) or I/64 (2-bit)
- * a power of two <= 32, and k + 1 <= 8 * 32 / (that number). */
+ * k <= 32, H <= 2048 and a multiple of 128, I a multiple of 128 with I/32
+ * (4-bit) or I/64 (2-bit) in {4, 8, 16, 32}, and the down kernel's tasks,
+ * (k + 1) * (rows per block) / (32 / that number), at most 64 (rows per
+ * block 8 when k + 1 <= 16, else 4). */
 size_t moe_layer_decode_ws_size(int E, int k, int I);
 int moe_layer_decode(int bits, const void *x, int x_dtype, const void *w_router, int w_dtype,
                      const float *bias, const float *logits_in, const void *const *expert_blobs,
@@ -205,8 +215,9 @@ int moe_layer_decode(int bits, const void *x, int x_dtype, const void *w_router,
  * scratch (the fp32 intermediate h, T*(k+1)*I*4 bytes) comes from one array
  * built into the library of moe_expert_ffn_noalloc_max_bytes() bytes (8 MiB),
  * which every GPU that loads the library holds until the process exits.
- *  - Calls needing more scratch than that, or H/I outside [128, 2048], are
- *    rejected with MOE_EINVAL before anything is launched.
+ *  - Calls needing more scratch than that, H/I outside [128, 2048], or an I
+ *    that GEMV mode does not take (see above), are rejected with MOE_EINVAL
+ *    before anything is launched.
  *  - It never calls cudaMalloc, cudaFree or any allocating routine.
  *  - The first call on a device looks up the array's device address (once per
  *    device, with that device current); make that first call before any stream

@@ -150,7 +150,12 @@ int moe_route_topk(const void *x, int x_dtype, const void *w_router, int w_dtype
     const float *logits = nullptr;
     if (w_router) {
         float *out = logits_out ? logits_out : static_cast<float *>(ws);
-        launch_router_logits(x, x_dtype, w_router, w_dtype, bias, T, H, E, out, st);
+        if (router_mma_supported(x_dtype, w_dtype, T, H)) {
+            int rc = launch_router_mma(x, w_router, bias, T, H, E, out, err, st);
+            if (rc) return rc;
+        } else {
+            launch_router_logits(x, x_dtype, w_router, w_dtype, bias, T, H, E, out, st);
+        }
         logits = out;
     } else {
         logits = logits_in;
@@ -197,14 +202,14 @@ int moe_permute(const int32_t *topk_ids, int T, int k, int E, int32_t *expert_of
 }
 
 // ------------------------------------------------------------- expert FFN
-static int resolve_mode(int mode, int T) {
-    if (mode == MOE_MODE_AUTO) return T <= 16 ? MOE_MODE_GEMV : MOE_MODE_GEMM;
+static int resolve_mode(int mode, int T, int bits, int H, int I) {
+    if (mode == MOE_MODE_AUTO) return T <= 16 && gemv_supported(bits, H, I) ? MOE_MODE_GEMV : MOE_MODE_GEMM;
     return mode;
 }
 
 size_t moe_expert_ffn_ws_size(int bits, int T, int k, int H, int I, int E, int mode) {
     if ((bits != 2 && bits != 4) || T <= 0 || k <= 0 || H <= 0 || I <= 0 || E <= 0) return 0;
-    mode = resolve_mode(mode, T);
+    mode = resolve_mode(mode, T, bits, H, I);
     if (mode == MOE_MODE_GEMM) return gemm_ws_bytes(bits, T, k, H, I, E);
     return gemv_ws_bytes(T, k, I);
 }
@@ -228,11 +233,13 @@ static int expert_ffn(int bits, const void *const *expert_blobs, const int32_t *
     REQUIRE(aligned16(x) && aligned16(y_perm) && (!y_shared || aligned16(y_shared)) &&
                 (!shared_blob || aligned16(shared_blob)) && aligned16(expert_blobs),
             "x/y_perm/y_shared/shared_blob/expert_blobs must be 16-byte aligned");
-    mode = resolve_mode(mode, T);
+    mode = resolve_mode(mode, T, bits, H, I);
     if (mode == MOE_MODE_GEMV) {
-        REQUIRE(H <= 2048 && I <= 2048, "GEMV mode supports H, I <= 2048 (got H=%d, I=%d)", H, I);
+        REQUIRE(gemv_supported(bits, H, I),
+                "GEMV mode needs H <= 2048 and I/32 (4-bit) or I/64 (2-bit) in {2, 4, 8, 16, 32} (got H=%d, I=%d)",
+                H, I);
     } else {
-        REQUIRE(gemm_supported(T, k, E), "GEMM mode supports at most 2047 active experts (min(E, T*k))");
+        REQUIRE(gemm_supported(bits, T, k, H, I, E), "GEMM mode supports at most 4095 active experts (min(E, T*k))");
     }
     const size_t need = moe_expert_ffn_ws_size(bits, T, k, H, I, E, mode);
     REQUIRE(ws && ws_bytes >= need && aligned16(ws), "workspace too small: need %zu bytes", need);

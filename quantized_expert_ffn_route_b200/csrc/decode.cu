@@ -2,19 +2,21 @@
 // programmatic dependent launch (each starts while its predecessor runs and
 // waits with griddepcontrol only where it reads the predecessor's results).
 //
-//   1. logits (one warp per router row, spread over E/4 SMs).
+//   1. route (one warp per router row, E/4 CTAs): logits; the last CTA to
+//      finish (a ticket counter in the workspace) selects the top-k and
+//      writes ids and gates.  With caller-given logits it is one CTA that
+//      only selects.
 //   2. gate/up (all selected experts + the shared expert, 16 rows per CTA):
-//      every routed CTA selects the top-k from the logits itself (a block
-//      top-k of a few hundred cycles, cheaper than another kernel boundary),
-//      then h_g[i] = silu(Wg_g[i] . x) * (Wu_g[i] . x); CTA 0 publishes ids
-//      and gates.  The shared expert's CTAs never wait for the logits.
+//      h_g[i] = silu(Wg_g[i] . x) * (Wu_g[i] . x).  The shared expert's CTAs
+//      never wait for the route kernel.
 //   3. down + combine (a few output rows per CTA, all groups; each lane one
 //      chunk of one row): every code load is issued before h is staged, then
 //      y[r] = sum_j w_j (Wd_{e_j}[r] . h_j) + Wd_shared[r] . h_shared, summed
 //      in slot order.
 // At one token the step streams ~20 MB of expert weights with little
-// arithmetic, so everything here is about keeping loads in flight: every warp
-// issues all of its weight loads before it touches shared memory.
+// arithmetic, so the kernels keep every weight load of a warp in flight
+// before touching shared memory, and every shape-dependent index is a
+// compile-time shift.
 //
 // Strata article, section 2 item 2: the router's choice decides which
 // experts are computed; only those experts' weights are streamed.
@@ -33,10 +35,13 @@ __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.lau
 
 __host__ __device__ inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
-// Workspace layout (bytes): ids [32] int32 | gates [32] fp32 | logits [E] | h [(k+1) * I]
+// Workspace layout (bytes): ids [32] int32 @0 | gates [32] fp32 @128 |
+// ticket counter @256 | logits [E] @512 | h [(k+1) * I] fp32 (256-aligned).
+// The counter must be zero before the first call; every call leaves it zero.
 struct DecodeWs {
     int32_t *ids;
     float *gates;
+    unsigned *ticket;
     float *logits;
     float *h;
 };
@@ -45,8 +50,9 @@ __host__ __device__ inline DecodeWs decode_ws(void *ws, int E) {
     DecodeWs w;
     w.ids = reinterpret_cast<int32_t *>(p);
     w.gates = reinterpret_cast<float *>(p + 128);
-    w.logits = reinterpret_cast<float *>(p + 256);
-    w.h = reinterpret_cast<float *>(p + 256 + ((static_cast<size_t>(E) * 4 + 255) / 256) * 256);
+    w.ticket = reinterpret_cast<unsigned *>(p + 256);
+    w.logits = reinterpret_cast<float *>(p + 512);
+    w.h = reinterpret_cast<float *>(p + 512 + ((static_cast<size_t>(E) * 4 + 255) / 256) * 256);
     return w;
 }
 
@@ -68,115 +74,207 @@ struct DecodeArgs {
     unsigned *err;
 };
 
-// ------------------------------------------------------------ 1. logits
-// One warp per router row, kLogitRows rows per CTA, so the E rows are read by
-// E / kLogitRows SMs at once; every lane issues all of its weight loads
-// before it stages x.
-constexpr int kLogitRows = 4;
-
-__global__ void __launch_bounds__(kLogitRows * 32) k_dec_logits(DecodeArgs a) {
-    __shared__ __align__(16) float xs[2048];
-    pdl_trigger();                                       // the gate/up kernel may start its prologue
-    const int H = a.H, E = a.E;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int e = blockIdx.x * kLogitRows + warp;
-    uint4 w[8];                                          // bf16 rows: 8 x 16 B per lane covers H <= 2048
-    if (a.w_bf16) {
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int hh = lane * 8 + 256 * j;
-            w[j] = make_uint4(0, 0, 0, 0);
-            if (e < E && hh < H)
-                w[j] = ldg_stream(static_cast<const __nv_bfloat16 *>(a.w_router) + static_cast<size_t>(e) * H + hh);
-        }
-    }
-    for (int i = threadIdx.x; i < H / 4; i += blockDim.x)
-        reinterpret_cast<float4 *>(xs)[i] = a.x_bf16 ? load4(static_cast<const __nv_bfloat16 *>(a.x) + 4 * i)
-                                                     : load4(static_cast<const float *>(a.x) + 4 * i);
-    __syncthreads();
-    if (e >= E) return;
-    float s = 0.f;
-    if (a.w_bf16) {
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int hh = lane * 8 + 256 * j;
-            if (hh < H) {
-                const float4 x0 = reinterpret_cast<const float4 *>(xs + hh)[0];
-                const float4 x1 = reinterpret_cast<const float4 *>(xs + hh)[1];
-                const uint4 u = w[j];
-                s = fmaf(__uint_as_float(u.x << 16), x0.x, s);
-                s = fmaf(__uint_as_float(u.x & 0xffff0000u), x0.y, s);
-                s = fmaf(__uint_as_float(u.y << 16), x0.z, s);
-                s = fmaf(__uint_as_float(u.y & 0xffff0000u), x0.w, s);
-                s = fmaf(__uint_as_float(u.z << 16), x1.x, s);
-                s = fmaf(__uint_as_float(u.z & 0xffff0000u), x1.y, s);
-                s = fmaf(__uint_as_float(u.w << 16), x1.z, s);
-                s = fmaf(__uint_as_float(u.w & 0xffff0000u), x1.w, s);
-            }
-        }
-    } else {
-        for (int hh = lane * 4; hh < H; hh += 128) {
-            const float4 wv = load4(static_cast<const float *>(a.w_router) + static_cast<size_t>(e) * H + hh);
-            const float4 xv = reinterpret_cast<const float4 *>(xs + hh)[0];
-            s = fmaf(wv.x, xv.x, s); s = fmaf(wv.y, xv.y, s);
-            s = fmaf(wv.z, xv.z, s); s = fmaf(wv.w, xv.w, s);
-        }
-    }
-    s = warp_sum(s);
-    if (lane == 0) {
-        const float l = s + (a.bias ? a.bias[e] : 0.f);
-        a.ws.logits[e] = l;
-        if (a.logits_out) a.logits_out[e] = l;
-    }
-}
-
-// Top-k (k <= 32) of E <= 1024 logits by one block of kDecThreads threads.
-// Each warp first takes the k best of its keys (k rounds of two warp max
-// reductions: the value key, then among equal values the larger low word,
-// i.e. the lower id), then warp 0 takes the k best of those 8k candidates.
-// sel[0..k-1] receives the selection keys in rank order.
+// ------------------------------------------------------------ top-k
+// k best of N keys per lane by one warp.  Each lane first sorts its keys
+// (descending, a bitonic network on registers); then every round the warp
+// takes the largest head: a max reduction of the value halves, and only when
+// several heads share that value a second one of the low words (the larger
+// low word is the lower id).  The winning lane pops its head.  dst[r]
+// receives the rank-r key.
 template <int N>
 __device__ __forceinline__ void warp_take(uint64_t (&keys)[N], int k, int lane, uint64_t *dst) {
-    uint64_t best = 0ull;
 #pragma unroll
-    for (int q = 0; q < N; ++q) best = keys[q] > best ? keys[q] : best;
-    for (int r = 0; r < k; ++r) {
-        const uint32_t hi = __reduce_max_sync(0xffffffffu, static_cast<uint32_t>(best >> 32));
-        const uint32_t lo =
-            __reduce_max_sync(0xffffffffu, static_cast<uint32_t>(best >> 32) == hi ? static_cast<uint32_t>(best) : 0u);
-        const uint64_t win = (static_cast<uint64_t>(hi) << 32) | lo;
-        if (lane == 0) dst[r] = win;
-        if (best == win && win != 0ull) {                // keys are distinct: exactly one lane holds it
-            best = 0ull;
+    for (int k2 = 2; k2 <= N; k2 <<= 1)
 #pragma unroll
-            for (int q = 0; q < N; ++q) {
-                if (keys[q] == win) keys[q] = 0ull;
-                best = keys[q] > best ? keys[q] : best;
+        for (int j = k2 >> 1; j > 0; j >>= 1)
+#pragma unroll
+            for (int i = 0; i < N; ++i) {
+                const int l = i ^ j;
+                if (l > i) {
+                    const bool desc = (i & k2) == 0;
+                    const uint64_t a = keys[i], b = keys[l];
+                    if (desc ? a < b : a > b) {
+                        keys[i] = b;
+                        keys[l] = a;
+                    }
+                }
             }
+    for (int r = 0; r < k; ++r) {
+        const uint64_t head = keys[0];
+        const uint32_t hv = static_cast<uint32_t>(head >> 32);
+        const uint32_t hi = __reduce_max_sync(0xffffffffu, hv);
+        const unsigned tied = __ballot_sync(0xffffffffu, hv == hi);
+        int winner;
+        if (__popc(tied) == 1) {
+            winner = __ffs(tied) - 1;
+        } else {
+            const uint32_t lo = __reduce_max_sync(0xffffffffu, hv == hi ? static_cast<uint32_t>(head) : 0u);
+            winner = __ffs(__ballot_sync(0xffffffffu, hv == hi && static_cast<uint32_t>(head) == lo)) - 1;
+        }
+        const uint32_t wlo = __shfl_sync(0xffffffffu, static_cast<uint32_t>(head), winner);
+        if (lane == 0) dst[r] = (static_cast<uint64_t>(hi) << 32) | wlo;
+        if (lane == winner) {
+#pragma unroll
+            for (int q = 0; q + 1 < N; ++q) keys[q] = keys[q + 1];
+            keys[N - 1] = 0ull;
         }
     }
 }
 
+// Top-k (k <= 32) of E <= 1024 logits by one block of NW warps: each warp
+// takes the k best of its keys, then warp 0 the k best of the NW*k
+// candidates.  sel[0..k-1] receives the selection keys in rank order.
+template <int NW>
 __device__ void block_topk(const float *logits, int E, int k, uint64_t *cand, uint64_t *sel) {
+    constexpr int KPT = 1024 / (32 * NW);            // keys per thread
+    constexpr int CPL = NW;                          // candidates per lane in the second stage (NW*32/32)
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     {
-        uint64_t keys[4];
+        uint64_t keys[KPT];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const int e = threadIdx.x + kDecThreads * q;
+        for (int q = 0; q < KPT; ++q) {
+            const int e = threadIdx.x + 32 * NW * q;
             keys[q] = e < E ? sel_key(__ldcg(logits + e), e) : 0ull;
         }
         warp_take(keys, k, lane, cand + warp * k);
     }
     __syncthreads();
     if (warp == 0) {
-        uint64_t keys[8];
+        uint64_t keys[CPL];
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
+        for (int q = 0; q < CPL; ++q) {
             const int i = lane + 32 * q;
-            keys[q] = i < kDecWarps * k ? cand[i] : 0ull;
+            keys[q] = i < NW * k ? cand[i] : 0ull;
         }
         warp_take(keys, k, lane, sel);
+    }
+    __syncthreads();
+}
+
+// ------------------------------------------------------------ 1. route
+// One warp per router row, kLogitRows rows per CTA, so the E rows are read by
+// E / kLogitRows SMs at once; every lane issues all of its weight loads
+// before it stages x.  Each CTA then takes a ticket; the CTA holding the last
+// one sees every logit (writes fenced before the ticket) and selects.
+constexpr int kLogitRows = 4;
+
+__global__ void __launch_bounds__(kLogitRows * 32) k_dec_route(DecodeArgs a) {
+    __shared__ __align__(16) float xs[2048];
+    __shared__ uint64_t cand[kLogitRows * 32], sel[32];
+    __shared__ unsigned ticket_s;
+    pdl_trigger();                                       // the gate/up kernel may start its prologue
+    const int H = a.H, E = a.E, k = a.k;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (!a.logits_in) {
+        const int e = blockIdx.x * kLogitRows + warp;
+        uint4 w[8];                                      // bf16 rows: 8 x 16 B per lane covers H <= 2048
+        if (a.w_bf16) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int hh = lane * 8 + 256 * j;
+                w[j] = make_uint4(0, 0, 0, 0);
+                if (e < E && hh < H)
+                    w[j] = ldg_stream(static_cast<const __nv_bfloat16 *>(a.w_router) + static_cast<size_t>(e) * H + hh);
+            }
+        }
+        for (int i = threadIdx.x; i < H / 4; i += blockDim.x)
+            reinterpret_cast<float4 *>(xs)[i] = a.x_bf16 ? load4(static_cast<const __nv_bfloat16 *>(a.x) + 4 * i)
+                                                         : load4(static_cast<const float *>(a.x) + 4 * i);
+        __syncthreads();
+        if (e < E) {
+            float s = 0.f;
+            if (a.w_bf16) {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int hh = lane * 8 + 256 * j;
+                    if (hh < H) {
+                        const float4 x0 = reinterpret_cast<const float4 *>(xs + hh)[0];
+                        const float4 x1 = reinterpret_cast<const float4 *>(xs + hh)[1];
+                        const uint4 u = w[j];
+                        s = fmaf(__uint_as_float(u.x << 16), x0.x, s);
+                        s = fmaf(__uint_as_float(u.x & 0xffff0000u), x0.y, s);
+                        s = fmaf(__uint_as_float(u.y << 16), x0.z, s);
+                        s = fmaf(__uint_as_float(u.y & 0xffff0000u), x0.w, s);
+                        s = fmaf(__uint_as_float(u.z << 16), x1.x, s);
+                        s = fmaf(__uint_as_float(u.z & 0xffff0000u), x1.y, s);
+                        s = fmaf(__uint_as_float(u.w << 16), x1.z, s);
+                        s = fmaf(__uint_as_float(u.w & 0xffff0000u), x1.w, s);
+                    }
+                }
+            } else {
+                for (int hh = lane * 4; hh < H; hh += 128) {
+                    const float4 wv = load4(static_cast<const float *>(a.w_router) + static_cast<size_t>(e) * H + hh);
+                    const float4 xv = reinterpret_cast<const float4 *>(xs + hh)[0];
+                    s = fmaf(wv.x, xv.x, s); s = fmaf(wv.y, xv.y, s);
+                    s = fmaf(wv.z, xv.z, s); s = fmaf(wv.w, xv.w, s);
+                }
+            }
+            s = warp_sum(s);
+            if (lane == 0) {
+                const float l = s + (a.bias ? a.bias[e] : 0.f);
+                a.ws.logits[e] = l;
+                if (a.logits_out) a.logits_out[e] = l;
+                __threadfence();                         // visible before this CTA's ticket
+            }
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) ticket_s = atomicAdd(a.ws.ticket, 1u);
+    __syncthreads();
+    const unsigned t = ticket_s;
+    if (t >= gridDim.x) {                                // the counter was not zero on entry
+        if (threadIdx.x == 0) report(a.err, MOE_DEVERR_WORKSPACE);
+        return;
+    }
+    if (t != gridDim.x - 1) return;
+    __threadfence();
+    block_topk<kLogitRows>(a.logits_in ? a.logits_in : a.ws.logits, E, k, cand, sel);
+    if (warp == 0) {
+        const uint64_t key = lane < k ? sel[lane] : 0ull;
+        const float my_v = key_float(static_cast<uint32_t>(key >> 32));
+        const int my_id = static_cast<int>(0xffffffffu - static_cast<uint32_t>(key));
+        const float v0 = __shfl_sync(0xffffffffu, my_v, 0);
+        const bool bad = lane < k && (my_v != my_v || my_v == __int_as_float(0x7f800000));
+        const bool any_bad = __any_sync(0xffffffffu, bad);
+        const float ex = lane < k ? expf(my_v - v0) : 0.f;
+        float sum = 0.f;
+        for (int j = 0; j < k; ++j) sum += __shfl_sync(0xffffffffu, ex, j);   // slot order
+        if (lane < k) {
+            const float wj = any_bad ? __int_as_float(0x7fc00000) : ex / sum;
+            a.ws.ids[lane] = my_id;
+            a.ws.gates[lane] = wj;
+            a.ids_out[lane] = my_id;
+            a.w_out[lane] = wj;
+        }
+        if (lane == 0) {
+            if (any_bad) report(a.err, MOE_DEVERR_NONFINITE);
+            *a.ws.ticket = 0u;                           // the next call starts from zero
+        }
+    }
+}
+
+// x as fp32 pieces in the order the chunk loops read them (piece q of chunk
+// c at q * nch + c) plus the pre-scaled block sums (128 + h) * sum(x over the
+// block); every divisor is a compile-time constant.
+template <int BITS>
+__device__ __forceinline__ void stage_x(float4 *xs, float *cs, int H, const void *x, int bf16) {
+    using Q = QT<BITS>;
+    const int nch = H / Q::EPC;
+    for (int g4 = threadIdx.x; g4 < H / 4; g4 += blockDim.x) {
+        const int c = g4 / Q::PPC, q = g4 % Q::PPC;
+        xs[q * nch + c] = bf16 ? load4(static_cast<const __nv_bfloat16 *>(x) + 4 * g4)
+                               : load4(static_cast<const float *>(x) + 4 * g4);
+    }
+    __syncthreads();
+    for (int b = threadIdx.x; b < H / 32; b += blockDim.x) {
+        const int c = b / Q::BPC, beta = b % Q::BPC;
+        float s = 0.f;
+#pragma unroll
+        for (int p = 0; p < 8; ++p) {
+            const float4 v = xs[(8 * beta + p) * nch + c];
+            s += (v.x + v.y) + (v.z + v.w);
+        }
+        cs[b] = static_cast<float>(128 + Q::HALF) * s;
     }
     __syncthreads();
 }
@@ -187,99 +285,69 @@ __device__ void block_topk(const float *logits, int E, int k, uint64_t *cand, ui
 // activation pieces of one chunk in registers and applies them to the four
 // weight rows of its warp (gate and up of two rows).
 template <int BITS>
-__global__ void __launch_bounds__(kDecThreads, BITS == 4 ? 3 : 2) k_dec_gateup(DecodeArgs a) {
+__global__ void __launch_bounds__(kDecThreads, 3) k_dec_gateup(DecodeArgs a) {
     using Q = QT<BITS>;
     extern __shared__ __align__(16) float4 gsm[];
-    __shared__ const uint8_t *blob_s;
+    pdl_trigger();                                       // the down kernel may start (it waits for us)
     const int H = a.H, I = a.I, k = a.k;
-    const int rows_per_block = kDecWarps * 2;
-    const int rblocks = I / rows_per_block;
+    constexpr int RPB = kDecWarps * 2;
+    const int rblocks = I / RPB;
     const int g = blockIdx.x / rblocks;
-    const int i0 = (blockIdx.x % rblocks) * rows_per_block;
+    const int i0 = (blockIdx.x - g * rblocks) * RPB;
     const bool shared_group = g == k;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     float4 *xs = gsm;
     float *cs = reinterpret_cast<float *>(gsm + H / 4);
-    {
-        const void *x = a.x;
-        stage_rows_fn<BITS>(xs, cs, 1, 1, H, [x](int) { return x; }, a.x_bf16);   // independent of the routing
-    }
-    pdl_trigger();                                       // the down kernel may start
-    if (!shared_group) {
-        pdl_wait();                                      // the logits are final from here on
-        __shared__ uint64_t cand[kDecWarps * 32], sel[32];
-        block_topk(a.logits_in ? a.logits_in : a.ws.logits, a.E, k, cand, sel);
-        if (blockIdx.x == 0 && threadIdx.x < 32) {       // one CTA publishes ids and gates
-            const int lane = threadIdx.x;
-            const uint64_t key = lane < k ? sel[lane] : 0ull;
-            const float my_v = key_float(static_cast<uint32_t>(key >> 32));
-            const int my_id = static_cast<int>(0xffffffffu - static_cast<uint32_t>(key));
-            const float v0 = __shfl_sync(0xffffffffu, my_v, 0);
-            const bool bad = lane < k && (my_v != my_v || my_v == __int_as_float(0x7f800000));
-            const bool any_bad = __any_sync(0xffffffffu, bad);
-            const float ex = lane < k ? expf(my_v - v0) : 0.f;
-            float sum = 0.f;
-            for (int j = 0; j < k; ++j) sum += __shfl_sync(0xffffffffu, ex, j);   // slot order
-            if (lane < k) {
-                const float wj = any_bad ? __int_as_float(0x7fc00000) : ex / sum;
-                a.ws.ids[lane] = my_id;
-                a.ws.gates[lane] = wj;
-                a.ids_out[lane] = my_id;
-                a.w_out[lane] = wj;
-            }
-            if (lane == 0 && any_bad) report(a.err, MOE_DEVERR_NONFINITE);
-        }
-        if (threadIdx.x == 0) {
-            const int e = static_cast<int>(0xffffffffu - static_cast<uint32_t>(sel[g]));
-            const uint8_t *b = (e >= 0 && e < a.E) ? a.blobs[e] : nullptr;
-            if (!b) report(a.err, (e >= 0 && e < a.E) ? MOE_DEVERR_NULL_BLOB : MOE_DEVERR_BAD_EXPERT);
-            blob_s = b;
-        }
-    } else if (threadIdx.x == 0) {
-        blob_s = a.shared;
-    }
-    __syncthreads();
-    const uint8_t *blob = blob_s;
-    if (!blob) return;
-    const BlobView bv = blob_view(blob, BITS, H, I);
     const int nch = H / Q::EPC;
     const int nscx = H / 32;
     const size_t xrowb = static_cast<size_t>(H) * BITS / 8;
-    // all code loads of the warp's four row vectors first
     constexpr int S = 2048 / Q::EPC / 32;               // chunks per lane (H <= 2048)
     uint4 code[4][S];
     float dsc[4][S][Q::BPC];
+    // all code loads of the warp's four row vectors
+    auto load_codes = [&](const uint8_t *blob) {
+        const BlobView bv = blob_view(blob, BITS, H, I);
 #pragma unroll
-    for (int v = 0; v < 4; ++v) {
-        const int i = i0 + warp * 2 + (v >> 1);
-        const uint8_t *cbase = (v & 1) ? bv.cu : bv.cg;
-        const __half *sbase = (v & 1) ? bv.su : bv.sg;
+        for (int v = 0; v < 4; ++v) {
+            const int i = i0 + warp * 2 + (v >> 1);
+            const uint8_t *cbase = (v & 1) ? bv.cu : bv.cg;
+            const __half *sbase = (v & 1) ? bv.su : bv.sg;
 #pragma unroll
-        for (int s = 0; s < S; ++s) {
-            const int cc = lane + 32 * s;
-            const bool valid = cc < nch;
-            code[v][s] = valid ? ldg_stream(cbase + static_cast<size_t>(i) * xrowb + static_cast<size_t>(cc) * 16)
-                               : make_uint4(0, 0, 0, 0);
-            load_scales<BITS>(sbase + static_cast<size_t>(i) * nscx, cc, valid, dsc[v][s]);
+            for (int s = 0; s < S; ++s) {
+                const int cc = lane + 32 * s;
+                const bool valid = cc < nch;
+                code[v][s] = valid ? ldg_stream(cbase + static_cast<size_t>(i) * xrowb + static_cast<size_t>(cc) * 16)
+                                   : make_uint4(0, 0, 0, 0);
+                load_scales<BITS>(sbase + static_cast<size_t>(i) * nscx, cc, valid, dsc[v][s]);
+            }
         }
+    };
+    stage_x<BITS>(xs, cs, H, a.x, a.x_bf16);
+    if (shared_group) {
+        load_codes(a.shared);                            // independent of the routing
+    } else {
+        pdl_wait();                                      // ids are final from here on
+        const int e = __ldcg(a.ws.ids + g);
+        const uint8_t *blob = (e >= 0 && e < a.E) ? a.blobs[e] : nullptr;
+        if (!blob) {
+            if (threadIdx.x == 0) report(a.err, (e >= 0 && e < a.E) ? MOE_DEVERR_NULL_BLOB : MOE_DEVERR_BAD_EXPERT);
+            return;                                      // uniform over the CTA; no barrier follows
+        }
+        load_codes(blob);
     }
     float dot[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int s = 0; s < S; ++s) {
         const int cc = lane + 32 * s;
         if (cc < nch) {
-            float4 xp[Q::PPC];
-#pragma unroll
-            for (int q = 0; q < Q::PPC; ++q) xp[q] = xs[q * nch + cc];
             float csum[Q::BPC];
 #pragma unroll
             for (int b = 0; b < Q::BPC; ++b) csum[b] = cs[cc * Q::BPC + b];
+            const uint4 cv[4] = {code[0][s], code[1][s], code[2][s], code[3][s]};
+            float fx[4][Q::BPC];
+            rows_fx<BITS, 4>(cv, xs + cc, nch, fx);
 #pragma unroll
-            for (int v = 0; v < 4; ++v) {
-                float fx[Q::BPC];
-                chunk_fx<BITS>(code[v][s], xp, fx);
-                dot[v] = chunk_finish<BITS>(fx, dsc[v][s], csum, dot[v]);
-            }
+            for (int v = 0; v < 4; ++v) dot[v] = chunk_finish<BITS>(fx[v], dsc[v][s], csum, dot[v]);
         }
     }
 #pragma unroll
@@ -291,80 +359,97 @@ __global__ void __launch_bounds__(kDecThreads, BITS == 4 ? 3 : 2) k_dec_gateup(D
 }
 
 // ------------------------------------------------------ 3. down + combine
-// Block = RB output rows x all groups.  Tasks (group, lane-row group) are
-// spread over the 8 warps; each lane takes one chunk of one row (lpr lanes
-// per row), with every code load of the warp issued before h is staged.
-// Per-group partials meet in shared memory and are summed in slot order.
+// Block = RB output rows x all groups.  Tasks (group, RPP rows) are spread
+// over the 8 warps; each lane takes one chunk of one row (LPR = I / chunk
+// lanes per row), with every code load of the warp issued before h is
+// staged.  Per-group partials meet in shared memory and are summed in slot
+// order.
 constexpr int kDownTasks = 8;                            // tasks per warp (checked on the host)
 
-template <int BITS>
-__global__ void __launch_bounds__(kDecThreads, 2) k_dec_down(DecodeArgs a, int ng, int RB) {
+template <int BITS, int LPR, int RB>
+__global__ void __launch_bounds__(kDecThreads, 2) k_dec_down(DecodeArgs a, int ng) {
     using Q = QT<BITS>;
+    constexpr int RPP = 32 / LPR;                        // rows per task
+    constexpr int TPG = RB / RPP;                        // tasks per group
+    constexpr int IL = LPR * Q::EPC;                     // the intermediate size I
+    static_assert(RB % RPP == 0, "rows per block");
     extern __shared__ __align__(16) float4 dsm[];
     __shared__ const uint8_t *blobs_s[33];
     __shared__ float gates_s[33];
-    const int H = a.H, I = a.I, k = a.k;
+    const int H = a.H, k = a.k;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int nchd = I / Q::EPC;                         // chunks per row == lanes per row (power of two)
-    const int lpr = nchd;
-    const int rpp = 32 / lpr;                            // rows per task
-    const int tpg = RB / rpp;                            // tasks per group
-    const int ntasks = ng * tpg;
+    const int ntasks = ng * TPG;
     const int r0 = blockIdx.x * RB;
-    const size_t drowb = static_cast<size_t>(I) * BITS / 8;
-    const int dnsc = I / 32;
-    float4 *hs = dsm;
-    float *hcs = reinterpret_cast<float *>(dsm + static_cast<size_t>(ng) * (I / 4));
-    float *part = hcs + static_cast<size_t>(ng) * (I / 32);
+    constexpr size_t drowb = static_cast<size_t>(IL) * BITS / 8;
+    constexpr int dnsc = IL / 32;
+    float4 *hs = dsm;                                    // [ng][PPC][LPR] pieces
+    float *hcs = reinterpret_cast<float *>(dsm + static_cast<size_t>(ng) * (IL / 4));
+    float *part = hcs + static_cast<size_t>(ng) * dnsc;
     pdl_wait();                                          // ids (route) and h (gate/up) are final
     if (threadIdx.x < ng) {
         const int g = threadIdx.x;
         const uint8_t *b = a.shared;
         float gw = 1.0f;
         if (g < k) {
-            const int e = a.ws.ids[g];
+            const int e = __ldcg(a.ws.ids + g);
             b = (e >= 0 && e < a.E) ? a.blobs[e] : nullptr;
-            gw = a.ws.gates[g];
+            gw = __ldcg(a.ws.gates + g);
         }
         blobs_s[g] = b;
         gates_s[g] = gw;
     }
     __syncthreads();
-    const int seg = lane % lpr, sub = lane / lpr;
+    const int seg = lane % LPR, sub = lane / LPR;
     uint4 code[kDownTasks];
     float dsc[kDownTasks][Q::BPC];
 #pragma unroll
     for (int t = 0; t < kDownTasks; ++t) {
         const int task = warp + kDecWarps * t;
-        const int g = task / tpg;
-        const int r = r0 + (task % tpg) * rpp + sub;
-        const bool valid = task < ntasks && r < H && blobs_s[g] != nullptr;
+        const int g = task / TPG;
+        const int r = r0 + (task % TPG) * RPP + sub;
+        const uint8_t *blob = task < ntasks ? blobs_s[g] : nullptr;
+        const bool valid = blob != nullptr && r < H;
         code[t] = make_uint4(0, 0, 0, 0);
-        const BlobView bv = blob_view(valid ? blobs_s[g] : a.shared, BITS, H, I);
+        const BlobView bv = blob_view(valid ? blob : a.shared, BITS, H, IL);
         if (valid) code[t] = ldg_stream(bv.cd + static_cast<size_t>(r) * drowb + static_cast<size_t>(seg) * 16);
         load_scales<BITS>(bv.sd + static_cast<size_t>(valid ? r : 0) * dnsc, seg, valid, dsc[t]);
     }
-    {
-        const float *h = a.ws.h;
-        stage_rows_fn<BITS>(hs, hcs, ng, ng, I,
-                            [h, I](int t) { return static_cast<const void *>(h + static_cast<size_t>(t) * I); }, 0);
-    }                                                    // ends with __syncthreads
+    // stage h of every group (gate/up's fp32 output) as pieces + block sums
+    for (int g4 = threadIdx.x; g4 < ng * (IL / 4); g4 += kDecThreads) {
+        const int t = g4 / (IL / 4), rem = g4 % (IL / 4);
+        const int c = rem / Q::PPC, q = rem % Q::PPC;
+        hs[(t * Q::PPC + q) * LPR + c] = __ldcg(reinterpret_cast<const float4 *>(a.ws.h) + g4);
+    }
+    __syncthreads();
+    for (int b = threadIdx.x; b < ng * dnsc; b += kDecThreads) {
+        const int t = b / dnsc, bb = b % dnsc;
+        const int c = bb / Q::BPC, beta = bb % Q::BPC;
+        float s = 0.f;
+#pragma unroll
+        for (int p = 0; p < 8; ++p) {
+            const float4 v = hs[(t * Q::PPC + 8 * beta + p) * LPR + c];
+            s += (v.x + v.y) + (v.z + v.w);
+        }
+        hcs[b] = static_cast<float>(128 + Q::HALF) * s;
+    }
+    __syncthreads();
 #pragma unroll
     for (int t = 0; t < kDownTasks; ++t) {
         const int task = warp + kDecWarps * t;
         if (task >= ntasks) break;                       // uniform over the warp
-        const int g = task / tpg;
-        const int rl = (task % tpg) * rpp + sub;
+        const int g = task / TPG;
+        const int rl = (task % TPG) * RPP + sub;
         float4 xp[Q::PPC];
 #pragma unroll
-        for (int q = 0; q < Q::PPC; ++q) xp[q] = hs[static_cast<size_t>(g) * (I / 4) + q * nchd + seg];
+        for (int q = 0; q < Q::PPC; ++q) xp[q] = hs[(g * Q::PPC + q) * LPR + seg];
         float csum[Q::BPC];
 #pragma unroll
-        for (int b = 0; b < Q::BPC; ++b) csum[b] = hcs[static_cast<size_t>(g) * (I / 32) + seg * Q::BPC + b];
+        for (int b = 0; b < Q::BPC; ++b) csum[b] = hcs[g * dnsc + seg * Q::BPC + b];
         float fx[Q::BPC];
         chunk_fx<BITS>(code[t], xp, fx);
         float v = blobs_s[g] ? chunk_finish<BITS>(fx, dsc[t], csum, 0.f) : 0.f;
-        for (int o = lpr >> 1; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+#pragma unroll
+        for (int o = LPR >> 1; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
         if (seg == 0) part[g * RB + rl] = v;
     }
     __syncthreads();
@@ -377,20 +462,49 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_dec_down(DecodeArgs a, int n
 
 // ------------------------------------------------------------------ host
 size_t decode_ws_bytes(int E, int k, int I) {
-    return 256 + ((static_cast<size_t>(E) * 4 + 255) / 256) * 256 + static_cast<size_t>(k + 1) * I * 4;
+    return 512 + ((static_cast<size_t>(E) * 4 + 255) / 256) * 256 + static_cast<size_t>(k + 1) * I * 4;
 }
 
-static int down_rows_per_block(int ng) { return ng <= 16 ? 8 : 4; }
+static int down_lpr(int bits, int I) { return I / (bits == 4 ? 32 : 64); }
+static int down_rows_per_block(int ng, int lpr) { return (ng <= 16 || lpr == 4) ? 8 : 4; }
 
 bool decode_supported(int bits, int H, int I, int E, int k) {
-    if (E > 1024 || k > 32 || H > 2048 || I % 128 != 0) return false;
-    const int nchd = I / (bits == 4 ? 32 : 64);
-    if (nchd > 32 || (nchd & (nchd - 1)) != 0) return false;    // one chunk per lane, power-of-two lanes per row
-    const int rpp = 32 / nchd, ng = k + 1, RB = down_rows_per_block(ng);
+    if (E > 1024 || k > 32 || H > 2048 || H % 128 != 0 || I % 128 != 0) return false;
+    const int lpr = down_lpr(bits, I);
+    if (lpr != 4 && lpr != 8 && lpr != 16 && lpr != 32) return false;   // one chunk per lane
+    const int rpp = 32 / lpr, ng = k + 1, RB = down_rows_per_block(ng, lpr);
     if (RB % rpp != 0 || ceil_div(ng * (RB / rpp), kDecWarps) > kDownTasks) return false;
     const size_t smem_down = static_cast<size_t>(ng) * I * 4 + static_cast<size_t>(ng) * (I / 32) * 4 +
                              static_cast<size_t>(ng) * RB * 4;
     return smem_down <= 200 * 1024;
+}
+
+template <int BITS, int LPR, int RB>
+static int launch_down(const DecodeArgs &a, int groups, const cudaLaunchAttribute &pdl, cudaStream_t s) {
+    const size_t smem = static_cast<size_t>(groups) * a.I * 4 + static_cast<size_t>(groups) * (a.I / 32) * 4 +
+                        static_cast<size_t>(groups) * RB * 4;
+    int rc = cuda_status(cudaFuncSetAttribute(k_dec_down<BITS, LPR, RB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                              static_cast<int>(smem)),
+                         "down smem attribute");
+    if (rc) return rc;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(ceil_div(a.H, RB));
+    cfg.blockDim = dim3(kDecThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr = pdl;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    rc = cuda_status(cudaLaunchKernelEx(&cfg, k_dec_down<BITS, LPR, RB>, a, groups), "decode down launch");
+    count_launches(1);
+    return rc;
+}
+
+template <int BITS, int LPR>
+static int launch_down_rb(const DecodeArgs &a, int groups, const cudaLaunchAttribute &pdl, cudaStream_t s) {
+    if constexpr (LPR == 4) return launch_down<BITS, LPR, 8>(a, groups, pdl, s);
+    else if (down_rows_per_block(groups, LPR) == 8) return launch_down<BITS, LPR, 8>(a, groups, pdl, s);
+    else return launch_down<BITS, LPR, 4>(a, groups, pdl, s);
 }
 
 template <int BITS>
@@ -399,13 +513,13 @@ static int launch_decode_t(DecodeArgs a, int groups, cudaStream_t s) {
     cudaLaunchAttribute pdl;
     pdl.id = cudaLaunchAttributeProgrammaticStreamSerialization;
     pdl.val.programmaticStreamSerializationAllowed = 1;
-    // 1. router logits (skipped when the caller supplies them)
-    if (!a.logits_in) {
+    // 1. route: logits over E/4 CTAs (one CTA that only selects when the caller gives logits)
+    {
         cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(ceil_div(E, kLogitRows));
+        cfg.gridDim = dim3(a.logits_in ? 1 : ceil_div(E, kLogitRows));
         cfg.blockDim = dim3(kLogitRows * 32);
         cfg.stream = s;
-        int rc = cuda_status(cudaLaunchKernelEx(&cfg, k_dec_logits, a), "decode logits launch");
+        int rc = cuda_status(cudaLaunchKernelEx(&cfg, k_dec_route, a), "decode route launch");
         count_launches(1);
         if (rc) return rc;
     }
@@ -419,30 +533,17 @@ static int launch_decode_t(DecodeArgs a, int groups, cudaStream_t s) {
         cfg.dynamicSmemBytes = smem;
         cfg.stream = s;
         cfg.attrs = &pdl;
-        cfg.numAttrs = a.logits_in ? 0 : 1;              // x and given logits come from earlier work: no overlap
+        cfg.numAttrs = 1;
         int rc = cuda_status(cudaLaunchKernelEx(&cfg, k_dec_gateup<BITS>, a), "decode gate/up launch");
         count_launches(1);
         if (rc) return rc;
     }
     // 3. down + combine
-    {
-        const int RB = down_rows_per_block(groups);
-        const size_t smem = static_cast<size_t>(groups) * I * 4 + static_cast<size_t>(groups) * (I / 32) * 4 +
-                            static_cast<size_t>(groups) * RB * 4;
-        int rc = cuda_status(cudaFuncSetAttribute(k_dec_down<BITS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                  static_cast<int>(smem)),
-                             "down smem attribute");
-        if (rc) return rc;
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(ceil_div(H, RB));
-        cfg.blockDim = dim3(kDecThreads);
-        cfg.dynamicSmemBytes = smem;
-        cfg.stream = s;
-        cfg.attrs = &pdl;
-        cfg.numAttrs = 1;
-        rc = cuda_status(cudaLaunchKernelEx(&cfg, k_dec_down<BITS>, a, groups, RB), "decode down launch");
-        count_launches(1);
-        return rc;
+    switch (down_lpr(BITS, I)) {
+        case 4: return launch_down_rb<BITS, 4>(a, groups, pdl, s);
+        case 8: return launch_down_rb<BITS, 8>(a, groups, pdl, s);
+        case 16: return launch_down_rb<BITS, 16>(a, groups, pdl, s);
+        default: return launch_down_rb<BITS, 32>(a, groups, pdl, s);
     }
 }
 

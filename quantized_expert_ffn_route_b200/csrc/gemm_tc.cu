@@ -4,20 +4,24 @@
 // of up to 8,192 tokens, and reading touches all the experts, so the expert
 // step becomes a dense contraction per expert: D = W_e (dequantised) x X_e^T.
 //
-// Per tile: 128 weight rows (MMA M) x up to 256 of the expert's tokens (MMA N),
-// K in steps of 64.  Weights are the A operand, so small token groups still
-// fill the M = 128 datapath ("swap AB").  Roles of one persistent CTA per SM:
-//   warps 0-7   copy their raw codes + scales a few k-steps ahead (cp.async
-//               into private slots) and dequantise them to fp16 into the
-//               128-byte-swizzled A stages;
-//   warps 13-14 gather the tile's token rows (fp16) into the B stages with
-//               cp.async, each thread arriving on the stage's barrier when
-//               its copies land (cp.async.mbarrier.arrive.noinc);
-//   warp  12    allocates TMEM and issues tcgen05.mma (one thread);
-//   warps 8-11  epilogue: tcgen05.ld the fp32 accumulators and write
+// Per tile: two 128-row weight matrices (gate and up rows m0..m0+127, or down
+// rows m0..m0+255 as two halves) x up to MAXN of the expert's tokens, K in
+// steps of 64.  Weights are the MMA's A operand (M = 128), tokens the N side,
+// so a group of ten tokens still fills the datapath ("swap AB"); both
+// matrices share the token tile.  Roles of one persistent CTA per SM:
+//   warps 0-15  each thread copies the codes + scale of one 32-weight block a
+//               few k-steps ahead (cp.async into private slots) and
+//               dequantises it to fp16 into a 128-byte-swizzled A stage;
+//   warps 21-22 gather the tile's token rows (fp16) into the B stages with
+//               cp.async, a few k-steps ahead; each warp publishes a stage
+//               with one barrier arrival once its copies have landed;
+//   warp  20    allocates TMEM and issues tcgen05.mma (one thread);
+//   warps 16-19 epilogue: tcgen05.ld the fp32 accumulators and write
 //               gate/up -> h = silu(g) * u (fp16) or down -> y rows (fp32).
-// Every mbarrier wait is bounded; a timeout sets MOE_DEVERR_TIMEOUT and all
-// roles leave their loops, after which TMEM is freed.
+// The CTA's tile list (expert blob, token range, weight rows) is built once
+// in shared memory.  Every mbarrier wait is bounded; a timeout sets
+// MOE_DEVERR_TIMEOUT and all roles leave their loops, after which TMEM is
+// freed.
 #include "common.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
@@ -25,41 +29,52 @@
 namespace moe {
 using namespace sm100;
 
-constexpr int kBM = 128;            // weight rows per tile
+constexpr int kBM = 128;            // weight rows per matrix of a tile (MMA M)
 constexpr int kBK = 64;             // K per stage: one 128-byte row of fp16
-constexpr int kProd = 256;          // dequantising threads: 128 rows x 2 parts
+constexpr int kDeq = 512;           // dequantising threads: 128 rows x 2 matrices x 2 blocks
 constexpr int kLoad = 64;           // token-row loader threads
-constexpr int kGemmThreads = 480;   // 8 dequant warps, 4 epilogue warps, 1 MMA warp, 2 loader warps
+constexpr int kEpiWarp0 = 16, kMmaWarp = 20, kLoadWarp0 = 21;
+constexpr int kGemmThreads = 736;   // 16 dequant, 4 epilogue, 1 MMA, 2 loader warps
 constexpr long kSpin = 1L << 22;    // polls before a wait gives up (about a second)
-constexpr int kMaxGroups = 2048;
+constexpr int kMaxGroups = 4096;    // groups (active experts + shared) one launch may hold
+constexpr size_t kSmemLimit = 232448;
+
+// One tile of a CTA's list.
+struct TileEntry {
+    const uint8_t *blob;
+    int row0;     // first permuted row of the group, or -1 for the shared expert
+    int n0;       // first token of the tile within the group
+    int m0;       // first weight row
+    int nvalid;   // tokens in the tile
+};
 
 // MAXN: tokens per tile.  Small tiles (64) leave room for deep rings (the
 // HBM-bound regime: few tokens per expert); large tiles (256) fill the
 // tensor cores when experts hold hundreds of tokens.
 template <int BITS, bool GATEUP, int MAXN>
 struct GemmCfg {
-    static constexpr int NA = GATEUP ? 2 : 1;                 // weight matrices per tile (gate, up)
-    static constexpr int ELEMS = GATEUP ? 64 : 32;            // elements one producer thread dequantises per k-step
-    static constexpr int RAW_CODE = ELEMS * BITS / 8;         // its code bytes per k-step
-    static constexpr int SEG = (RAW_CODE + 4 + 15) / 16 * 16; // codes + two fp16 scales, 16-byte aligned
-    static constexpr int SA = GATEUP ? 3 : 4;                 // A (dequantised weight) stages
-    static constexpr int SB = MAXN > 128 ? (GATEUP ? 3 : 4) : 8;   // B (token row) stages
-    static constexpr int L = MAXN > 128 ? (GATEUP ? 2 : 3) : 4;    // k-steps the code copies run ahead (= slots)
-    static constexpr int ACC = NA * MAXN * 2 <= 512 ? 2 : 1;  // TMEM accumulator buffers
-    static constexpr int TMEM_COLS = ACC * NA * MAXN <= 128 ? 128 : (ACC * NA * MAXN <= 256 ? 256 : 512);
-    static constexpr size_t A_STAGE = static_cast<size_t>(NA) * kBM * 128;
+    static constexpr int CODE = 32 * BITS / 8;                // code bytes of one block
+    static constexpr int SA = MAXN > 128 ? 2 : 3;             // A (dequantised weight) stages
+    static constexpr int SB = MAXN > 128 ? 4 : 8;             // B (token row) stages
+    static constexpr int L = MAXN > 128 ? 2 : 4;              // k-steps the code copies run ahead (= slots)
+    static constexpr int ACC = 2 * MAXN * 2 <= 512 ? 2 : 1;   // TMEM accumulator buffers
+    static constexpr int TMEM_COLS = ACC * 2 * MAXN <= 128 ? 128 : (ACC * 2 * MAXN <= 256 ? 256 : 512);
+    static constexpr size_t A_STAGE = static_cast<size_t>(2) * kBM * 128;
     static constexpr size_t B_STAGE = static_cast<size_t>(MAXN) * 128;
-    static constexpr size_t RAW_STAGE = static_cast<size_t>(kProd) * SEG;
+    static constexpr size_t RC_STAGE = static_cast<size_t>(kDeq) * CODE;
+    static constexpr size_t RS_STAGE = static_cast<size_t>(kDeq) * 4;
     static constexpr size_t OFF_A = 0;
     static constexpr size_t OFF_B = OFF_A + SA * A_STAGE;
-    static constexpr size_t OFF_RAW = OFF_B + SB * B_STAGE;
-    static constexpr size_t OFF_TOK = OFF_RAW + L * RAW_STAGE;
-    static constexpr size_t OFF_GS = OFF_TOK + MAXN * 4;
-    static constexpr size_t OFF_BAR = (OFF_GS + (kMaxGroups + 1) * 4 + 15) / 16 * 16;
-    static constexpr size_t SMEM = OFF_BAR + 32 * 8 + 16 + 1024;   // bars, TMEM address, tile count, abort
-                                                                   // flag; + slack for 1024-byte alignment
+    static constexpr size_t OFF_RC = OFF_B + SB * B_STAGE;
+    static constexpr size_t OFF_RS = OFF_RC + L * RC_STAGE;
+    static constexpr size_t OFF_TOK = OFF_RS + L * RS_STAGE;
+    static constexpr size_t OFF_BAR = (OFF_TOK + MAXN * 4 + 15) / 16 * 16;
+    static constexpr size_t OFF_TILES = OFF_BAR + 32 * 8 + 16;   // bars, TMEM address, tile count, abort flag
+    static constexpr size_t FIXED = OFF_TILES + 1024;            // + slack for 1024-byte alignment
+    static size_t smem(int cap) { return FIXED + static_cast<size_t>(cap) * sizeof(TileEntry); }
     static_assert(2 * SA + 2 * SB + 5 <= 32, "barrier slots");
-    static_assert(SMEM <= 232448, "shared memory per block (no static shared memory is used)");
+    static_assert(SB * B_STAGE >= (kMaxGroups + 1) * 4, "group scratch fits the B ring");
+    static_assert(FIXED <= kSmemLimit, "shared memory per block");
 };
 
 struct GemmArgs {
@@ -99,12 +114,6 @@ __device__ __forceinline__ GroupInfo group_info(const GemmArgs &a, int g, int n_
     if (!G.blob) G.n = 0;
     return G;
 }
-
-// One tile of this CTA's sequence: group, first token, first weight row.
-struct TileInfo {
-    GroupInfo G;
-    int n0, m0, nvalid, N;
-};
 
 // bytes hold one code per byte; builds the half2 (1024 + q_a, 1024 + q_b)
 __device__ __forceinline__ uint32_t pair16(uint32_t bytes, uint32_t sel) { return __byte_perm(bytes, 0x64646464u, sel); }
@@ -149,256 +158,320 @@ __device__ __forceinline__ void dequant_block(const uint8_t *codes, __half2 d2, 
 }
 
 template <int BITS, bool GATEUP, int MAXN>
-__global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(GemmArgs a) {
+__global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(GemmArgs a, int tile_cap) {
     using Cfg = GemmCfg<BITS, GATEUP, MAXN>;
-    constexpr int SA = Cfg::SA, SB = Cfg::SB, L = Cfg::L, ACC = Cfg::ACC, NA = Cfg::NA;
+    constexpr int SA = Cfg::SA, SB = Cfg::SB, L = Cfg::L, ACC = Cfg::ACC;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sA = smem + Cfg::OFF_A;
     uint8_t *sB = smem + Cfg::OFF_B;
-    uint8_t *sRaw = smem + Cfg::OFF_RAW;
+    uint8_t *sRC = smem + Cfg::OFF_RC;
+    uint8_t *sRS = smem + Cfg::OFF_RS;
     int32_t *tok_s = reinterpret_cast<int32_t *>(smem + Cfg::OFF_TOK);
-    int32_t *gstart = reinterpret_cast<int32_t *>(smem + Cfg::OFF_GS);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::OFF_BAR);
     uint64_t *fullA = bars, *emptyA = bars + SA, *fullB = bars + 2 * SA, *emptyB = bars + 2 * SA + SB;
     uint64_t *accF = bars + 2 * SA + 2 * SB, *accE = accF + 2, *drain = accF + 4;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 32);
-    int *total_tiles_p = reinterpret_cast<int *>(bars + 32) + 1;
     volatile int &abort_s = *(reinterpret_cast<int *>(bars + 32) + 2);   // read in loop conditions: never cached
+    TileEntry *tiles = reinterpret_cast<TileEntry *>(smem + Cfg::OFF_TILES);
+    int32_t *gcnt = reinterpret_cast<int32_t *>(sB);   // per-group tile counts while the tile list is built
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int K = GATEUP ? a.H : a.I;           // reduction length
-    const int Mtot = GATEUP ? a.I : a.H;        // weight rows
-    const int MT = Mtot / kBM;
+    const int K = GATEUP ? a.H : a.I;                  // reduction length
+    const int Mtot = GATEUP ? a.I : a.H;               // weight rows
+    const int MROWS = GATEUP ? kBM : 2 * kBM;          // weight rows a tile advances by
+    const int MT = (Mtot + MROWS - 1) / MROWS;
     const int nk = K / kBK;
     const int n_act = min(max(a.active[0], 0), min(a.E, a.T * a.k));
-    const int ng = n_act + (a.shared ? 1 : 0);
+    const int ng = min(n_act + (a.shared ? 1 : 0), kMaxGroups);
 
     if (tid == 0) {
         abort_s = 0;
         for (int i = 0; i < SA; ++i) {
-            mbar_init(fullA + i, kProd);
+            mbar_init(fullA + i, kDeq / 32);           // one arrival per dequantising warp
             mbar_init(emptyA + i, 1);
         }
         for (int i = 0; i < SB; ++i) {
-            mbar_init(fullB + i, kLoad);
+            mbar_init(fullB + i, kLoad / 32);          // one arrival per loader warp
             mbar_init(emptyB + i, 1);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(accF + i, 1);
-            mbar_init(accE + i, 128);
+            mbar_init(accE + i, 4);                     // one arrival per epilogue warp
         }
         mbar_init(drain, 1);
         fence_barrier_init();
         fence_proxy_async();
     }
-    // tile prefix sums over the groups (one warp)
-    if (warp == 0) {
+    // ---- the CTA's tile list: tiles are numbered group by group, m-tile
+    // fastest, and dealt to CTAs round robin (tile t -> CTA t % grid)
+    for (int g = tid; g < ng; g += blockDim.x) {
+        const GroupInfo G = group_info(a, g, n_act);
+        gcnt[g] = ((G.n + MAXN - 1) / MAXN) * MT;
+    }
+    __syncthreads();
+    if (warp == 0) {                                   // exclusive prefix sum, in place
         int run = 0;
         for (int base = 0; base < ng; base += 32) {
             const int g = base + lane;
-            int t = 0;
-            if (g < ng) {
-                const GroupInfo G = group_info(a, g, n_act);
-                t = ((G.n + MAXN - 1) / MAXN) * MT;
-            }
+            const int t = g < ng ? gcnt[g] : 0;
             int incl = t;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
                 const int v = __shfl_up_sync(0xffffffffu, incl, o);
                 if (lane >= o) incl += v;
             }
-            if (g < ng) gstart[g] = run + incl - t;
+            if (g < ng) gcnt[g] = run + incl - t;
             run += __shfl_sync(0xffffffffu, incl, 31);
         }
-        if (lane == 0) {
-            gstart[ng] = run;
-            *total_tiles_p = run;
-        }
+        if (lane == 0) gcnt[ng] = run;
     }
-    if (warp == 12) {
+    if (warp == kMmaWarp) {
         tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
         tmem_relinquish();
     }
-    tc_fence_before();
     __syncthreads();
+    const int total = gcnt[ng];
+    const int grid = static_cast<int>(gridDim.x), bid = static_cast<int>(blockIdx.x);
+    int n_my = bid < total ? (total - 1 - bid) / grid + 1 : 0;
+    for (int g = tid; g < ng; g += blockDim.x) {
+        const int start = gcnt[g], cnt = gcnt[g + 1] - start;
+        if (cnt <= 0) continue;
+        const GroupInfo G = group_info(a, g, n_act);
+        for (int tt = start + ((bid - start) % grid + grid) % grid; tt < start + cnt; tt += grid) {
+            const int i = (tt - bid) / grid, local = tt - start;
+            if (i >= tile_cap) break;
+            TileEntry te;
+            te.blob = G.blob;
+            te.row0 = G.row0;
+            te.n0 = (local / MT) * MAXN;
+            te.m0 = (local % MT) * MROWS;
+            te.nvalid = min(MAXN, G.n - te.n0);
+            tiles[i] = te;
+        }
+    }
+    if (n_my > tile_cap) {                             // offsets inconsistent with T*k: do nothing
+        if (tid == 0) report(a.err, MOE_DEVERR_BAD_ROW);
+        n_my = 0;
+    }
+    tc_fence_before();
+    __syncthreads();                                   // tile list final; the B ring is free again
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const int total = *total_tiles_p;
-    const int n_my = blockIdx.x < total ? (total - 1 - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x) + 1 : 0;
-    const long J = static_cast<long>(n_my) * nk;   // k-steps of this CTA
-
-    auto tile_of = [&](int i) {                  // i-th tile of this CTA
-        const int t = blockIdx.x + i * gridDim.x;
-        int lo = 0, hi = ng;                     // largest g with gstart[g] <= t
-        while (hi - lo > 1) {
-            const int mid = (lo + hi) >> 1;
-            if (gstart[mid] <= t) lo = mid;
-            else hi = mid;
-        }
-        TileInfo ti;
-        ti.G = group_info(a, lo, n_act);
-        const int local = t - gstart[lo];
-        ti.n0 = (local / MT) * MAXN;
-        ti.m0 = (local % MT) * kBM;
-        ti.nvalid = min(MAXN, ti.G.n - ti.n0);
-        ti.N = (ti.nvalid + 15) & ~15;
-        return ti;
-    };
+    const long J = static_cast<long>(n_my) * nk;      // k-steps of this CTA
     auto fail = [&]() {
         report(a.err, MOE_DEVERR_TIMEOUT);
         abort_s = 1;
     };
+    auto aborted = [&]() { return __shfl_sync(0xffffffffu, abort_s, 0) != 0; };   // the same answer on every lane
 
-    if (warp < 8) {
+    if (warp < kEpiWarp0) {
         // ------------------------------------------------- dequantisation
-        const int row = tid & 127, part = tid >> 7;
+        // thread -> (row, matrix, block of the k-step)
+        const int row = tid & 127, mat = (tid >> 7) & 1, half = tid >> 8;
         const size_t rowbytes = static_cast<size_t>(K) * BITS / 8;
         const int nsc = K / 32;
-        int raw_tile = -1;
-        TileInfo rt{};
-        // copies of this thread's codes + scales of k-step jr into its slot jr % L
-        auto issue_raw = [&](long jr) {
+        int cur = -1;
+        TileEntry te{};
+        // warp 0 asks L2 for a whole tile's codes and scales (its rows are
+        // contiguous) one tile ahead, so the 16-byte copies below mostly hit L2
+        // and DRAM sees long sequential reads
+        auto prefetch_tile = [&](int i) {
+            if (i >= n_my) return;
+            const TileEntry tp = tiles[i];
+            const BlobView pv = blob_view(tp.blob, BITS, a.H, a.I);
+            constexpr uint32_t kPiece = 8192;
+#pragma unroll
+            for (int pm = 0; pm < 2; ++pm) {
+                const int m0 = tp.m0 + (GATEUP ? 0 : kBM * pm);
+                const int nrows = min(kBM, Mtot - m0);
+                if (nrows <= 0) continue;
+                const uint8_t *cbase = (GATEUP ? (pm ? pv.cu : pv.cg) : pv.cd) + static_cast<size_t>(m0) * rowbytes;
+                const size_t cbytes = static_cast<size_t>(nrows) * rowbytes;
+                for (size_t off = static_cast<size_t>(lane) * kPiece; off < cbytes; off += 32 * kPiece)
+                    prefetch_l2(cbase + off, static_cast<uint32_t>(min(static_cast<size_t>(kPiece), cbytes - off)));
+                const __half *sbase = (GATEUP ? (pm ? pv.su : pv.sg) : pv.sd) + static_cast<size_t>(m0) * nsc;
+                const size_t sbytes = static_cast<size_t>(nrows) * nsc * 2;
+                if (lane == 31 && (reinterpret_cast<uintptr_t>(sbase) & 15) == 0 && (sbytes & 15) == 0)
+                    prefetch_l2(sbase, static_cast<uint32_t>(sbytes));
+            }
+        };
+        if (warp == 0) prefetch_tile(0);
+        auto issue = [&](long jr) {
             if (jr >= J) return;
             const int i = static_cast<int>(jr / nk), s = static_cast<int>(jr % nk);
-            if (i != raw_tile) {
-                rt = tile_of(i);
-                raw_tile = i;
+            if (i != cur) {
+                te = tiles[i];
+                cur = i;
+                if (warp == 0) prefetch_tile(i + 1);
             }
-            const BlobView bv = blob_view(rt.G.blob, BITS, a.H, a.I);
-            const uint8_t *codes = GATEUP ? (part ? bv.cu : bv.cg) : bv.cd;
-            const __half *scl = GATEUP ? (part ? bv.su : bv.sg) : bv.sd;
-            const size_t m = static_cast<size_t>(rt.m0 + row);
-            const uint8_t *src = codes + m * rowbytes + static_cast<size_t>(s) * (kBK * BITS / 8) +
-                                 (GATEUP ? 0 : part * Cfg::RAW_CODE);
-            const uint32_t dst = smem_addr(sRaw + (jr % L) * Cfg::RAW_STAGE + static_cast<size_t>(tid) * Cfg::SEG);
-            if constexpr (Cfg::RAW_CODE >= 16) {
-#pragma unroll
-                for (int q = 0; q < Cfg::RAW_CODE / 16; ++q) cp_async16(dst + q * 16, src + q * 16, 16);
-            } else {
-                asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dst), "l"(src) : "memory");
-            }
-            cp_async4(dst + Cfg::RAW_CODE, scl + m * nsc + 2 * s);
+            const BlobView bv = blob_view(te.blob, BITS, a.H, a.I);
+            const uint8_t *codes = GATEUP ? (mat ? bv.cu : bv.cg) : bv.cd;
+            const __half *scl = GATEUP ? (mat ? bv.su : bv.sg) : bv.sd;
+            const int m = te.m0 + (GATEUP ? 0 : kBM * mat) + row;
+            const bool ok = m < Mtot;
+            const size_t mm = ok ? static_cast<size_t>(m) : 0;
+            const uint8_t *src = codes + mm * rowbytes + static_cast<size_t>(2 * s + half) * Cfg::CODE;
+            const int slot = static_cast<int>(jr % L);
+            const uint32_t dc = smem_addr(sRC + slot * Cfg::RC_STAGE + static_cast<size_t>(tid) * Cfg::CODE);
+            if constexpr (Cfg::CODE == 16) cp_async16(dc, src, ok ? 16u : 0u);
+            else cp_async8z(dc, src, ok ? 8u : 0u);
+            cp_async4z(smem_addr(sRS + slot * Cfg::RS_STAGE + static_cast<size_t>(tid) * 4), scl + mm * nsc + 2 * s,
+                       ok ? 4u : 0u);
         };
-        for (int p = 0; p < L; ++p) {             // prologue: one commit group per k-step
-            issue_raw(p);
+        for (int p = 0; p < L; ++p) {                  // prologue: one commit group per k-step
+            issue(p);
             cp_async_commit();
         }
-        for (long j = 0; j < J && !abort_s; ++j) {
-            cp_async_wait<L - 1>();              // this thread's codes of k-step j have landed
+        for (long j = 0; j < J && !aborted(); ++j) {
+            cp_async_wait<L - 1>();                    // this thread's codes of k-step j have landed
             const int sa = static_cast<int>(j % SA);
-            if (!mbar_wait(emptyA + sa, static_cast<uint32_t>(((j / SA) & 1) ^ 1), kSpin)) {
+            // one lane per warp polls the stage barrier; the warp follows it
+            int ok = 1;
+            if (lane == 0) ok = mbar_wait(emptyA + sa, static_cast<uint32_t>(((j / SA) & 1) ^ 1), kSpin);
+            if (!__shfl_sync(0xffffffffu, ok, 0)) {
                 fail();
                 break;
             }
-            const uint8_t *raw = sRaw + (j % L) * Cfg::RAW_STAGE + static_cast<size_t>(tid) * Cfg::SEG;
-            const __half2 s01 = *reinterpret_cast<const __half2 *>(raw + Cfg::RAW_CODE);
-            const uint32_t a_row = smem_addr(sA + sa * Cfg::A_STAGE +
-                                             static_cast<size_t>(GATEUP ? part : 0) * kBM * 128 +
+            const int slot = static_cast<int>(j % L);
+            const __half2 s01 = *reinterpret_cast<const __half2 *>(sRS + slot * Cfg::RS_STAGE + static_cast<size_t>(tid) * 4);
+            const uint32_t a_row = smem_addr(sA + sa * Cfg::A_STAGE + static_cast<size_t>(mat) * kBM * 128 +
                                              static_cast<size_t>(row) * 128);
-            if (GATEUP) {
-                dequant_block<BITS>(raw, __low2half2(s01), a_row, 0, row & 7);
-                dequant_block<BITS>(raw + 4 * BITS, __high2half2(s01), a_row, 4, row & 7);
-            } else {
-                dequant_block<BITS>(raw, part ? __high2half2(s01) : __low2half2(s01), a_row, 4 * part, row & 7);
-            }
-            fence_proxy_async();
-            mbar_arrive(fullA + sa);
-            issue_raw(j + L);                    // into the slot just read
+            dequant_block<BITS>(sRC + slot * Cfg::RC_STAGE + static_cast<size_t>(tid) * Cfg::CODE,
+                                half ? __high2half2(s01) : __low2half2(s01), a_row, 4 * half, row & 7);
+            fence_proxy_async();                       // this thread's A writes -> async proxy
+            __syncwarp();                              // ... ordered before lane 0's release-arrive
+            if (lane == 0) mbar_arrive(fullA + sa);
+            issue(j + L);                              // into the slot just read
             cp_async_commit();
         }
         cp_async_wait<0>();
-    } else if (warp >= 13) {
+    } else if (warp >= kLoadWarp0) {
         // --------------------------------------------------- token rows
         // Loader warp lw copies rows lw*MAXN/2 .. of each tile: lane = 8 x row
         // + 16-byte chunk.  Its token indices live in a warp-private table.
-        const int lw = warp - 13;
+        const int lw = warp - kLoadWarp0;
         constexpr int HALF = MAXN / 2;
         int32_t *tok = tok_s + lw * HALF;
         const uint8_t *bsrc = GATEUP ? reinterpret_cast<const uint8_t *>(a.x16)
                                      : reinterpret_cast<const uint8_t *>(a.h16);
         const size_t brow = static_cast<size_t>(K) * 2;
         const int c = lane & 7;
-        int cur = -1;
-        TileInfo bt{};
-        for (long j = 0; j < J && !abort_s; ++j) {
-            const int i = static_cast<int>(j / nk), s = static_cast<int>(j % nk);
-            if (i != cur) {
-                bt = tile_of(i);
-                cur = i;
-                __syncwarp();
-                for (int nl = lane; nl < HALF; nl += 32) {
-                    const int n = lw * HALF + nl;
-                    int v = 0;
-                    if (n < bt.nvalid) {
-                        if (GATEUP)
-                            v = min(max(bt.G.row0 >= 0 ? a.perm_src[bt.G.row0 + bt.n0 + n] : bt.n0 + n, 0), a.T - 1);
-                        else
-                            v = (bt.G.row0 >= 0 ? bt.G.row0 : a.T * a.k) + bt.n0 + n;
+        int cur = -1, N = 0, nvalid = 0;
+        // Copies of k-step j are issued at iteration j and published at
+        // iteration j + D, after this thread's cp.async group for j has
+        // landed: wait, proxy fence, then one arrival per warp.
+        constexpr int D = SB / 2;                  // leaves SB - D stages for the MMAs to overlap with
+        for (long j = 0; j < J + D; ++j) {
+            if (aborted()) break;
+            if (j < J) {
+                const int i = static_cast<int>(j / nk), s = static_cast<int>(j % nk);
+                if (i != cur) {
+                    const TileEntry te = tiles[i];
+                    cur = i;
+                    nvalid = te.nvalid;
+                    N = (nvalid + 15) & ~15;
+                    __syncwarp();
+                    for (int nl = lane; nl < HALF; nl += 32) {
+                        const int n = lw * HALF + nl;
+                        int v = 0;
+                        if (n < nvalid) {
+                            if (GATEUP)
+                                v = min(max(te.row0 >= 0 ? a.perm_src[te.row0 + te.n0 + n] : te.n0 + n, 0), a.T - 1);
+                            else
+                                v = (te.row0 >= 0 ? te.row0 : a.T * a.k) + te.n0 + n;
+                        }
+                        tok[nl] = v;
                     }
-                    tok[nl] = v;
+                    __syncwarp();
                 }
-                __syncwarp();
-            }
-            const int sb = static_cast<int>(j % SB);
-            if (!mbar_wait(emptyB + sb, static_cast<uint32_t>(((j / SB) & 1) ^ 1), kSpin)) {
-                fail();
-                break;
-            }
-            const uint32_t bdst = smem_addr(sB + sb * Cfg::B_STAGE);
+                const int sb = static_cast<int>(j % SB);
+                int ok = 1;
+                if (lane == 0) ok = mbar_wait(emptyB + sb, static_cast<uint32_t>(((j / SB) & 1) ^ 1), kSpin);
+                if (!__shfl_sync(0xffffffffu, ok, 0)) {
+                    fail();
+                    break;
+                }
+                const uint32_t bdst = smem_addr(sB + sb * Cfg::B_STAGE);
 #pragma unroll 4
-            for (int nl = lane >> 3; nl < HALF; nl += 4) {
-                const int n = lw * HALF + nl;
-                if (n < bt.N) {
-                    const uint8_t *src = bsrc + static_cast<size_t>(tok[nl]) * brow + static_cast<size_t>(s) * 128 + c * 16;
-                    cp_async16(bdst + n * 128 + ((c ^ (n & 7)) << 4), src, n < bt.nvalid ? 16u : 0u);
+                for (int nl = lane >> 3; nl < HALF; nl += 4) {
+                    const int n = lw * HALF + nl;
+                    if (n < N) {
+                        const uint8_t *src =
+                            bsrc + static_cast<size_t>(tok[nl]) * brow + static_cast<size_t>(s) * 128 + c * 16;
+                        cp_async16(bdst + n * 128 + ((c ^ (n & 7)) << 4), src, n < nvalid ? 16u : 0u);
+                    }
                 }
             }
-            asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_addr(fullB + sb))
-                         : "memory");
+            cp_async_commit();                         // one group per iteration (empty while draining)
+            if (j >= D) {
+                cp_async_wait<D>();                    // this thread's copies of k-step j - D have landed
+                fence_proxy_async();                   // ... and are visible to the tensor cores
+                __syncwarp();
+                if (lane == 0) mbar_arrive(fullB + (j - D) % SB);
+            }
         }
         cp_async_wait<0>();
-    } else if (warp < 12) {
+    } else if (warp < kMmaWarp) {
         // -------------------------------------------------------- epilogue
-        const int q = warp & 3;                   // TMEM lanes 32q .. 32q+31
-        const int m = 32 * q + lane;              // weight row within the tile
-        for (int i = 0; i < n_my && !abort_s; ++i) {
-            const TileInfo ti = tile_of(i);
+        const int q = warp & 3;                        // TMEM lanes 32q .. 32q+31
+        const int m = 32 * q + lane;                   // weight row within a matrix of the tile
+        for (int i = 0; i < n_my && !aborted(); ++i) {
+            const TileEntry te = tiles[i];
             const int b = i % ACC;
-            if (!mbar_wait(accF + b, static_cast<uint32_t>((i / ACC) & 1), kSpin)) {
+            int ok = 1;
+            if (lane == 0) ok = mbar_wait(accF + b, static_cast<uint32_t>((i / ACC) & 1), kSpin);
+            if (!__shfl_sync(0xffffffffu, ok, 0)) {
                 fail();
                 break;
             }
             tc_fence_after();
-            const uint32_t base = tmem + (static_cast<uint32_t>(32 * q) << 16) + b * NA * MAXN;
-            for (int c0 = 0; c0 < ti.nvalid; c0 += 16) {
-                float gv[16], uv[16];
-                tmem_ld16(base + c0, gv);
-                if (GATEUP) tmem_ld16(base + MAXN + c0, uv);
-                tmem_ld_wait();
+            const uint32_t base = tmem + (static_cast<uint32_t>(32 * q) << 16) + b * 2 * MAXN;
+            const size_t rbase = static_cast<size_t>(te.row0 >= 0 ? te.row0 : a.T * a.k) + te.n0;
+            if (GATEUP) {
+                for (int c0 = 0; c0 < te.nvalid; c0 += 16) {
+                    float gv[16], uv[16];
+                    tmem_ld16(base + c0, gv);
+                    tmem_ld16(base + MAXN + c0, uv);
+                    tmem_ld_wait();
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const int n = c0 + e;
-                    if (n >= ti.nvalid) break;
-                    if (GATEUP) {
-                        const float h = gv[e] / (1.0f + expf(-gv[e])) * uv[e];
-                        const size_t r = static_cast<size_t>(ti.G.row0 >= 0 ? ti.G.row0 : a.T * a.k) + ti.n0 + n;
-                        a.h16[r * a.I + ti.m0 + m] = __float2half_rn(h);
-                    } else {
-                        float *dst = ti.G.row0 >= 0 ? a.y_perm + (static_cast<size_t>(ti.G.row0) + ti.n0 + n) * a.H
-                                                    : a.y_shared + (static_cast<size_t>(ti.n0) + n) * a.H;
-                        dst[ti.m0 + m] = gv[e];
+                    for (int e = 0; e < 16; ++e) {
+                        const int n = c0 + e;
+                        if (n >= te.nvalid) break;
+                        const float h = __fdividef(gv[e], 1.0f + __expf(-gv[e])) * uv[e];
+                        a.h16[(rbase + n) * a.I + te.m0 + m] = __float2half_rn(h);
+                    }
+                }
+            } else {
+                for (int mat = 0; mat < 2; ++mat) {
+                    const int mrow = te.m0 + kBM * mat + m;
+                    if (te.m0 + kBM * mat >= a.H) break;     // ragged last tile: one matrix
+                    for (int c0 = 0; c0 < te.nvalid; c0 += 16) {
+                        float v[16];
+                        tmem_ld16(base + mat * MAXN + c0, v);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) {
+                            const int n = c0 + e;
+                            if (n >= te.nvalid) break;
+                            float *dst = te.row0 >= 0 ? a.y_perm + (rbase + n) * a.H
+                                                      : a.y_shared + (static_cast<size_t>(te.n0) + n) * a.H;
+                            if (mrow < a.H) dst[mrow] = v[e];
+                        }
                     }
                 }
             }
             tc_fence_before();
-            mbar_arrive(accE + b);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(accE + b);
         }
-    } else {
+    } else if (warp == kMmaWarp) {
         // ------------------------------------------------------ MMA issuer
-        for (int i = 0; i < n_my && !abort_s; ++i) {
-            const TileInfo ti = tile_of(i);
-            const uint32_t idesc = idesc_f16_f32(kBM, ti.N);
+        for (int i = 0; i < n_my && !aborted(); ++i) {
+            const TileEntry te = tiles[i];
+            const int N = (te.nvalid + 15) & ~15;
+            const uint32_t idesc = idesc_f16_f32(kBM, N);
+            const int nmat = (GATEUP || te.m0 + kBM < a.H) ? 2 : 1;
             const int b = i % ACC;
             if (lane == 0) {
                 if (!mbar_wait(accE + b, static_cast<uint32_t>(((i / ACC) & 1) ^ 1), kSpin)) fail();
@@ -413,16 +486,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(GemmArgs a) {
                     }
                     tc_fence_after();
                     const uint32_t b_addr = smem_addr(sB + sb * Cfg::B_STAGE);
+                    const uint32_t a_addr = smem_addr(sA + sa * Cfg::A_STAGE);
 #pragma unroll
                     for (int kk = 0; kk < kBK / 16; ++kk) {
                         const uint64_t bdesc = desc_sw128(b_addr + kk * 32);
-#pragma unroll
-                        for (int mat = 0; mat < NA; ++mat) {
-                            const uint32_t a_addr =
-                                smem_addr(sA + sa * Cfg::A_STAGE + static_cast<size_t>(mat) * kBM * 128) + kk * 32;
-                            mma_f16(tmem + b * NA * MAXN + mat * MAXN, desc_sw128(a_addr), bdesc, idesc,
-                                    (s | kk) != 0);
-                        }
+                        for (int mat = 0; mat < nmat; ++mat)
+                            mma_f16(tmem + b * 2 * MAXN + mat * MAXN, desc_sw128(a_addr + mat * kBM * 128 + kk * 32),
+                                    bdesc, idesc, (s | kk) != 0);
                     }
                     mma_commit(emptyA + sa);
                     mma_commit(emptyB + sb);
@@ -440,7 +510,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(GemmArgs a) {
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 12) {
+    if (warp == kMmaWarp) {
         tc_fence_after();
         tmem_dealloc(tmem, Cfg::TMEM_COLS);
     }
@@ -469,30 +539,70 @@ size_t gemm_ws_bytes(int bits, int T, int k, int H, int I, int E) {
     return align256(static_cast<size_t>(T) * H * 2) + align256(static_cast<size_t>(T) * (k + 1) * I * 2);
 }
 
-bool gemm_supported(int T, int k, int E) { return (T * k < E ? T * k : E) + 1 <= kMaxGroups; }
+// Upper bound on the tiles of one launch: a group of n tokens has
+// ceil(n / maxn) <= n / maxn + 1 token tiles, the shared expert ceil(T / maxn).
+static long tiles_bound(int T, int k, int E, int MT, int maxn) {
+    const long rows = static_cast<long>(T) * k;
+    const long groups = rows < E ? rows : E;
+    return (rows / maxn + groups + (T + maxn - 1) / maxn) * static_cast<long>(MT);
+}
+
+struct GemmPlan {
+    bool large;      // 256-token tiles (else 64)
+    int cap_gu;      // tile-list capacity per CTA, gate/up launch
+    int cap_dn;      // same, down launch
+};
+
+template <int BITS>
+static bool make_plan(int T, int k, int H, int I, int E, GemmPlan &p) {
+    const long groups = static_cast<long>(T) * k < E ? static_cast<long>(T) * k : E;
+    if (groups + 1 > kMaxGroups || H % kBK != 0 || I % kBM != 0) return false;
+    // tiles of 256 tokens once experts hold more than ~48 tokens on average
+    p.large = static_cast<long>(T) * k > 48L * (groups > 0 ? groups : 1);
+    const int maxn = p.large ? 256 : 64;
+    const long grid = num_sms();
+    const long bg = tiles_bound(T, k, E, I / kBM, maxn), bd = tiles_bound(T, k, E, (H + 2 * kBM - 1) / (2 * kBM), maxn);
+    const long cg = (bg + grid - 1) / grid, cd = (bd + grid - 1) / grid;
+    if (cg > 65536 || cd > 65536) return false;
+    p.cap_gu = static_cast<int>(cg > 0 ? cg : 1);
+    p.cap_dn = static_cast<int>(cd > 0 ? cd : 1);
+    if (p.large)
+        return GemmCfg<BITS, true, 256>::smem(p.cap_gu) <= kSmemLimit &&
+               GemmCfg<BITS, false, 256>::smem(p.cap_dn) <= kSmemLimit;
+    return GemmCfg<BITS, true, 64>::smem(p.cap_gu) <= kSmemLimit && GemmCfg<BITS, false, 64>::smem(p.cap_dn) <= kSmemLimit;
+}
+
+bool gemm_supported(int bits, int T, int k, int H, int I, int E) {
+    GemmPlan p;
+    return bits == 4 ? make_plan<4>(T, k, H, I, E, p) : make_plan<2>(T, k, H, I, E, p);
+}
 
 template <int BITS, bool GATEUP, int MAXN>
-static int launch_k_gemm(const GemmArgs &a, cudaStream_t s) {
+static int launch_k_gemm(const GemmArgs &a, int cap, cudaStream_t s) {
     using Cfg = GemmCfg<BITS, GATEUP, MAXN>;
+    const size_t smem = Cfg::smem(cap);
     int rc = cuda_status(cudaFuncSetAttribute(k_gemm<BITS, GATEUP, MAXN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                              static_cast<int>(Cfg::SMEM)),
+                                              static_cast<int>(smem)),
                          "gemm smem attribute");
     if (rc) return rc;
-    k_gemm<BITS, GATEUP, MAXN><<<num_sms(), kGemmThreads, Cfg::SMEM, s>>>(a);
+    k_gemm<BITS, GATEUP, MAXN><<<num_sms(), kGemmThreads, smem, s>>>(a, cap);
     count_launches(1);
     return cuda_status(cudaGetLastError(), "gemm launch");
 }
 
 template <int BITS>
-static int launch_pair(const GemmArgs &a, bool large, cudaStream_t s) {
-    int rc = large ? launch_k_gemm<BITS, true, 256>(a, s) : launch_k_gemm<BITS, true, 64>(a, s);
+static int launch_pair(const GemmArgs &a, const GemmPlan &p, cudaStream_t s) {
+    int rc = p.large ? launch_k_gemm<BITS, true, 256>(a, p.cap_gu, s) : launch_k_gemm<BITS, true, 64>(a, p.cap_gu, s);
     if (rc) return rc;
-    return large ? launch_k_gemm<BITS, false, 256>(a, s) : launch_k_gemm<BITS, false, 64>(a, s);
+    return p.large ? launch_k_gemm<BITS, false, 256>(a, p.cap_dn, s) : launch_k_gemm<BITS, false, 64>(a, p.cap_dn, s);
 }
 
 int launch_gemm(int bits, const uint8_t *const *blobs, const int32_t *offsets, const int32_t *active,
                 const int32_t *perm_src, const void *x, int x_dtype, int T, int k, int H, int I, int E,
                 const uint8_t *shared_blob, float *y_perm, float *y_shared, void *ws, unsigned *err, cudaStream_t s) {
+    GemmPlan plan;
+    if (!(bits == 4 ? make_plan<4>(T, k, H, I, E, plan) : make_plan<2>(T, k, H, I, E, plan)))
+        return cuda_status(cudaErrorInvalidConfiguration, "gemm plan");
     uint8_t *p = static_cast<uint8_t *>(ws);
     GemmArgs a;
     a.blobs = blobs;
@@ -517,10 +627,7 @@ int launch_gemm(int bits, const uint8_t *const *blobs, const int32_t *offsets, c
         k_to_half<<<blocks, 256, 0, s>>>(x, x_dtype == MOE_BF16, n, const_cast<__half *>(a.x16));
         count_launches(1);
     }
-    // tiles of 256 tokens once experts hold more than ~48 tokens on average, else 64
-    const int groups = T * k < E ? T * k : E;
-    const bool large = static_cast<long>(T) * k > 48L * (groups > 0 ? groups : 1);
-    return bits == 4 ? launch_pair<4>(a, large, s) : launch_pair<2>(a, large, s);
+    return bits == 4 ? launch_pair<4>(a, plan, s) : launch_pair<2>(a, plan, s);
 }
 
 }  // namespace moe

@@ -43,190 +43,175 @@ __device__ __forceinline__ bool group_of(int g, int n_act, const int32_t *active
     return G.n > 0;
 }
 
-constexpr int kWarps = 8;
-constexpr int kRowsPerWarpGU = 2;
-constexpr int kNTS = 16;   // most tokens staged at once
+constexpr int kGvThreads = 256;
+constexpr int kGvWarps = kGvThreads / 32;
+constexpr int kGvRows = 16;      // gate/up rows per task (2 per warp)
+constexpr int kGvNT = 16;        // token rows staged per pass
+// down: row groups per warp (4-bit codes need more registers per chunk)
+template <int BITS>
+struct GvTPW { static constexpr int value = BITS == 4 ? 2 : 4; };
 
 // ---------------------------------------------------------------- gate/up
-template <int BITS, int NT>
-__device__ __forceinline__ void rows_gateup(const BlobView &bv, int H, int I, int i0, const float4 *xs,
-                                            const float *cs, int nt, float *hrow0, size_t hld, int lane) {
-    using Q = QT<BITS>;
-    const int nch = H / Q::EPC;
-    const size_t rowbytes = static_cast<size_t>(H) * BITS / 8;
-    const int nsc = H / 32;
-    constexpr int SPL = 2;     // chunks per lane: H <= 64 chunks (q4: 2048, q2: 4096)
-    uint4 cg[kRowsPerWarpGU][SPL], cu[kRowsPerWarpGU][SPL];
-#pragma unroll
-    for (int rr = 0; rr < kRowsPerWarpGU; ++rr)
-#pragma unroll
-        for (int s = 0; s < SPL; ++s) {
-            const int c = lane + 32 * s;
-            const size_t off = static_cast<size_t>(i0 + rr) * rowbytes + static_cast<size_t>(c) * 16;
-            if (c < nch) {
-                cg[rr][s] = ldg_stream(bv.cg + off);
-                cu[rr][s] = ldg_stream(bv.cu + off);
-            } else {
-                cg[rr][s] = cu[rr][s] = make_uint4(0, 0, 0, 0);
-            }
-        }
-#pragma unroll
-    for (int rr = 0; rr < kRowsPerWarpGU; ++rr) {
-        float dg[NT], du[NT];
-#pragma unroll
-        for (int t = 0; t < NT; ++t) dg[t] = du[t] = 0.f;
-#pragma unroll
-        for (int s = 0; s < SPL; ++s) {
-            const int c = lane + 32 * s;
-            const bool valid = c < nch;
-            float sg[Q::BPC], su[Q::BPC];
-            load_scales<BITS>(bv.sg + static_cast<size_t>(i0 + rr) * nsc, c, valid, sg);
-            load_scales<BITS>(bv.su + static_cast<size_t>(i0 + rr) * nsc, c, valid, su);
-            if (valid) {
-                chunk_dot<BITS, NT>(cg[rr][s], sg, xs, cs, nch, c, dg);
-                chunk_dot<BITS, NT>(cu[rr][s], su, xs, cs, nch, c, du);
-            }
-        }
-#pragma unroll
-        for (int t = 0; t < NT; ++t) {
-            const float g = warp_sum(dg[t]);
-            const float u = warp_sum(du[t]);
-            if (lane == t && t < nt) hrow0[static_cast<size_t>(t) * hld + i0 + rr] = g / (1.0f + expf(-g)) * u;
-        }
-    }
-}
-
-template <int BITS, int NT>
-__global__ void __launch_bounds__(256) k_gemv_gateup(const uint8_t *const *__restrict__ blobs,
-                                                      const int32_t *__restrict__ offsets,
-                                                      const int32_t *__restrict__ active,
-                                                      const int32_t *__restrict__ perm_src,
-                                                      const void *__restrict__ x, int x_bf16, int T, int k, int H,
-                                                      int I, int E,
-                                                      const uint8_t *__restrict__ shared_blob,
-                                                      float *__restrict__ hbuf, int NTS, unsigned *err) {
+// Task = (group, 16 rows).  The codes of a warp's four row vectors (gate and
+// up of two rows) stay in registers while the group's tokens are staged 16
+// at a time and streamed past them, one token per pass over the codes.
+template <int BITS>
+__global__ void __launch_bounds__(kGvThreads, 2) k_gemv_gateup(const uint8_t *const *__restrict__ blobs,
+                                                               const int32_t *__restrict__ offsets,
+                                                               const int32_t *__restrict__ active,
+                                                               const int32_t *__restrict__ perm_src,
+                                                               const void *__restrict__ x, int x_bf16, int T, int k,
+                                                               int H, int I, int E,
+                                                               const uint8_t *__restrict__ shared_blob,
+                                                               float *__restrict__ hbuf, unsigned *err) {
     using Q = QT<BITS>;
     extern __shared__ float4 smem[];
     float4 *xs = smem;
-    float *cs = reinterpret_cast<float *>(smem + static_cast<size_t>(NTS) * (H / 4));
-    __shared__ const void *rows[kNTS];
+    float *cs = reinterpret_cast<float *>(smem + static_cast<size_t>(kGvNT) * (H / 4));
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int n_act = min(max(active[0], 0), min(E, T * k));   // a corrupt count cannot run past `active`
     const int n_groups = n_act + (shared_blob ? 1 : 0);
-    const int rows_per_block = kWarps * kRowsPerWarpGU;
+    const int row_blocks = I / kGvRows;
+    const int nch = H / Q::EPC, nblk = H / 32, nsc = H / 32;
+    const size_t xrowb = static_cast<size_t>(H) * BITS / 8;
     const size_t xrow = static_cast<size_t>(H) * (x_bf16 ? 2 : 4);
-    const int row_blocks = I / rows_per_block;
+    constexpr int S = 2048 / Q::EPC / 32;               // chunks per lane (H <= 2048)
     for (int task = blockIdx.x; task < n_groups * row_blocks; task += gridDim.x) {
-        const int g = task / row_blocks, rb = task % row_blocks;
+        const int g = task / row_blocks, rb = task - g * row_blocks;
         Group G;
         if (!group_of(g, n_act, active, offsets, blobs, shared_blob, T, k, E, err, G)) continue;
         const BlobView bv = blob_view(G.blob, BITS, H, I);
-        const int i0 = rb * rows_per_block + warp * kRowsPerWarpGU;
-        for (int sub = 0; sub < G.n; sub += NTS) {
-            const int nt = min(NTS, G.n - sub);
-            if (threadIdx.x < NTS) {
-                const int r = sub + static_cast<int>(threadIdx.x);
-                const int tok = r < G.n ? (G.row0 >= 0 ? perm_src[G.row0 + r] : r) : 0;
-                rows[threadIdx.x] = static_cast<const uint8_t *>(x) + static_cast<size_t>(tok < 0 || tok >= T ? 0 : tok) * xrow;
+        const int i0 = rb * kGvRows + warp * 2;
+        uint4 code[4][S];
+        float dsc[4][S][Q::BPC];
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+            const int i = i0 + (v >> 1);
+            const uint8_t *cbase = (v & 1) ? bv.cu : bv.cg;
+            const __half *sbase = (v & 1) ? bv.su : bv.sg;
+#pragma unroll
+            for (int s = 0; s < S; ++s) {
+                const int cc = lane + 32 * s;
+                const bool valid = cc < nch;
+                code[v][s] = valid ? ldg_stream(cbase + static_cast<size_t>(i) * xrowb + static_cast<size_t>(cc) * 16)
+                                   : make_uint4(0, 0, 0, 0);
+                load_scales<BITS>(sbase + static_cast<size_t>(i) * nsc, cc, valid, dsc[v][s]);
             }
-            __syncthreads();
-            stage_rows<BITS>(xs, cs, NTS, nt, H, rows, x_bf16);
-            float *hrow0 = hbuf + static_cast<size_t>(G.row0 >= 0 ? G.row0 + sub : T * k + sub) * I;
-            if (NT == 1 || nt == 1) rows_gateup<BITS, 1>(bv, H, I, i0, xs, cs, nt, hrow0, I, lane);
-            else rows_gateup<BITS, NT>(bv, H, I, i0, xs, cs, nt, hrow0, I, lane);
-            __syncthreads();
+        }
+        const size_t hrow0 = static_cast<size_t>(G.row0 >= 0 ? G.row0 : T * k);
+#pragma unroll 1
+        for (int sub = 0; sub < G.n; sub += kGvNT) {
+            const int nt = min(kGvNT, G.n - sub);
+            const int row0 = G.row0;
+            stage_rows_fn<BITS>(
+                xs, cs, nt, nt, H,
+                [=](int t) {
+                    const int r = sub + t;
+                    int tok = row0 >= 0 ? perm_src[row0 + r] : r;
+                    tok = tok < 0 || tok >= T ? 0 : tok;
+                    return static_cast<const void *>(static_cast<const uint8_t *>(x) + static_cast<size_t>(tok) * xrow);
+                },
+                x_bf16);
+#pragma unroll 1
+            for (int t = 0; t < nt; ++t) {
+                float dot[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int s = 0; s < S; ++s) {
+                    const int cc = lane + 32 * s;
+                    if (cc < nch) {
+                        float csum[Q::BPC];
+#pragma unroll
+                        for (int b = 0; b < Q::BPC; ++b) csum[b] = cs[t * nblk + cc * Q::BPC + b];
+                        uint4 cv[4] = {code[0][s], code[1][s], code[2][s], code[3][s]};
+#pragma unroll
+                        for (int v = 0; v < 4; ++v) opaque(cv[v]);
+                        float fx[4][Q::BPC];
+                        rows_fx<BITS, 4>(cv, xs + static_cast<size_t>(t) * Q::PPC * nch + cc, nch, fx);
+#pragma unroll
+                        for (int v = 0; v < 4; ++v) dot[v] = chunk_finish<BITS>(fx[v], dsc[v][s], csum, dot[v]);
+                    }
+                }
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const float gv = warp_sum(dot[2 * j]);
+                    const float uv = warp_sum(dot[2 * j + 1]);
+                    if (lane == 0) hbuf[(hrow0 + sub + t) * I + i0 + j] = gv / (1.0f + expf(-gv)) * uv;
+                }
+            }
+            __syncthreads();                             // before the next pass restages
         }
     }
 }
 
 // ------------------------------------------------------------------- down
-constexpr int kRowPassesD = 2;
-
-template <int BITS, int NT>
-__device__ __forceinline__ void rows_down(const BlobView &bv, int H, int I, int r0, int lpr, const float4 *hs,
-                                          const float *cs, int nt, float *yrow0, int lane) {
+// Task = (group, RB output rows): each lane one 16-byte chunk of one row
+// (LPR lanes per row), GvTPW rows per lane kept in registers; the group's
+// h rows are staged 16 at a time.
+template <int BITS, int LPR>
+__global__ void __launch_bounds__(kGvThreads, 2) k_gemv_down(const uint8_t *const *__restrict__ blobs,
+                                                             const int32_t *__restrict__ offsets,
+                                                             const int32_t *__restrict__ active,
+                                                             const float *__restrict__ hbuf, int T, int k, int H,
+                                                             int E, const uint8_t *__restrict__ shared_blob,
+                                                             float *__restrict__ y_perm, float *__restrict__ y_shared,
+                                                             unsigned *err) {
     using Q = QT<BITS>;
-    const int nch = I / Q::EPC;
-    const size_t rowbytes = static_cast<size_t>(I) * BITS / 8;
-    const int nsc = I / 32;
-    const int seg = lane % lpr;
-    const int rpp = 32 / lpr;
-    const int spl = (nch + lpr - 1) / lpr;
-    uint4 code[kRowPassesD][2];
-#pragma unroll
-    for (int pp = 0; pp < kRowPassesD; ++pp) {
-        const int r = r0 + pp * rpp + lane / lpr;
-#pragma unroll
-        for (int s = 0; s < 2; ++s) {
-            const int c = seg + lpr * s;
-            code[pp][s] = (s < spl && c < nch && r < H)
-                              ? ldg_stream(bv.cd + static_cast<size_t>(r) * rowbytes + static_cast<size_t>(c) * 16)
-                              : make_uint4(0, 0, 0, 0);
-        }
-    }
-#pragma unroll
-    for (int pp = 0; pp < kRowPassesD; ++pp) {
-        const int r = r0 + pp * rpp + lane / lpr;
-        float dot[NT];
-#pragma unroll
-        for (int t = 0; t < NT; ++t) dot[t] = 0.f;
-#pragma unroll
-        for (int s = 0; s < 2; ++s) {
-            const int c = seg + lpr * s;
-            const bool valid = s < spl && c < nch && r < H;
-            float d[Q::BPC];
-            load_scales<BITS>(bv.sd + static_cast<size_t>(r < H ? r : 0) * nsc, c, valid, d);
-            if (valid) chunk_dot<BITS, NT>(code[pp][s], d, hs, cs, nch, c, dot);
-        }
-#pragma unroll
-        for (int t = 0; t < NT; ++t) {
-            float v = dot[t];
-            for (int o = lpr >> 1; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-            dot[t] = v;
-        }
-        if (r < H) {
-#pragma unroll
-            for (int t = 0; t < NT; ++t)
-                if (t % lpr == seg && t < nt) yrow0[static_cast<size_t>(t) * H + r] = dot[t];
-        }
-    }
-}
-
-template <int BITS, int NT>
-__global__ void __launch_bounds__(256) k_gemv_down(const uint8_t *const *__restrict__ blobs,
-                                                    const int32_t *__restrict__ offsets,
-                                                    const int32_t *__restrict__ active,
-                                                    const float *__restrict__ hbuf, int T, int k, int H, int I,
-                                                    int E, const uint8_t *__restrict__ shared_blob,
-                                                    float *__restrict__ y_perm, float *__restrict__ y_shared,
-                                                    int NTS, int lpr, unsigned *err) {
-    using Q = QT<BITS>;
+    constexpr int kGvTPW = GvTPW<BITS>::value;
+    constexpr int RPP = 32 / LPR;                        // rows per warp pass
+    constexpr int RB = kGvWarps * kGvTPW * RPP;          // rows per task
+    constexpr int IL = LPR * Q::EPC;                     // the intermediate size I
+    constexpr int nblk = IL / 32;
+    constexpr size_t drowb = static_cast<size_t>(IL) * BITS / 8;
     extern __shared__ float4 smem[];
     float4 *hs = smem;
-    float *cs = reinterpret_cast<float *>(smem + static_cast<size_t>(NTS) * (I / 4));
-    __shared__ const void *rows[kNTS];
+    float *hcs = reinterpret_cast<float *>(smem + static_cast<size_t>(kGvNT) * (IL / 4));
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int n_act = min(max(active[0], 0), min(E, T * k));   // a corrupt count cannot run past `active`
+    const int seg = lane % LPR, subr = lane / LPR;
+    const int n_act = min(max(active[0], 0), min(E, T * k));
     const int n_groups = n_act + (shared_blob ? 1 : 0);
-    const int rpp = 32 / lpr;
-    const int rows_per_block = kWarps * kRowPassesD * rpp;
-    const int row_blocks = (H + rows_per_block - 1) / rows_per_block;
+    const int row_blocks = (H + RB - 1) / RB;
     for (int task = blockIdx.x; task < n_groups * row_blocks; task += gridDim.x) {
-        const int g = task / row_blocks, rb = task % row_blocks;
+        const int g = task / row_blocks, rb = task - g * row_blocks;
         Group G;
         if (!group_of(g, n_act, active, offsets, blobs, shared_blob, T, k, E, err, G)) continue;
-        const BlobView bv = blob_view(G.blob, BITS, H, I);
-        const int r0 = rb * rows_per_block + warp * kRowPassesD * rpp;
-        for (int sub = 0; sub < G.n; sub += NTS) {
-            const int nt = min(NTS, G.n - sub);
-            const size_t hrow = static_cast<size_t>(G.row0 >= 0 ? G.row0 + sub : T * k + sub);
-            if (threadIdx.x < NTS) rows[threadIdx.x] = hbuf + (hrow + min(static_cast<int>(threadIdx.x), nt - 1)) * I;
-            __syncthreads();
-            stage_rows<BITS>(hs, cs, NTS, nt, I, rows, 0);
-            float *yrow0 = G.row0 >= 0 ? y_perm + static_cast<size_t>(G.row0 + sub) * H
-                                       : y_shared + static_cast<size_t>(sub) * H;
-            if (NT == 1 || nt == 1) rows_down<BITS, 1>(bv, H, I, r0, lpr, hs, cs, nt, yrow0, lane);
-            else rows_down<BITS, NT>(bv, H, I, r0, lpr, hs, cs, nt, yrow0, lane);
+        const BlobView bv = blob_view(G.blob, BITS, H, IL);
+        uint4 code[kGvTPW];
+        float dsc[kGvTPW][Q::BPC];
+        int rows[kGvTPW];
+#pragma unroll
+        for (int tt = 0; tt < kGvTPW; ++tt) {
+            const int r = rb * RB + (warp * kGvTPW + tt) * RPP + subr;
+            rows[tt] = r;
+            const bool valid = r < H;
+            code[tt] = valid ? ldg_stream(bv.cd + static_cast<size_t>(r) * drowb + static_cast<size_t>(seg) * 16)
+                             : make_uint4(0, 0, 0, 0);
+            load_scales<BITS>(bv.sd + static_cast<size_t>(valid ? r : 0) * nblk, seg, valid, dsc[tt]);
+        }
+        const size_t hrow0 = static_cast<size_t>(G.row0 >= 0 ? G.row0 : T * k);
+        float *yrow0 = G.row0 >= 0 ? y_perm + static_cast<size_t>(G.row0) * H : y_shared;
+#pragma unroll 1
+        for (int sub = 0; sub < G.n; sub += kGvNT) {
+            const int nt = min(kGvNT, G.n - sub);
+            stage_rows_fn<BITS>(
+                hs, hcs, nt, nt, IL,
+                [=](int t) { return static_cast<const void *>(hbuf + (hrow0 + sub + t) * IL); }, 0);
+#pragma unroll 1
+            for (int t = 0; t < nt; ++t) {
+                float csum[Q::BPC];
+#pragma unroll
+                for (int b = 0; b < Q::BPC; ++b) csum[b] = hcs[t * nblk + seg * Q::BPC + b];
+                float fx[kGvTPW][Q::BPC];
+#pragma unroll
+                for (int tt = 0; tt < kGvTPW; ++tt) opaque(code[tt]);
+                rows_fx<BITS, kGvTPW>(code, hs + static_cast<size_t>(t) * Q::PPC * LPR + seg, LPR, fx);
+#pragma unroll
+                for (int tt = 0; tt < kGvTPW; ++tt) {
+                    float v = chunk_finish<BITS>(fx[tt], dsc[tt], csum, 0.f);
+#pragma unroll
+                    for (int o = LPR >> 1; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+                    if (seg == 0 && rows[tt] < H) yrow0[static_cast<size_t>(sub + t) * H + rows[tt]] = v;
+                }
+            }
             __syncthreads();
         }
     }
@@ -237,37 +222,26 @@ size_t gemv_ws_bytes(int T, int k, int I) {
     return static_cast<size_t>(T) * (k + 1) * I * sizeof(float);
 }
 
-template <int BITS, int NT>
-static void launch_gemv_nt(const uint8_t *const *blobs, const int32_t *offsets, const int32_t *active,
-                           const int32_t *perm_src, const void *x, int x_bf16, int T, int k, int H, int I, int E,
-                           const uint8_t *shared_blob, float *y_perm, float *y_shared, float *hbuf, unsigned *err,
-                           cudaStream_t s) {
+bool gemv_supported(int bits, int H, int I) {
+    const int lpr = I / (bits == 4 ? 32 : 64);
+    return H >= 128 && H <= 2048 && H % 128 == 0 && I % 128 == 0 &&
+           (lpr == 2 || lpr == 4 || lpr == 8 || lpr == 16 || lpr == 32);
+}
+
+template <int BITS, int LPR>
+static void launch_down(const uint8_t *const *blobs, const int32_t *offsets, const int32_t *active, const float *hbuf,
+                        int T, int k, int H, int E, const uint8_t *shared_blob, float *y_perm, float *y_shared,
+                        unsigned *err, int max_groups, cudaStream_t s) {
     using Q = QT<BITS>;
-    const int NTS = NT;
-    const int max_groups = (T * k < E ? T * k : E) + (shared_blob ? 1 : 0);
-    const int sms = num_sms();
-    {
-        const size_t smem = static_cast<size_t>(NTS) * H * 4 + static_cast<size_t>(NTS) * (H / 32) * 4;
-        const int row_blocks = I / (kWarps * kRowsPerWarpGU);
-        long blocks = static_cast<long>(max_groups) * row_blocks;
-        if (blocks > sms * 8L) blocks = sms * 8L;
-        cudaFuncSetAttribute(k_gemv_gateup<BITS, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-        k_gemv_gateup<BITS, NT><<<blocks, 256, smem, s>>>(blobs, offsets, active, perm_src, x, x_bf16, T, k, H, I, E,
-                                                          shared_blob, hbuf, NTS, err); count_launches(1);
-    }
-    {
-        const int nch = I / Q::EPC;
-        int lpr = 1;
-        while (lpr * 2 <= nch && lpr * 2 <= 32) lpr *= 2;
-        const size_t smem = static_cast<size_t>(NTS) * I * 4 + static_cast<size_t>(NTS) * (I / 32) * 4;
-        const int rows_per_block = kWarps * kRowPassesD * (32 / lpr);
-        const int row_blocks = (H + rows_per_block - 1) / rows_per_block;
-        long blocks = static_cast<long>(max_groups) * row_blocks;
-        if (blocks > sms * 8L) blocks = sms * 8L;
-        cudaFuncSetAttribute(k_gemv_down<BITS, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-        k_gemv_down<BITS, NT><<<blocks, 256, smem, s>>>(blobs, offsets, active, hbuf, T, k, H, I, E, shared_blob,
-                                                        y_perm, y_shared, NTS, lpr, err); count_launches(1);
-    }
+    constexpr int IL = LPR * Q::EPC;
+    constexpr int RB = kGvWarps * GvTPW<BITS>::value * (32 / LPR);
+    const size_t smem = static_cast<size_t>(kGvNT) * IL * 4 + static_cast<size_t>(kGvNT) * (IL / 32) * 4;
+    long blocks = static_cast<long>(max_groups) * ((H + RB - 1) / RB);
+    if (blocks > num_sms() * 8L) blocks = num_sms() * 8L;
+    cudaFuncSetAttribute(k_gemv_down<BITS, LPR>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    k_gemv_down<BITS, LPR><<<blocks, kGvThreads, smem, s>>>(blobs, offsets, active, hbuf, T, k, H, E, shared_blob,
+                                                            y_perm, y_shared, err);
+    count_launches(1);
 }
 
 template <int BITS>
@@ -275,15 +249,24 @@ static int launch_gemv_t(const uint8_t *const *blobs, const int32_t *offsets, co
                          const int32_t *perm_src, const void *x, int x_bf16, int T, int k, int H, int I, int E,
                          const uint8_t *shared_blob, float *y_perm, float *y_shared, float *hbuf, unsigned *err,
                          cudaStream_t s) {
-#define MOE_GEMV_NT(N) \
-    launch_gemv_nt<BITS, N>(blobs, offsets, active, perm_src, x, x_bf16, T, k, H, I, E, shared_blob, y_perm, y_shared, \
-                            hbuf, err, s)
-    if (T <= 1) MOE_GEMV_NT(1);
-    else if (T <= 2) MOE_GEMV_NT(2);
-    else if (T <= 4) MOE_GEMV_NT(4);
-    else if (T <= 8) MOE_GEMV_NT(8);
-    else MOE_GEMV_NT(16);
-#undef MOE_GEMV_NT
+    using Q = QT<BITS>;
+    const int max_groups = (T * k < E ? T * k : E) + (shared_blob ? 1 : 0);
+    {
+        const size_t smem = static_cast<size_t>(kGvNT) * H * 4 + static_cast<size_t>(kGvNT) * (H / 32) * 4;
+        long blocks = static_cast<long>(max_groups) * (I / kGvRows);
+        if (blocks > num_sms() * 8L) blocks = num_sms() * 8L;
+        cudaFuncSetAttribute(k_gemv_gateup<BITS>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+        k_gemv_gateup<BITS><<<blocks, kGvThreads, smem, s>>>(blobs, offsets, active, perm_src, x, x_bf16, T, k, H, I,
+                                                             E, shared_blob, hbuf, err);
+        count_launches(1);
+    }
+    switch (I / Q::EPC) {
+        case 2: launch_down<BITS, 2>(blobs, offsets, active, hbuf, T, k, H, E, shared_blob, y_perm, y_shared, err, max_groups, s); break;
+        case 4: launch_down<BITS, 4>(blobs, offsets, active, hbuf, T, k, H, E, shared_blob, y_perm, y_shared, err, max_groups, s); break;
+        case 8: launch_down<BITS, 8>(blobs, offsets, active, hbuf, T, k, H, E, shared_blob, y_perm, y_shared, err, max_groups, s); break;
+        case 16: launch_down<BITS, 16>(blobs, offsets, active, hbuf, T, k, H, E, shared_blob, y_perm, y_shared, err, max_groups, s); break;
+        default: launch_down<BITS, 32>(blobs, offsets, active, hbuf, T, k, H, E, shared_blob, y_perm, y_shared, err, max_groups, s); break;
+    }
     return cuda_status(cudaGetLastError(), "expert GEMV launch");
 }
 

@@ -9,6 +9,9 @@ namespace moe {
 
 void launch_router_logits(const void *x, int x_dtype, const void *w, int w_dtype, const float *bias, int T, int H,
                           int E, float *out, cudaStream_t s);
+bool router_mma_supported(int x_dtype, int w_dtype, int T, int H);
+int launch_router_mma(const void *x, const void *w, const float *bias, int T, int H, int E, float *out,
+                      unsigned *err, cudaStream_t s);
 void launch_topk(const float *logits, int T, int E, int k, int32_t *ids, float *w, unsigned *err, cudaStream_t s);
 
 size_t permute_ws_bytes(int T, int k, int E);
@@ -16,12 +19,13 @@ int launch_permute(const int32_t *ids, int T, int k, int E, int32_t *offsets, in
                    int32_t *active, void *ws, unsigned *err, cudaStream_t s);
 
 size_t gemv_ws_bytes(int T, int k, int I);
+bool gemv_supported(int bits, int H, int I);
 int launch_gemv(int bits, const uint8_t *const *blobs, const int32_t *offsets, const int32_t *active,
                 const int32_t *perm_src, const void *x, int x_dtype, int T, int k, int H, int I, int E,
                 const uint8_t *shared_blob, float *y_perm, float *y_shared, void *ws, unsigned *err, cudaStream_t s);
 
 size_t gemm_ws_bytes(int bits, int T, int k, int H, int I, int E);
-bool gemm_supported(int T, int k, int E);
+bool gemm_supported(int bits, int T, int k, int H, int I, int E);
 int launch_gemm(int bits, const uint8_t *const *blobs, const int32_t *offsets, const int32_t *active,
                 const int32_t *perm_src, const void *x, int x_dtype, int T, int k, int H, int I, int E,
                 const uint8_t *shared_blob, float *y_perm, float *y_shared, void *ws, unsigned *err, cudaStream_t s);

@@ -73,6 +73,7 @@ extern "C" int moe_expert_ffn_noalloc(int bits, const void *const *expert_blobs,
     NA_REQUIRE(k >= 1 && k <= 32 && k <= E, "k must be in [1, min(E, 32)] (got k=%d, E=%d)", k, E);
     NA_REQUIRE(H >= 128 && H % 128 == 0 && H <= 2048, "H must be a multiple of 128 in [128, 2048] (got %d)", H);
     NA_REQUIRE(I >= 128 && I % 128 == 0 && I <= 2048, "I must be a multiple of 128 in [128, 2048] (got %d)", I);
+    NA_REQUIRE(gemv_supported(bits, H, I), "I/32 (4-bit) or I/64 (2-bit) must be 2, 4, 8, 16 or 32 (got I=%d)", I);
     if (T == 0) return MOE_OK;
     NA_REQUIRE(x_dtype == MOE_F32 || x_dtype == MOE_BF16, "x_dtype must be MOE_F32 or MOE_BF16");
     NA_REQUIRE(expert_blobs && expert_offsets && active && perm_src && x && y_perm,

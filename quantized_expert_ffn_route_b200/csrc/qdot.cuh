@@ -120,28 +120,32 @@ __device__ void stage_rows_fn(float4 *xs, float *cs, int NTS, int nt, int K, Row
     using Q = QT<BITS>;
     const int nch = K / Q::EPC;
     const int g4n = K / 4;
-    for (int idx = threadIdx.x; idx < NTS * g4n; idx += blockDim.x) {
-        const int t = idx / g4n, g4 = idx % g4n;
-        const int c = (4 * g4) / Q::EPC, q = ((4 * g4) % Q::EPC) / 4;
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (t < nt)
-            v = bf16 ? load4(static_cast<const __nv_bfloat16 *>(row_of(t)) + 4 * g4)
-                     : load4(static_cast<const float *>(row_of(t)) + 4 * g4);
-        xs[(t * Q::PPC + q) * nch + c] = v;
+#pragma unroll 1
+    for (int t = 0; t < NTS; ++t) {                 // divisors below are compile-time constants
+        const void *row = t < nt ? row_of(t) : nullptr;
+        for (int g4 = threadIdx.x; g4 < g4n; g4 += blockDim.x) {
+            const int c = g4 / Q::PPC, q = g4 % Q::PPC;
+            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (row)
+                v = bf16 ? load4(static_cast<const __nv_bfloat16 *>(row) + 4 * g4)
+                         : load4(static_cast<const float *>(row) + 4 * g4);
+            xs[(t * Q::PPC + q) * nch + c] = v;
+        }
     }
     __syncthreads();
     const int nblk = K / 32;
-    for (int idx = threadIdx.x; idx < NTS * nblk; idx += blockDim.x) {
-        const int t = idx / nblk, b = idx % nblk;
-        const int c = b / Q::BPC, beta = b % Q::BPC;
-        float s = 0.f;
+#pragma unroll 1
+    for (int t = 0; t < NTS; ++t)
+        for (int b = threadIdx.x; b < nblk; b += blockDim.x) {
+            const int c = b / Q::BPC, beta = b % Q::BPC;
+            float s = 0.f;
 #pragma unroll
-        for (int p = 0; p < 8; ++p) {
-            const float4 v = xs[(t * Q::PPC + 8 * beta + p) * nch + c];
-            s += v.x; s += v.y; s += v.z; s += v.w;
+            for (int p = 0; p < 8; ++p) {
+                const float4 v = xs[(t * Q::PPC + 8 * beta + p) * nch + c];
+                s += (v.x + v.y) + (v.z + v.w);
+            }
+            cs[t * nblk + b] = static_cast<float>(128 + Q::HALF) * s;
         }
-        cs[t * nblk + b] = static_cast<float>(128 + Q::HALF) * s;
-    }
     __syncthreads();
 }
 
@@ -163,40 +167,104 @@ template <int BITS>
 __device__ __forceinline__ void chunk_fx(const uint4 &code, const float4 (&xp)[QT<BITS>::PPC],
                                          float (&out)[QT<BITS>::BPC]) {
     const uint32_t words[4] = {code.x, code.y, code.z, code.w};
+    // Each packed FMA pairs neighbouring elements (j, j+1) of one code word
+    // with the neighbouring x values of one float4, so operands sit in
+    // register pairs as loaded.
     if constexpr (BITS == 4) {
-        float2 acc = make_float2(0.f, 0.f);
+        float2 lo = make_float2(0.f, 0.f);
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
             const uint32_t L = (words[m] & 0x0F0F0F0Fu) | 0x80808080u;
             const uint32_t Hh = ((words[m] >> 4) & 0x0F0F0F0Fu) | 0x80808080u;
             const float4 a = xp[m], b = xp[4 + m];   // elements 4m..4m+3 (low nibbles), 16+4m.. (high)
-            acc = __ffma2_rn(make_float2(magic(L, 0), magic(Hh, 0)), make_float2(a.x, b.x), acc);
-            acc = __ffma2_rn(make_float2(magic(L, 1), magic(Hh, 1)), make_float2(a.y, b.y), acc);
-            acc = __ffma2_rn(make_float2(magic(L, 2), magic(Hh, 2)), make_float2(a.z, b.z), acc);
-            acc = __ffma2_rn(make_float2(magic(L, 3), magic(Hh, 3)), make_float2(a.w, b.w), acc);
+            lo = __ffma2_rn(make_float2(magic(L, 0), magic(L, 1)), make_float2(a.x, a.y), lo);
+            lo = __ffma2_rn(make_float2(magic(L, 2), magic(L, 3)), make_float2(a.z, a.w), lo);
+            lo = __ffma2_rn(make_float2(magic(Hh, 0), magic(Hh, 1)), make_float2(b.x, b.y), lo);
+            lo = __ffma2_rn(make_float2(magic(Hh, 2), magic(Hh, 3)), make_float2(b.z, b.w), lo);
         }
-        out[0] = acc.x + acc.y;
+        out[0] = lo.x + lo.y;
     } else {
-        float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+        float2 acc[2][2] = {{make_float2(0.f, 0.f), make_float2(0.f, 0.f)},
+                            {make_float2(0.f, 0.f), make_float2(0.f, 0.f)}};
 #pragma unroll
         for (int wi = 0; wi < 4; ++wi) {
             const int beta = wi >> 1, m = wi & 1;
 #pragma unroll
-            for (int s = 0; s < 4; s += 2) {
-                const uint32_t L0 = ((words[wi] >> (2 * s)) & 0x03030303u) | 0x80808080u;
-                const uint32_t L1 = ((words[wi] >> (2 * s + 2)) & 0x03030303u) | 0x80808080u;
-                const float4 a = xp[8 * beta + 2 * s + m], b = xp[8 * beta + 2 * (s + 1) + m];
-                float2 v = acc[beta];
-                v = __ffma2_rn(make_float2(magic(L0, 0), magic(L1, 0)), make_float2(a.x, b.x), v);
-                v = __ffma2_rn(make_float2(magic(L0, 1), magic(L1, 1)), make_float2(a.y, b.y), v);
-                v = __ffma2_rn(make_float2(magic(L0, 2), magic(L1, 2)), make_float2(a.z, b.z), v);
-                v = __ffma2_rn(make_float2(magic(L0, 3), magic(L1, 3)), make_float2(a.w, b.w), v);
-                acc[beta] = v;
+            for (int s = 0; s < 4; ++s) {            // crumb level s: elements 8s + 4m + j of block beta
+                const uint32_t Ls = ((words[wi] >> (2 * s)) & 0x03030303u) | 0x80808080u;
+                const float4 a = xp[8 * beta + 2 * s + m];
+                float2 &v = acc[beta][s & 1];
+                v = __ffma2_rn(make_float2(magic(Ls, 0), magic(Ls, 1)), make_float2(a.x, a.y), v);
+                v = __ffma2_rn(make_float2(magic(Ls, 2), magic(Ls, 3)), make_float2(a.z, a.w), v);
             }
         }
-        out[0] = acc[0].x + acc[0].y;
-        out[1] = acc[1].x + acc[1].y;
+        out[0] = (acc[0][0].x + acc[0][0].y) + (acc[0][1].x + acc[0][1].y);
+        out[1] = (acc[1][0].x + acc[1][0].y) + (acc[1][1].x + acc[1][1].y);
     }
+}
+
+// chunk_fx for NV weight rows that share one chunk of x: the x pieces are
+// read from shared memory (piece q at xs[q * stride]) one code word at a
+// time and applied to all NV rows, so only two or four pieces are live.
+template <int BITS, int NV>
+__device__ __forceinline__ void rows_fx(const uint4 (&code)[NV], const float4 *xs, int stride,
+                                        float (&out)[NV][QT<BITS>::BPC]) {
+    if constexpr (BITS == 4) {
+        float2 acc[NV];
+#pragma unroll
+        for (int v = 0; v < NV; ++v) acc[v] = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            const float4 a = xs[m * stride], b = xs[(4 + m) * stride];
+#pragma unroll
+            for (int v = 0; v < NV; ++v) {
+                const uint32_t w = m == 0 ? code[v].x : m == 1 ? code[v].y : m == 2 ? code[v].z : code[v].w;
+                const uint32_t L = (w & 0x0F0F0F0Fu) | 0x80808080u;
+                const uint32_t Hh = ((w >> 4) & 0x0F0F0F0Fu) | 0x80808080u;
+                acc[v] = __ffma2_rn(make_float2(magic(L, 0), magic(L, 1)), make_float2(a.x, a.y), acc[v]);
+                acc[v] = __ffma2_rn(make_float2(magic(L, 2), magic(L, 3)), make_float2(a.z, a.w), acc[v]);
+                acc[v] = __ffma2_rn(make_float2(magic(Hh, 0), magic(Hh, 1)), make_float2(b.x, b.y), acc[v]);
+                acc[v] = __ffma2_rn(make_float2(magic(Hh, 2), magic(Hh, 3)), make_float2(b.z, b.w), acc[v]);
+            }
+        }
+#pragma unroll
+        for (int v = 0; v < NV; ++v) out[v][0] = acc[v].x + acc[v].y;
+    } else {
+        float2 acc[NV][2];
+#pragma unroll
+        for (int v = 0; v < NV; ++v) acc[v][0] = acc[v][1] = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int wi = 0; wi < 4; ++wi) {
+            const int beta = wi >> 1, m = wi & 1;
+            float4 xq[4];                            // crumb level s: elements 8s + 4m + j of block beta
+#pragma unroll
+            for (int sl = 0; sl < 4; ++sl) xq[sl] = xs[(8 * beta + 2 * sl + m) * stride];
+#pragma unroll
+            for (int v = 0; v < NV; ++v) {
+                const uint32_t w = wi == 0 ? code[v].x : wi == 1 ? code[v].y : wi == 2 ? code[v].z : code[v].w;
+#pragma unroll
+                for (int sl = 0; sl < 4; ++sl) {
+                    const uint32_t Ls = ((w >> (2 * sl)) & 0x03030303u) | 0x80808080u;
+                    acc[v][beta] = __ffma2_rn(make_float2(magic(Ls, 0), magic(Ls, 1)), make_float2(xq[sl].x, xq[sl].y),
+                                              acc[v][beta]);
+                    acc[v][beta] = __ffma2_rn(make_float2(magic(Ls, 2), magic(Ls, 3)), make_float2(xq[sl].z, xq[sl].w),
+                                              acc[v][beta]);
+                }
+            }
+        }
+#pragma unroll
+        for (int v = 0; v < NV; ++v) {
+            out[v][0] = acc[v][0].x + acc[v][0].y;
+            out[v][1] = acc[v][1].x + acc[v][1].y;
+        }
+    }
+}
+
+// Makes the compiler treat a code chunk as changed here, so the dequantised
+// values derived from it are rebuilt per token instead of being hoisted out
+// of a token loop (hoisting them would need 32-64 registers per chunk).
+__device__ __forceinline__ void opaque(uint4 &c) {
+    asm volatile("" : "+r"(c.x), "+r"(c.y), "+r"(c.z), "+r"(c.w));
 }
 
 // dot += sum over the chunk's blocks of d_b * (128 * fx_b - cs_b)

@@ -54,9 +54,9 @@ def test_noalloc_matches_workspace_entry_point(bits, T):
 def test_noalloc_rejects_oversized_calls():
     cap = M.moe_expert_ffn_noalloc_max_bytes()
     assert cap == 8 << 20
-    # T*(k+1)*I*4 bytes of scratch: T = 1024, k = 10, I = 2048 needs 92 MB
+    # T*(k+1)*I*4 bytes of scratch: T = 1024, k = 10, I = 2048 (2-bit) needs 92 MB
     p = torch.zeros(64, dtype=torch.int64, device="cuda")
     with pytest.raises(M.MoEError) as ei:
-        M.moe_expert_ffn_noalloc(4, p, p, p, p, p, M.MOE_BF16, 1024, 10, 2048, 2048, 512, None, p, None)
+        M.moe_expert_ffn_noalloc(2, p, p, p, p, p, M.MOE_BF16, 1024, 10, 2048, 2048, 512, None, p, None)
     assert ei.value.status == M.MOE_EINVAL
     assert "scratch" in M.moe_last_error()

@@ -273,37 +273,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(GemmArgs a, int tile_c
         const int nsc = K / 32;
         int cur = -1;
         TileEntry te{};
-        // warp 0 asks L2 for a whole tile's codes and scales (its rows are
-        // contiguous) one tile ahead, so the 16-byte copies below mostly hit L2
-        // and DRAM sees long sequential reads
-        auto prefetch_tile = [&](int i) {
-            if (i >= n_my) return;
-            const TileEntry tp = tiles[i];
-            const BlobView pv = blob_view(tp.blob, BITS, a.H, a.I);
-            constexpr uint32_t kPiece = 8192;
-#pragma unroll
-            for (int pm = 0; pm < 2; ++pm) {
-                const int m0 = tp.m0 + (GATEUP ? 0 : kBM * pm);
-                const int nrows = min(kBM, Mtot - m0);
-                if (nrows <= 0) continue;
-                const uint8_t *cbase = (GATEUP ? (pm ? pv.cu : pv.cg) : pv.cd) + static_cast<size_t>(m0) * rowbytes;
-                const size_t cbytes = static_cast<size_t>(nrows) * rowbytes;
-                for (size_t off = static_cast<size_t>(lane) * kPiece; off < cbytes; off += 32 * kPiece)
-                    prefetch_l2(cbase + off, static_cast<uint32_t>(min(static_cast<size_t>(kPiece), cbytes - off)));
-                const __half *sbase = (GATEUP ? (pm ? pv.su : pv.sg) : pv.sd) + static_cast<size_t>(m0) * nsc;
-                const size_t sbytes = static_cast<size_t>(nrows) * nsc * 2;
-                if (lane == 31 && (reinterpret_cast<uintptr_t>(sbase) & 15) == 0 && (sbytes & 15) == 0)
-                    prefetch_l2(sbase, static_cast<uint32_t>(sbytes));
-            }
-        };
-        if (warp == 0) prefetch_tile(0);
         auto issue = [&](long jr) {
             if (jr >= J) return;
             const int i = static_cast<int>(jr / nk), s = static_cast<int>(jr % nk);
             if (i != cur) {
                 te = tiles[i];
                 cur = i;
-                if (warp == 0) prefetch_tile(i + 1);
             }
             const BlobView bv = blob_view(te.blob, BITS, a.H, a.I);
             const uint8_t *codes = GATEUP ? (mat ? bv.cu : bv.cg) : bv.cd;
@@ -479,8 +454,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(GemmArgs a, int tile_c
                 for (int s = 0; s < nk && !abort_s; ++s) {
                     const long j = static_cast<long>(i) * nk + s;
                     const int sa = static_cast<int>(j % SA), sb = static_cast<int>(j % SB);
-                    if (!mbar_wait(fullA + sa, static_cast<uint32_t>((j / SA) & 1), kSpin) ||
-                        !mbar_wait(fullB + sb, static_cast<uint32_t>((j / SB) & 1), kSpin)) {
+                    if (!mbar_spin(fullA + sa, static_cast<uint32_t>((j / SA) & 1), kSpin * 16) ||
+                        !mbar_spin(fullB + sb, static_cast<uint32_t>((j / SB) & 1), kSpin * 16)) {
                         fail();
                         break;
                     }

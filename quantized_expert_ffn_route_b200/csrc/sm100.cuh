@@ -35,6 +35,23 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, long l
         if (mbar_try_wait(bar, parity)) return true;
     return false;
 }
+// Non-suspending test of the phase (for the one thread that issues MMAs,
+// which should see a completed phase at once).
+__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{ .reg .pred p; mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// Spins on mbar_test_wait, at most `limit` polls.  Returns false on timeout.
+__device__ __forceinline__ bool mbar_spin(uint64_t *bar, uint32_t parity, long limit) {
+    for (long i = 0; i < limit; ++i)
+        if (mbar_test_wait(bar, parity)) return true;
+    return false;
+}
 __device__ __forceinline__ void fence_barrier_init() {
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
@@ -60,11 +77,6 @@ __device__ __forceinline__ void cp_async4(uint32_t dst, const void *src) {
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
-
-// Asks L2 to fetch [src, src + bytes) (16-byte aligned, bytes a multiple of 16).
-__device__ __forceinline__ void prefetch_l2(const void *src, uint32_t bytes) {
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
-}
 
 // --------------------------------------------------------------- tcgen05
 __device__ __forceinline__ void tmem_alloc(uint32_t *dst_smem, uint32_t ncols) {

@@ -375,7 +375,8 @@ def bench_layer(args, world, rank, pk):
                 "frac": round(gbs / pk["hbm_gbs"], 4)}
     sha = src_hash("decode.cu" if fused else ("gemv.cu" if kind != "prefill" else "gemm_tc.cu"))
     roof["traffic"] = traffic_from_profiles("k_decode" if fused else f"expert_ffn_{kind}", sha)
-    roof["kernel"] = ("k_decode (moe_layer_decode: route + top-k + experts + combine, one launch)" if fused
+    roof["kernel"] = ("moe_layer_decode (k_dec_logits -> k_dec_gateup -> k_dec_down, chained by programmatic "
+                      "dependent launch; one call)" if fused
                       else "moe_expert_ffn (gate/up + down kernels)")
     roof["ms_per_launch"] = round(ffn_avg_ms, 5)
     roof["timing"] = ffn_timing
@@ -429,8 +430,7 @@ def bench_layer(args, world, rank, pk):
         cpu = {"value": round(ntok / dt, 3), "unit": "tokens/s", "cores": host_cores(), "kind": "oracle",
                "sample": f"{ntok} tokens of the {kind} workload through the fp64 oracle in batches of 8, {dt:.1f} s"}
 
-    cfg = {"workload": f"{kind}: hidden {H}, {E} experts + 1 shared, top-{k}, intermediate {I}, "
-                       f"{bits}-bit blocks of 32 + fp16 scale, {T} token(s)/step",
+    cfg = {"workload": workload_name(kind, H, E, k, I, bits, T),
            "tokens_per_step": T, "layer_copies": n_layers,
            "l2": f"inputs larger than L2: {n_layers} layer copies x {E + 1} experts x {blob} B rotate per step",
            "mode": "fused decode kernel" if fused else {0: "auto", 1: "gemv", 2: "gemm"}[mode],
@@ -586,6 +586,11 @@ def bench_paging(args, world, rank, pk):
                 launches=launches, config=cfg, dtype="fp32 (CUDA-core FMA on 2-bit codes)")
 
 
+def workload_name(kind, H, E, k, I, bits, T):
+    return (f"{kind}: hidden {H}, {E} experts + 1 shared, top-{k}, intermediate {I}, "
+            f"{bits}-bit blocks of 32 + fp16 scale, {T} token(s)/step")
+
+
 def bench_reference(args, world, rank):
     """The oracle on the host cores, each step a bounded sample (one token / window)."""
     import oracle
@@ -609,7 +614,9 @@ def bench_reference(args, world, rank):
         one(i)
     dt = time.perf_counter() - t0
     v = args.steps * T / dt
-    return dict(value=v, ms=dt * 1e3, T=T, kind=kind)
+    name = workload_name(kind, layer.H, layer.E, layer.k, layer.I, layer.bits,
+                         {"decode": 1, "verify": args.window, "prefill": args.chunk}[kind])
+    return dict(value=v, ms=dt * 1e3, T=T, kind=kind, name=name)
 
 
 def main():
@@ -642,9 +649,10 @@ def main():
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(r["ms"] / args.steps, 3),
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
                 "data": "synthetic (seeded)", "impl": "reference",
-                "config": {"workload": f"{r['kind']} (oracle: {r['T']} token(s) per step)"},
+                "config": {"workload": r["name"], "tokens_per_step": r["T"], "parallelism": "replicas x1"},
                 "cpu_baseline": {"value": round(r["value"], 4), "unit": "tokens/s", "cores": host_cores(),
-                                 "kind": "oracle", "sample": f"{args.steps} steps of {r['T']} token(s)"},
+                                 "kind": "oracle",
+                                 "sample": f"{args.steps} steps of {r['T']} token(s) of that workload"},
                 "e2e": {"value": round(r["value"], 4), "unit": "tokens/s", "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}}
         print(json.dumps(line), flush=True)

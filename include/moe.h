@@ -78,7 +78,6 @@ typedef struct CUstream_st *moe_stream_t;   /* same type as cudaStream_t */
 #define MOE_DEVERR_NONFINITE 4u      /* a selected logit was NaN or +inf */
 #define MOE_DEVERR_BAD_ROW 8u        /* offsets/perm_src inconsistent */
 #define MOE_DEVERR_TIMEOUT 16u       /* a bounded in-kernel wait ran out */
-#define MOE_DEVERR_WORKSPACE 32u     /* moe_layer_decode: the workspace ticket counter was not zero */
 
 /* Thread-local message of the last failing call ("" if none). */
 const char *moe_last_error(void);
@@ -180,18 +179,15 @@ int moe_expert_ffn_q2(const void *const *expert_blobs, const int32_t *expert_off
  * moe_expert_ffn_q4/q2 (GEMV mode) -> moe_combine (Strata article, section 2
  * item 2: only the experts the router picks are computed; at one token the
  * step is bound by streaming those experts' weights).  Three kernels chained
- * with programmatic dependent launch (route: logits over E/4 CTAs, the last
- * CTA to finish selects; then gate/up; then down + combine); no in-kernel
- * waits spin.
+ * with programmatic dependent launch (logits over E/4 CTAs; gate/up, whose
+ * routed CTAs each select the top-k; down + combine); no in-kernel waits
+ * spin.
  *  x [H] (x_dtype), w_router [E,H] (w_dtype) or NULL with logits_in [E];
  *  expert_blobs device [E] blob pointers; shared_blob or NULL;
  *  topk_ids [k] int32 out, topk_w [k] fp32 out, logits_out [E] or NULL
  *  (written only when the logits are computed here), y [H] fp32 out.
- *  ws: moe_layer_decode_ws_size() bytes of scratch, zero-filled before its
- *  first use with this call (e.g. one cudaMemsetAsync after allocation); it
- *  holds a ticket counter that every completed call leaves at zero.  A
- *  counter found non-zero sets MOE_DEVERR_WORKSPACE (the outputs of that
- *  call are then not valid).  Calls sharing one ws must not overlap.
+ *  ws: moe_layer_decode_ws_size() bytes of scratch (no initialisation
+ *  needed).  Calls sharing one ws must not overlap.
  * Supported shapes (else MOE_EINVAL: use the separate calls): E <= 1024,
  * k <= 32, H <= 2048 and a multiple of 128, I a multiple of 128 with I/32
  * (4-bit) or I/64 (2-bit) in {4, 8, 16, 32}, and the down kernel's tasks,

@@ -23,7 +23,7 @@ MOE_OK, MOE_EINVAL, MOE_ENOMEM, MOE_ECUDA, MOE_EBUSY, MOE_ETIMEDOUT, MOE_EIO, MO
 MOE_F32, MOE_BF16 = 0, 1
 MOE_MODE_AUTO, MOE_MODE_GEMV, MOE_MODE_GEMM = 0, 1, 2
 DEVERR_BAD_EXPERT, DEVERR_NULL_BLOB, DEVERR_NONFINITE, DEVERR_BAD_ROW = 1, 2, 4, 8
-MOE_DEVERR_TIMEOUT, MOE_DEVERR_WORKSPACE = 16, 32
+MOE_DEVERR_TIMEOUT = 16
 
 _STATUS = {1: "MOE_EINVAL", 2: "MOE_ENOMEM", 3: "MOE_ECUDA", 4: "MOE_EBUSY", 5: "MOE_ETIMEDOUT",
            6: "MOE_EIO", 7: "MOE_EDEVICE"}

@@ -2,13 +2,14 @@
 // programmatic dependent launch (each starts while its predecessor runs and
 // waits with griddepcontrol only where it reads the predecessor's results).
 //
-//   1. route (one warp per router row, E/4 CTAs): logits; the last CTA to
-//      finish (a ticket counter in the workspace) selects the top-k and
-//      writes ids and gates.  With caller-given logits it is one CTA that
-//      only selects.
+//   1. logits (one warp per router row, E/4 CTAs); skipped when the caller
+//      gives the logits.
 //   2. gate/up (all selected experts + the shared expert, 16 rows per CTA):
-//      h_g[i] = silu(Wg_g[i] . x) * (Wu_g[i] . x).  The shared expert's CTAs
-//      never wait for the route kernel.
+//      every routed CTA selects the top-k from the logits itself (a block
+//      top-k of well under a microsecond, cheaper than another kernel
+//      boundary or a grid-wide hand-off), then
+//      h_g[i] = silu(Wg_g[i] . x) * (Wu_g[i] . x); CTA 0 publishes ids and
+//      gates.  The shared expert's CTAs never wait for the logits.
 //   3. down + combine (a few output rows per CTA, all groups; each lane one
 //      chunk of one row): every code load is issued before h is staged, then
 //      y[r] = sum_j w_j (Wd_{e_j}[r] . h_j) + Wd_shared[r] . h_shared, summed
@@ -36,12 +37,11 @@ __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.lau
 __host__ __device__ inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
 // Workspace layout (bytes): ids [32] int32 @0 | gates [32] fp32 @128 |
-// ticket counter @256 | logits [E] @512 | h [(k+1) * I] fp32 (256-aligned).
-// The counter must be zero before the first call; every call leaves it zero.
+// logits [E] @512 | h [(k+1) * I] fp32 (256-aligned).  Nothing in it needs
+// to start at any value.
 struct DecodeWs {
     int32_t *ids;
     float *gates;
-    unsigned *ticket;
     float *logits;
     float *h;
 };
@@ -50,7 +50,6 @@ __host__ __device__ inline DecodeWs decode_ws(void *ws, int E) {
     DecodeWs w;
     w.ids = reinterpret_cast<int32_t *>(p);
     w.gates = reinterpret_cast<float *>(p + 128);
-    w.ticket = reinterpret_cast<unsigned *>(p + 256);
     w.logits = reinterpret_cast<float *>(p + 512);
     w.h = reinterpret_cast<float *>(p + 512 + ((static_cast<size_t>(E) * 4 + 255) / 256) * 256);
     return w;
@@ -151,19 +150,16 @@ __device__ void block_topk(const float *logits, int E, int k, uint64_t *cand, ui
     __syncthreads();
 }
 
-// ------------------------------------------------------------ 1. route
+// ------------------------------------------------------------ 1. logits
 // One warp per router row, kLogitRows rows per CTA, so the E rows are read by
 // E / kLogitRows SMs at once; every lane issues all of its weight loads
-// before it stages x.  Each CTA then takes a ticket; the CTA holding the last
-// one sees every logit (writes fenced before the ticket) and selects.
+// before it stages x.
 constexpr int kLogitRows = 4;
 
-__global__ void __launch_bounds__(kLogitRows * 32) k_dec_route(DecodeArgs a) {
+__global__ void __launch_bounds__(kLogitRows * 32) k_dec_logits(DecodeArgs a) {
     __shared__ __align__(16) float xs[2048];
-    __shared__ uint64_t cand[kLogitRows * 32], sel[32];
-    __shared__ unsigned ticket_s;
     pdl_trigger();                                       // the gate/up kernel may start its prologue
-    const int H = a.H, E = a.E, k = a.k;
+    const int H = a.H, E = a.E;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     if (!a.logits_in) {
         const int e = blockIdx.x * kLogitRows + warp;
@@ -214,41 +210,7 @@ __global__ void __launch_bounds__(kLogitRows * 32) k_dec_route(DecodeArgs a) {
                 const float l = s + (a.bias ? a.bias[e] : 0.f);
                 a.ws.logits[e] = l;
                 if (a.logits_out) a.logits_out[e] = l;
-                __threadfence();                         // visible before this CTA's ticket
             }
-        }
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) ticket_s = atomicAdd(a.ws.ticket, 1u);
-    __syncthreads();
-    const unsigned t = ticket_s;
-    if (t >= gridDim.x) {                                // the counter was not zero on entry
-        if (threadIdx.x == 0) report(a.err, MOE_DEVERR_WORKSPACE);
-        return;
-    }
-    if (t != gridDim.x - 1) return;
-    __threadfence();
-    block_topk<kLogitRows>(a.logits_in ? a.logits_in : a.ws.logits, E, k, cand, sel);
-    if (warp == 0) {
-        const uint64_t key = lane < k ? sel[lane] : 0ull;
-        const float my_v = key_float(static_cast<uint32_t>(key >> 32));
-        const int my_id = static_cast<int>(0xffffffffu - static_cast<uint32_t>(key));
-        const float v0 = __shfl_sync(0xffffffffu, my_v, 0);
-        const bool bad = lane < k && (my_v != my_v || my_v == __int_as_float(0x7f800000));
-        const bool any_bad = __any_sync(0xffffffffu, bad);
-        const float ex = lane < k ? expf(my_v - v0) : 0.f;
-        float sum = 0.f;
-        for (int j = 0; j < k; ++j) sum += __shfl_sync(0xffffffffu, ex, j);   // slot order
-        if (lane < k) {
-            const float wj = any_bad ? __int_as_float(0x7fc00000) : ex / sum;
-            a.ws.ids[lane] = my_id;
-            a.ws.gates[lane] = wj;
-            a.ids_out[lane] = my_id;
-            a.w_out[lane] = wj;
-        }
-        if (lane == 0) {
-            if (any_bad) report(a.err, MOE_DEVERR_NONFINITE);
-            *a.ws.ticket = 0u;                           // the next call starts from zero
         }
     }
 }
@@ -326,8 +288,29 @@ __global__ void __launch_bounds__(kDecThreads, 3) k_dec_gateup(DecodeArgs a) {
     if (shared_group) {
         load_codes(a.shared);                            // independent of the routing
     } else {
-        pdl_wait();                                      // ids are final from here on
-        const int e = __ldcg(a.ws.ids + g);
+        pdl_wait();                                      // the logits are final from here on
+        __shared__ uint64_t cand[kDecWarps * 32], sel[32];
+        block_topk<kDecWarps>(a.logits_in ? a.logits_in : a.ws.logits, a.E, k, cand, sel);
+        if (blockIdx.x == 0 && warp == 0) {              // one CTA publishes ids and gates
+            const uint64_t key = lane < k ? sel[lane] : 0ull;
+            const float my_v = key_float(static_cast<uint32_t>(key >> 32));
+            const int my_id = static_cast<int>(0xffffffffu - static_cast<uint32_t>(key));
+            const float v0 = __shfl_sync(0xffffffffu, my_v, 0);
+            const bool bad = lane < k && (my_v != my_v || my_v == __int_as_float(0x7f800000));
+            const bool any_bad = __any_sync(0xffffffffu, bad);
+            const float ex = lane < k ? expf(my_v - v0) : 0.f;
+            float sum = 0.f;
+            for (int j = 0; j < k; ++j) sum += __shfl_sync(0xffffffffu, ex, j);   // slot order
+            if (lane < k) {
+                const float wj = any_bad ? __int_as_float(0x7fc00000) : ex / sum;
+                a.ws.ids[lane] = my_id;
+                a.ws.gates[lane] = wj;
+                a.ids_out[lane] = my_id;
+                a.w_out[lane] = wj;
+            }
+            if (lane == 0 && any_bad) report(a.err, MOE_DEVERR_NONFINITE);
+        }
+        const int e = static_cast<int>(0xffffffffu - static_cast<uint32_t>(sel[g]));
         const uint8_t *blob = (e >= 0 && e < a.E) ? a.blobs[e] : nullptr;
         if (!blob) {
             if (threadIdx.x == 0) report(a.err, (e >= 0 && e < a.E) ? MOE_DEVERR_NULL_BLOB : MOE_DEVERR_BAD_EXPERT);
@@ -513,13 +496,13 @@ static int launch_decode_t(DecodeArgs a, int groups, cudaStream_t s) {
     cudaLaunchAttribute pdl;
     pdl.id = cudaLaunchAttributeProgrammaticStreamSerialization;
     pdl.val.programmaticStreamSerializationAllowed = 1;
-    // 1. route: logits over E/4 CTAs (one CTA that only selects when the caller gives logits)
-    {
+    // 1. router logits (skipped when the caller supplies them)
+    if (!a.logits_in) {
         cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(a.logits_in ? 1 : ceil_div(E, kLogitRows));
+        cfg.gridDim = dim3(ceil_div(E, kLogitRows));
         cfg.blockDim = dim3(kLogitRows * 32);
         cfg.stream = s;
-        int rc = cuda_status(cudaLaunchKernelEx(&cfg, k_dec_route, a), "decode route launch");
+        int rc = cuda_status(cudaLaunchKernelEx(&cfg, k_dec_logits, a), "decode logits launch");
         count_launches(1);
         if (rc) return rc;
     }
@@ -533,7 +516,7 @@ static int launch_decode_t(DecodeArgs a, int groups, cudaStream_t s) {
         cfg.dynamicSmemBytes = smem;
         cfg.stream = s;
         cfg.attrs = &pdl;
-        cfg.numAttrs = 1;
+        cfg.numAttrs = a.logits_in ? 0 : 1;              // x and given logits come from earlier work: no overlap
         int rc = cuda_status(cudaLaunchKernelEx(&cfg, k_dec_gateup<BITS>, a), "decode gate/up launch");
         count_launches(1);
         if (rc) return rc;

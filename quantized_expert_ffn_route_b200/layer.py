@@ -124,7 +124,7 @@ class MoELayer:
         return self._bufs[key]
 
     def decode_buffers(self):
-        """Buffers of the fused one-token step (the workspace starts zeroed, as it must)."""
+        """Buffers of the fused one-token step."""
         import torch
         from . import moe_layer_decode_ws_size
         if "decode" not in self._bufs:

@@ -374,7 +374,7 @@ def bench_layer(args, world, rank, pk):
         roof = {"bound": "hbm", "achieved": round(gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
                 "frac": round(gbs / pk["hbm_gbs"], 4)}
     sha = src_hash("decode.cu" if fused else ("gemv.cu" if kind != "prefill" else "gemm_tc.cu"))
-    roof["traffic"] = traffic_from_profiles("k_decode" if fused else f"expert_ffn_{kind}", sha)
+    roof["traffic"] = traffic_from_profiles("k_decode" if fused else f"expert_ffn_{kind}_{T}", sha)
     roof["kernel"] = ("moe_layer_decode (k_dec_logits -> k_dec_gateup -> k_dec_down, chained by programmatic "
                       "dependent launch; one call)" if fused
                       else "moe_expert_ffn (gate/up + down kernels)")

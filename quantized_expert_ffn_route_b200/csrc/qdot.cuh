@@ -38,66 +38,6 @@ __device__ __forceinline__ uint4 ldg_stream(const void *p) {
     return r;
 }
 
-// Accumulates one 16-byte code chunk against NT staged activation rows.
-// xs: float4 [NT][PPC][nch]; cs: float [NT][nch*BPC] (pre-scaled block sums).
-template <int BITS, int NT>
-__device__ __forceinline__ void chunk_dot(const uint4 &code, const float (&d)[QT<BITS>::BPC], const float4 *xs,
-                                          const float *cs, int nch, int c, float (&dot)[NT]) {
-    using Q = QT<BITS>;
-    float A[NT][2];
-#pragma unroll
-    for (int t = 0; t < NT; ++t) A[t][0] = A[t][1] = 0.f;
-    const uint32_t words[4] = {code.x, code.y, code.z, code.w};
-    if constexpr (BITS == 4) {
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
-            const uint32_t L = (words[m] & 0x0F0F0F0Fu) | 0x80808080u;
-            const uint32_t Hh = ((words[m] >> 4) & 0x0F0F0F0Fu) | 0x80808080u;
-            const float l0 = magic(L, 0), l1 = magic(L, 1), l2 = magic(L, 2), l3 = magic(L, 3);
-            const float h0 = magic(Hh, 0), h1 = magic(Hh, 1), h2 = magic(Hh, 2), h3 = magic(Hh, 3);
-#pragma unroll
-            for (int t = 0; t < NT; ++t) {
-                const float4 a = xs[(t * Q::PPC + m) * nch + c];
-                const float4 b = xs[(t * Q::PPC + 4 + m) * nch + c];
-                float s0 = A[t][0], s1 = A[t][1];
-                s0 = fmaf(l0, a.x, s0); s1 = fmaf(h0, b.x, s1);
-                s0 = fmaf(l1, a.y, s0); s1 = fmaf(h1, b.y, s1);
-                s0 = fmaf(l2, a.z, s0); s1 = fmaf(h2, b.z, s1);
-                s0 = fmaf(l3, a.w, s0); s1 = fmaf(h3, b.w, s1);
-                A[t][0] = s0; A[t][1] = s1;
-            }
-        }
-#pragma unroll
-        for (int t = 0; t < NT; ++t)
-            dot[t] = fmaf(d[0], fmaf(128.f, A[t][0] + A[t][1], -cs[t * nch + c]), dot[t]);
-    } else {
-#pragma unroll
-        for (int wi = 0; wi < 4; ++wi) {
-            const int beta = wi >> 1, m = wi & 1;
-#pragma unroll
-            for (int s = 0; s < 4; ++s) {
-                const uint32_t Ls = ((words[wi] >> (2 * s)) & 0x03030303u) | 0x80808080u;
-                const float f0 = magic(Ls, 0), f1 = magic(Ls, 1), f2 = magic(Ls, 2), f3 = magic(Ls, 3);
-                const int piece = 8 * beta + 2 * s + m;
-#pragma unroll
-                for (int t = 0; t < NT; ++t) {
-                    const float4 a = xs[(t * Q::PPC + piece) * nch + c];
-                    float v = A[t][beta];
-                    v = fmaf(f0, a.x, v); v = fmaf(f1, a.y, v); v = fmaf(f2, a.z, v); v = fmaf(f3, a.w, v);
-                    A[t][beta] = v;
-                }
-            }
-        }
-#pragma unroll
-        for (int t = 0; t < NT; ++t) {
-            float r = dot[t];
-            r = fmaf(d[0], fmaf(128.f, A[t][0], -cs[(t * nch + c) * 2 + 0]), r);
-            r = fmaf(d[1], fmaf(128.f, A[t][1], -cs[(t * nch + c) * 2 + 1]), r);
-            dot[t] = r;
-        }
-    }
-}
-
 template <int BITS>
 __device__ __forceinline__ void load_scales(const __half *row_scales, int c, bool valid, float (&d)[QT<BITS>::BPC]) {
     if constexpr (BITS == 4) {
@@ -149,10 +89,6 @@ __device__ void stage_rows_fn(float4 *xs, float *cs, int NTS, int nt, int K, Row
     __syncthreads();
 }
 
-template <int BITS>
-__device__ void stage_rows(float4 *xs, float *cs, int NTS, int nt, int K, const void *const *rows, int bf16) {
-    stage_rows_fn<BITS>(xs, cs, NTS, nt, K, [rows](int t) { return rows[t]; }, bf16);
-}
 
 }  // namespace moe
 

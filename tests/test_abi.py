@@ -120,3 +120,25 @@ def test_fused_decode_shape_checks_on_host():
         rc = L.moe_layer_decode(bits, p, M.MOE_BF16, p, M.MOE_BF16, None, None, p, p, H, I, E, k, p, p, None, p,
                                 p, M.moe_layer_decode_ws_size(E, k, I), None)
         assert rc == M.MOE_EINVAL
+
+
+def test_ffn_mode_shape_rules_on_host():
+    """GEMV takes I/32 (4-bit) or I/64 (2-bit) in {2, 4, 8, 16, 32}; AUTO falls
+    back to GEMM for other intermediates; GEMM takes at most 4095 groups."""
+    buf = np.zeros(1 << 16, np.int32)
+    p = buf.ctypes.data
+    L = M.lib()
+    gemm_ws = M.moe_expert_ffn_ws_size(4, 4, 2, 256, 384, 16, M.MOE_MODE_GEMM)
+    gemv_ws = M.moe_expert_ffn_ws_size(4, 4, 2, 256, 384, 16, M.MOE_MODE_GEMV)
+    assert M.moe_expert_ffn_ws_size(4, 4, 2, 256, 384, 16, M.MOE_MODE_AUTO) == gemm_ws != gemv_ws
+    assert M.moe_expert_ffn_ws_size(4, 4, 2, 256, 512, 16, M.MOE_MODE_AUTO) == \
+        M.moe_expert_ffn_ws_size(4, 4, 2, 256, 512, 16, M.MOE_MODE_GEMV)
+    f = L.moe_expert_ffn_q4
+    rc = f(p, p, p, p, p, 1, 4, 2, 256, 384, 16, None, p, None, M.MOE_MODE_GEMV, p, 1 << 20, None)
+    assert rc == M.MOE_EINVAL and "GEMV mode" in M.moe_last_error()
+    # 32768 experts and 4096 * 2 pairs: 4097 groups is one too many for GEMM
+    rc = f(p, p, p, p, p, 1, 4096, 2, 256, 256, 32768, None, p, None, M.MOE_MODE_GEMM, p, 1 << 30, None)
+    assert rc == M.MOE_EINVAL and "GEMM" in M.moe_last_error()
+    # the allocation-free call takes the GEMV shapes only
+    rc = L.moe_expert_ffn_noalloc(4, p, p, p, p, p, 1, 1, 2, 256, 2048, 16, None, p, None, None)
+    assert rc == M.MOE_EINVAL and "I/32" in M.moe_last_error()

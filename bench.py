@@ -392,10 +392,11 @@ def bench_layer(args, world, rank, pk):
         yh = torch.empty(T * H, dtype=torch.float32).pin_memory()
         xd = torch.empty(T, H, dtype=torch.bfloat16, device="cuda")
         s = torch.cuda.current_stream()
+        prepared = [c.prepare_decode(xd, M.MOE_BF16, stream=s, bufs=dbuf) for c in copies] if fused else None
         for i in range(3):
             xd.copy_(xh[:T], non_blocking=True)
             if fused:
-                copies[i % n_layers].forward_decode(xd, M.MOE_BF16, bufs=dbuf)
+                prepared[i % n_layers]()
                 yh.copy_(dbuf["y"][:H], non_blocking=True)
             else:
                 copies[i % n_layers].forward(xd, M.MOE_BF16, T=T, mode=mode, bufs=bufs)
@@ -408,7 +409,7 @@ def bench_layer(args, world, rank, pk):
             j = i * T if kind != "prefill" else 0
             xd.copy_(xh[j:j + T], non_blocking=True)
             if fused:
-                copies[i % n_layers].forward_decode(xd, M.MOE_BF16, bufs=dbuf)
+                prepared[i % n_layers]()
                 yh.copy_(dbuf["y"][:H], non_blocking=True)
             else:
                 copies[i % n_layers].forward(xd, M.MOE_BF16, T=T, mode=mode, bufs=bufs)
@@ -419,7 +420,8 @@ def bench_layer(args, world, rank, pk):
         e_ms = max_over_ranks(a.elapsed_time(b2), world)
         e2e = {"value": round(sum_over_ranks(n_e2e * T, world) / (e_ms / 1e3), 1), "unit": "tokens/s",
                "h2d_bytes_per_step": T * H * 2, "d2h_bytes_per_step": T * H * 4, "steps": n_e2e,
-               "note": ("MoELayer.forward_decode" if fused else "MoELayer.forward") +
+               "note": ("MoELayer.prepare_decode (one moe_layer_decode call per step)" if fused
+                        else "MoELayer.forward") +
                        " via the C ABI; pinned host x in, fp32 y out, stream sync every step"}
 
     cpu = None

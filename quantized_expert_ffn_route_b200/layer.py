@@ -147,6 +147,25 @@ class MoELayer:
                          b["w"], b["logits"], b["y"], b["ws"], b["ws_bytes"], stream)
         return b
 
+    def prepare_decode(self, x, x_dtype, stream=None, bufs=None):
+        """A prepared one-token step on fixed buffers: every argument of
+        moe_layer_decode is marshalled once, so each call of the returned
+        function is one C call (the step reads x from the same device buffer
+        and runs on the stream given, or current, at preparation)."""
+        from . import _check, _p, _stream, lib
+        b = bufs or self.decode_buffers()
+        fn = lib().moe_layer_decode
+        args = (self.bits, _p(x), x_dtype, _p(self.w_router), self.w_dtype, _p(self.bias), None, _p(self.table),
+                _p(self.shared), self.H, self.I, self.E, self.k, _p(b["ids"]), _p(b["w"]), _p(b["logits"]),
+                _p(b["y"]), _p(b["ws"]), b["ws_bytes"], _stream(stream))
+
+        def step():
+            rc = fn(*args)
+            if rc:
+                _check(rc)
+            return b
+        return step
+
     def forward(self, x, x_dtype, T=None, mode=0, logits_in=None, stream=None, bufs=None):
         """x: device tensor [T, H] (float32 or bfloat16); returns the StepBuffers (y in bufs.y)."""
         from . import moe_combine, moe_expert_ffn_q2, moe_expert_ffn_q4, moe_permute, moe_route_topk

@@ -312,6 +312,24 @@ def _run_fused(g, x, x_dtype, logits_in=None):
                 w=b["w"][:g.k].cpu().numpy(), logits=b["logits"].cpu().numpy(), y=b["y"].cpu().numpy())
 
 
+def test_prepared_decode_matches_forward_decode():
+    """The prepared one-token call runs the same kernels on the same buffers."""
+    layer = W.make_layer(430, 4, 256, 256, 24, 4, shared=True, w_dtype="bf16")
+    x = W.make_tokens(431, 3, 256, "bf16")
+    g = _layer_gpu(layer)
+    xd = torch.empty(1, 256, dtype=torch.bfloat16, device="cuda")
+    step = g.prepare_decode(xd, M.MOE_BF16)
+    for t in range(3):
+        xd.copy_(dev_x(x[t:t + 1], "bf16"))
+        b = step()
+        torch.cuda.synchronize()
+        y1, ids1 = b["y"].clone(), b["ids"][:4].clone()
+        f = _run_fused(g, x[t:t + 1], "bf16")
+        assert f["err"] == 0
+        assert np.array_equal(ids1.cpu().numpy(), f["ids"])
+        assert np.array_equal(y1.cpu().numpy(), f["y"])
+
+
 def test_fused_decode_full_size(decode_layer):
     layer, g = decode_layer
     x = W.make_tokens(W.SEED["decode"] + 500, 6, layer.H, "bf16")

@@ -9,9 +9,11 @@
 // steps of 64.  Weights are the MMA's A operand (M = 128), tokens the N side,
 // so a group of ten tokens still fills the datapath ("swap AB"); both
 // matrices share the token tile.  Roles of one persistent CTA per SM:
-//   warps 0-15  each thread copies the codes + scale of one 32-weight block a
-//               few k-steps ahead (cp.async into private slots) and
-//               dequantises it to fp16 into a 128-byte-swizzled A stage;
+//   warps 0-15  copy the weight codes of a tile's rows, a few k-steps at a
+//               time, into raw slots (each row's span is contiguous, so the
+//               copies are whole lines), then each thread dequantises one
+//               32-weight block per k-step to fp16 into a 128-byte-swizzled
+//               A stage;
 //   warps 21-22 gather the tile's token rows (fp16) into the B stages with
 //               cp.async, a few k-steps ahead; each warp publishes a stage
 //               with one barrier arrival once its copies have landed;
@@ -54,26 +56,29 @@ struct TileEntry {
 template <int BITS, bool GATEUP, int MAXN>
 struct GemmCfg {
     static constexpr int CODE = 32 * BITS / 8;                // code bytes of one block
+    static constexpr int CBK = 2 * CODE;                      // code bytes of one row per k-step
     static constexpr int SA = MAXN > 128 ? 2 : 3;             // A (dequantised weight) stages
-    static constexpr int SB = MAXN > 128 ? 4 : 8;             // B (token row) stages
-    static constexpr int L = MAXN > 128 ? 2 : 4;              // k-steps the code copies run ahead (= slots)
+    static constexpr int SB = MAXN > 128 ? 3 : 4;             // B (token row) stages
+    static constexpr int R = 2;                               // raw-code slots
+    static constexpr int KSMAX = MAXN > 128 ? 2 : 4;          // k-steps per raw slot
+    static constexpr int CS = KSMAX * CBK + 16;               // padded row stride of a slot's codes
     static constexpr int ACC = 2 * MAXN * 2 <= 512 ? 2 : 1;   // TMEM accumulator buffers
     static constexpr int TMEM_COLS = ACC * 2 * MAXN <= 128 ? 128 : (ACC * 2 * MAXN <= 256 ? 256 : 512);
     static constexpr size_t A_STAGE = static_cast<size_t>(2) * kBM * 128;
     static constexpr size_t B_STAGE = static_cast<size_t>(MAXN) * 128;
-    static constexpr size_t RC_STAGE = static_cast<size_t>(kDeq) * CODE;
-    static constexpr size_t RS_STAGE = static_cast<size_t>(kDeq) * 4;
+    static constexpr size_t RAW_CODES = static_cast<size_t>(2 * kBM) * CS;
+    static constexpr size_t RAW_SLOT = RAW_CODES + static_cast<size_t>(2 * kBM) * 16;   // + 16 B of scales per row
     static constexpr size_t OFF_A = 0;
     static constexpr size_t OFF_B = OFF_A + SA * A_STAGE;
-    static constexpr size_t OFF_RC = OFF_B + SB * B_STAGE;
-    static constexpr size_t OFF_RS = OFF_RC + L * RC_STAGE;
-    static constexpr size_t OFF_TOK = OFF_RS + L * RS_STAGE;
+    static constexpr size_t OFF_RAW = OFF_B + SB * B_STAGE;
+    static constexpr size_t OFF_TOK = OFF_RAW + R * RAW_SLOT;
     static constexpr size_t OFF_BAR = (OFF_TOK + MAXN * 4 + 15) / 16 * 16;
     static constexpr size_t OFF_TILES = OFF_BAR + 32 * 8 + 16;   // bars, TMEM address, tile count, abort flag
     static constexpr size_t FIXED = OFF_TILES + 1024;            // + slack for 1024-byte alignment
     static size_t smem(int cap) { return FIXED + static_cast<size_t>(cap) * sizeof(TileEntry); }
-    static_assert(2 * SA + 2 * SB + 5 <= 32, "barrier slots");
+    static_assert(2 * SA + 2 * SB + 5 + 2 * R <= 32, "barrier slots");
     static_assert(SB * B_STAGE >= (kMaxGroups + 1) * 4, "group scratch fits the B ring");
+    static_assert(KSMAX * 4 <= 16, "scale bytes of a row per slot");
     static_assert(FIXED <= kSmemLimit, "shared memory per block");
 };
 
@@ -160,17 +165,17 @@ __device__ __forceinline__ void dequant_block(const uint8_t *codes, __half2 d2, 
 template <int BITS, bool GATEUP, int MAXN>
 __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(GemmArgs a, int tile_cap) {
     using Cfg = GemmCfg<BITS, GATEUP, MAXN>;
-    constexpr int SA = Cfg::SA, SB = Cfg::SB, L = Cfg::L, ACC = Cfg::ACC;
+    constexpr int SA = Cfg::SA, SB = Cfg::SB, R = Cfg::R, ACC = Cfg::ACC;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sA = smem + Cfg::OFF_A;
     uint8_t *sB = smem + Cfg::OFF_B;
-    uint8_t *sRC = smem + Cfg::OFF_RC;
-    uint8_t *sRS = smem + Cfg::OFF_RS;
+    uint8_t *sRaw = smem + Cfg::OFF_RAW;
     int32_t *tok_s = reinterpret_cast<int32_t *>(smem + Cfg::OFF_TOK);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::OFF_BAR);
     uint64_t *fullA = bars, *emptyA = bars + SA, *fullB = bars + 2 * SA, *emptyB = bars + 2 * SA + SB;
     uint64_t *accF = bars + 2 * SA + 2 * SB, *accE = accF + 2, *drain = accF + 4;
+    uint64_t *rawFull = drain + 1, *rawEmpty = rawFull + R;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 32);
     volatile int &abort_s = *(reinterpret_cast<int *>(bars + 32) + 2);   // read in loop conditions: never cached
     TileEntry *tiles = reinterpret_cast<TileEntry *>(smem + Cfg::OFF_TILES);
@@ -182,6 +187,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(GemmArgs a, int tile_c
     const int MROWS = GATEUP ? kBM : 2 * kBM;          // weight rows a tile advances by
     const int MT = (Mtot + MROWS - 1) / MROWS;
     const int nk = K / kBK;
+    // k-steps per raw-code slot: the largest of KSMAX, 2, 1 dividing nk (a
+    // slot never spans two tiles)
+    const int KS = nk % Cfg::KSMAX == 0 ? Cfg::KSMAX : (nk % 2 == 0 ? 2 : 1);
     const int n_act = min(max(a.active[0], 0), min(a.E, a.T * a.k));
     const int ng = min(n_act + (a.shared ? 1 : 0), kMaxGroups);
 
@@ -200,6 +208,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(GemmArgs a, int tile_c
             mbar_init(accE + i, 4);                     // one arrival per epilogue warp
         }
         mbar_init(drain, 1);
+        for (int i = 0; i < R; ++i) {
+            mbar_init(rawFull + i, kDeq / 32);         // one arrival per dequantising warp
+            mbar_init(rawEmpty + i, kDeq / 32);
+        }
         fence_barrier_init();
         fence_proxy_async();
     }
@@ -267,39 +279,75 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(GemmArgs a, int tile_c
 
     if (warp < kEpiWarp0) {
         // ------------------------------------------------- dequantisation
-        // thread -> (row, matrix, block of the k-step)
+        // The 512 threads first copy, together, the codes of KS k-steps of the
+        // tile's 256 weight rows into a raw slot: each row's span is
+        // contiguous in the blob, so eight lanes cover 128 bytes of one row
+        // and a warp instruction touches four whole lines.  Slots are handed
+        // over with (bounded) barriers: rawFull when every warp's copies
+        // landed, rawEmpty when every warp has read the slot.  Then each
+        // thread dequantises one 32-weight block per k-step, thread -> (row,
+        // matrix, block), from the slot into a 128-byte-swizzled A stage.
         const int row = tid & 127, mat = (tid >> 7) & 1, half = tid >> 8;
+        const int r = mat * kBM + row;
         const size_t rowbytes = static_cast<size_t>(K) * BITS / 8;
         const int nsc = K / 32;
-        int cur = -1;
-        TileEntry te{};
-        auto issue = [&](long jr) {
-            if (jr >= J) return;
-            const int i = static_cast<int>(jr / nk), s = static_cast<int>(jr % nk);
-            if (i != cur) {
-                te = tiles[i];
-                cur = i;
-            }
+        const long U = J / KS;
+        auto issue = [&](long u) {                     // copies of slot u (all threads)
+            if (u >= U) return;
+            const long j0 = u * KS;
+            const TileEntry te = tiles[j0 / nk];
+            const int s0 = static_cast<int>(j0 % nk);
             const BlobView bv = blob_view(te.blob, BITS, a.H, a.I);
-            const uint8_t *codes = GATEUP ? (mat ? bv.cu : bv.cg) : bv.cd;
-            const __half *scl = GATEUP ? (mat ? bv.su : bv.sg) : bv.sd;
-            const int m = te.m0 + (GATEUP ? 0 : kBM * mat) + row;
-            const bool ok = m < Mtot;
-            const size_t mm = ok ? static_cast<size_t>(m) : 0;
-            const uint8_t *src = codes + mm * rowbytes + static_cast<size_t>(2 * s + half) * Cfg::CODE;
-            const int slot = static_cast<int>(jr % L);
-            const uint32_t dc = smem_addr(sRC + slot * Cfg::RC_STAGE + static_cast<size_t>(tid) * Cfg::CODE);
-            if constexpr (Cfg::CODE == 16) cp_async16(dc, src, ok ? 16u : 0u);
-            else cp_async8z(dc, src, ok ? 8u : 0u);
-            cp_async4z(smem_addr(sRS + slot * Cfg::RS_STAGE + static_cast<size_t>(tid) * 4), scl + mm * nsc + 2 * s,
-                       ok ? 4u : 0u);
+            uint8_t *raw = sRaw + (u % R) * Cfg::RAW_SLOT;
+            const int cpr = KS * Cfg::CBK / 16;        // 16-byte chunks of one row
+            for (int q = tid; q < 2 * kBM * cpr; q += kDeq) {
+                const int rr = q / cpr, c = q - rr * cpr;
+                const int mt = rr >> 7, m = te.m0 + (GATEUP ? 0 : kBM * mt) + (rr & 127);
+                const bool ok = m < Mtot;
+                const uint8_t *codes = GATEUP ? (mt ? bv.cu : bv.cg) : bv.cd;
+                cp_async16(smem_addr(raw + rr * Cfg::CS + c * 16),
+                           codes + (ok ? static_cast<size_t>(m) : 0) * rowbytes + s0 * Cfg::CBK + c * 16, ok ? 16u : 0u);
+            }
+            if (tid < 2 * kBM) {                       // one row's scales: 4*KS bytes
+                const int mt = tid >> 7, m = te.m0 + (GATEUP ? 0 : kBM * mt) + (tid & 127);
+                const bool ok = m < Mtot;
+                const __half *scl = (GATEUP ? (mt ? bv.su : bv.sg) : bv.sd) + (ok ? static_cast<size_t>(m) : 0) * nsc +
+                                    2 * s0;
+                const uint32_t dst = smem_addr(raw + Cfg::RAW_CODES + tid * 16);
+                if (KS == 4) cp_async16(dst, scl, ok ? 16u : 0u);
+                else if (KS == 2) cp_async8z(dst, scl, ok ? 8u : 0u);
+                else cp_async4z(dst, scl, ok ? 4u : 0u);
+            }
         };
-        for (int p = 0; p < L; ++p) {                  // prologue: one commit group per k-step
-            issue(p);
-            cp_async_commit();
-        }
+        issue(0);
+        cp_async_commit();
         for (long j = 0; j < J && !aborted(); ++j) {
-            cp_async_wait<L - 1>();                    // this thread's codes of k-step j have landed
+            const long u = j / KS;
+            const int sl = static_cast<int>(j - u * KS), slot = static_cast<int>(u % R);
+            if (sl == 0) {
+                // the next slot: wait until every warp has read its previous
+                // contents (slot u + 1 - R), then copy
+                int ok = 1;
+                if (lane == 0 && u + 1 >= R)
+                    ok = mbar_wait(rawEmpty + (u + 1) % R, static_cast<uint32_t>(((u + 1 - R) / R) & 1), kSpin);
+                if (!__shfl_sync(0xffffffffu, ok, 0)) {
+                    fail();
+                    break;
+                }
+                issue(u + 1);
+                cp_async_commit();
+                cp_async_wait<1>();                    // this thread's copies of slot u have landed
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(rawFull + slot);
+                    ok = mbar_wait(rawFull + slot, static_cast<uint32_t>((u / R) & 1), kSpin);
+                }
+                if (!__shfl_sync(0xffffffffu, ok, 0)) {
+                    fail();
+                    break;
+                }
+                __syncwarp();                          // the lanes read the slot after lane 0's acquire
+            }
             const int sa = static_cast<int>(j % SA);
             // one lane per warp polls the stage barrier; the warp follows it
             int ok = 1;
@@ -308,17 +356,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(GemmArgs a, int tile_c
                 fail();
                 break;
             }
-            const int slot = static_cast<int>(j % L);
-            const __half2 s01 = *reinterpret_cast<const __half2 *>(sRS + slot * Cfg::RS_STAGE + static_cast<size_t>(tid) * 4);
+            const uint8_t *raw = sRaw + slot * Cfg::RAW_SLOT;
+            const __half2 s01 = *reinterpret_cast<const __half2 *>(raw + Cfg::RAW_CODES + r * 16 + sl * 4);
             const uint32_t a_row = smem_addr(sA + sa * Cfg::A_STAGE + static_cast<size_t>(mat) * kBM * 128 +
                                              static_cast<size_t>(row) * 128);
-            dequant_block<BITS>(sRC + slot * Cfg::RC_STAGE + static_cast<size_t>(tid) * Cfg::CODE,
+            dequant_block<BITS>(raw + r * Cfg::CS + sl * Cfg::CBK + half * Cfg::CODE,
                                 half ? __high2half2(s01) : __low2half2(s01), a_row, 4 * half, row & 7);
             fence_proxy_async();                       // this thread's A writes -> async proxy
             __syncwarp();                              // ... ordered before lane 0's release-arrive
-            if (lane == 0) mbar_arrive(fullA + sa);
-            issue(j + L);                              // into the slot just read
-            cp_async_commit();
+            if (lane == 0) {
+                mbar_arrive(fullA + sa);
+                if (sl == KS - 1) mbar_arrive(rawEmpty + slot);   // this warp is done with slot u
+            }
         }
         cp_async_wait<0>();
     } else if (warp >= kLoadWarp0) {

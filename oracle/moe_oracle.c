@@ -6,9 +6,9 @@
  * shares no code with it: no header, helper, table or constant generator.
  *
  * What it computes (the pages describe the step in words only; the formulas
- * below are the plain definitions, in the order the pages give the flow:
- * "the router picks experts, resident ones are computed at once, the rest
- * are fetched first" -- Strata article, section 2 item 2):
+ * below are the plain definitions, in the order of the flow the Strata
+ * article gives in section 2 item 2: routing first, then the selected
+ * experts -- those in VRAM at once, the others after they are moved in):
  *
  *   dequant   w = d * (q - 2^(b-1)), blocks of 32 codes with one fp16 scale
  *             (27B dense report: Q4_0 costs 0.5625 B per value; Strata

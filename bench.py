@@ -437,6 +437,8 @@ def bench_layer(args, world, rank, pk):
            "l2": f"inputs larger than L2: {n_layers} layer copies x {E + 1} experts x {blob} B rotate per step",
            "mode": "fused decode kernel" if fused else {0: "auto", 1: "gemv", 2: "gemm"}[mode],
            "parallelism": f"replicas x{world}"}
+    if kind == "verify":
+        cfg["routing"] = routing_stats(step, bufs, T, k, n_steps)
     return dict(value=value, ms=ms_max, steps=args.steps, roofline=roof, e2e=e2e, cpu=cpu, clocks=clk,
                 launches=launches, config=cfg, dtype="fp32 (CUDA-core FMA on 4-bit codes)" if kind == "decode"
                 else ("fp32 (CUDA-core FMA on 2-bit codes)" if kind == "verify" else "fp16 tensor cores, fp32 accum"))
@@ -586,6 +588,32 @@ def bench_paging(args, world, rank, pk):
            "l2": "weights paged from host; HBM slots 2 GB > L2", "parallelism": f"replicas x{world}"}
     return dict(value=value, ms=ms, steps=args.steps, roofline=roof, e2e=e2e, cpu=cpu, clocks=clk,
                 launches=launches, config=cfg, dtype="fp32 (CUDA-core FMA on 2-bit codes)")
+
+
+def expert_stats(ids_per_step, hot=42):
+    """Routing of some steps (one int array of selected ids per step): mean
+    distinct experts per step and the share of selections that fall on the
+    `hot` most often selected experts."""
+    distinct = [len(np.unique(a)) for a in ids_per_step]
+    allids = np.concatenate([np.asarray(a).ravel() for a in ids_per_step])
+    counts = np.sort(np.bincount(allids))[::-1]
+    return {"distinct_experts_per_step": round(float(np.mean(distinct)), 2),
+            f"top{hot}_share": round(float(counts[:hot].sum() / max(1, allids.size)), 4),
+            "steps": len(ids_per_step)}
+
+
+def routing_stats(step, bufs, T, k, n_steps, n=64):
+    """Runs n steps eagerly and reads the selected ids back (verify windows)."""
+    import torch
+    try:
+        got = []
+        for i in range(min(n, n_steps)):
+            step(i)
+            torch.cuda.synchronize()
+            got.append(bufs.ids[:T * k].cpu().numpy())
+        return expert_stats(got)
+    except Exception as e:                             # a statistic only: never lose the bench line
+        return {"error": str(e)[:200]}
 
 
 def workload_name(kind, H, E, k, I, bits, T):

@@ -35,3 +35,13 @@ def test_traffic_lookup_matches_source_hash(tmp_path, monkeypatch):
     assert bench.traffic_from_profiles("k_decode", sha) == 12345.0
     assert bench.traffic_from_profiles("k_decode", "ffffffffffffffff") is None
     assert bench.traffic_from_profiles("expert_ffn_prefill_512", sha) is None
+
+
+def test_expert_stats():
+    import numpy as np
+    import bench
+    steps = [np.array([[0, 1], [1, 2]]), np.array([[3, 4], [3, 5]])]
+    st = bench.expert_stats(steps, hot=2)
+    assert st["distinct_experts_per_step"] == 3.0          # {0,1,2} and {3,4,5}
+    assert st["top2_share"] == 0.5                         # experts 1 and 3 take 4 of 8 selections
+    assert st["steps"] == 2

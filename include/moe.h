@@ -101,7 +101,9 @@ size_t moe_expert_blob_bytes(int bits, int H, int I);
  * Router logits and top-k gate (Strata article, summary table and section 2
  * item 2: 10 of 24,576 experts per token; the router's choice decides the
  * compute path).
- *   l[t,e]  = sum_h x[t,h] * w_router[e,h] (+ bias[e]), fp32 accumulation;
+ *   l[t,e]  = sum_h x[t,h] * w_router[e,h] (+ bias[e]), fp32 accumulation
+ *             (bf16 x and w_router with T >= 64 and H % 64 == 0: a tensor-core
+ *             bf16 GEMM, fp32 accumulation; else CUDA-core dot products);
  *             or, when w_router == NULL, l = logits_in [T,E] fp32 (device).
  *   ids[t,:] = the k experts first in the order (l descending, id ascending);
  *             NaN ranks below -inf.

@@ -124,6 +124,7 @@ size_t moe_route_ws_size(int T, int E, int k) {
 int moe_route_topk(const void *x, int x_dtype, const void *w_router, int w_dtype, const float *logits_in,
                    const float *bias, int T, int H, int E, int k, int32_t *topk_ids, float *topk_w,
                    float *logits_out, void *ws, size_t ws_bytes, moe_stream_t s) {
+    moe::NvtxRange nvtx_range("moe_route_topk");
     t_err.clear();
     REQUIRE(T >= 0, "T must be >= 0 (got %d)", T);
     REQUIRE(E >= 1 && E <= 32768, "E must be in [1, 32768] (got %d)", E);
@@ -178,6 +179,7 @@ size_t moe_permute_ws_size(int T, int k, int E) {
 
 int moe_permute(const int32_t *topk_ids, int T, int k, int E, int32_t *expert_offsets, int32_t *perm_src,
                 int32_t *perm_dst, int32_t *active, void *ws, size_t ws_bytes, moe_stream_t s) {
+    moe::NvtxRange nvtx_range("moe_permute");
     t_err.clear();
     REQUIRE(T >= 0, "T must be >= 0 (got %d)", T);
     REQUIRE(E >= 1 && E <= 32768, "E must be in [1, 32768] (got %d)", E);
@@ -218,6 +220,7 @@ static int expert_ffn(int bits, const void *const *expert_blobs, const int32_t *
                       const int32_t *active, const int32_t *perm_src, const void *x, int x_dtype, int T, int k, int H,
                       int I, int E, const void *shared_blob, float *y_perm, float *y_shared, int mode, void *ws,
                       size_t ws_bytes, moe_stream_t s) {
+    moe::NvtxRange nvtx_range("moe_expert_ffn");
     t_err.clear();
     REQUIRE(T >= 0, "T must be >= 0 (got %d)", T);
     REQUIRE(E >= 1 && E <= 32768, "E must be in [1, 32768] (got %d)", E);
@@ -281,6 +284,7 @@ int moe_layer_decode(int bits, const void *x, int x_dtype, const void *w_router,
                      const float *logits_in, const void *const *expert_blobs, const void *shared_blob, int H, int I,
                      int E, int k, int32_t *topk_ids, float *topk_w, float *logits_out, float *y, void *ws,
                      size_t ws_bytes, moe_stream_t s) {
+    moe::NvtxRange nvtx_range("moe_layer_decode");
     t_err.clear();
     REQUIRE(bits == 4 || bits == 2, "bits must be 4 or 2 (got %d)", bits);
     REQUIRE(E >= 1 && k >= 1 && k <= E, "need 1 <= k <= E (got k=%d, E=%d)", k, E);
@@ -309,6 +313,7 @@ int moe_layer_decode(int bits, const void *x, int x_dtype, const void *w_router,
 // ---------------------------------------------------------------- combine
 int moe_combine(const float *y_perm, const int32_t *perm_dst, const float *topk_w, const float *y_shared, int T, int k,
                 int H, float *y, moe_stream_t s) {
+    moe::NvtxRange nvtx_range("moe_combine");
     t_err.clear();
     REQUIRE(T >= 0, "T must be >= 0 (got %d)", T);
     REQUIRE(k >= 1 && k <= 32, "k must be in [1, 32] (got %d)", k);

@@ -1,6 +1,8 @@
 // Shared device/host helpers of libmoe (not shared with the oracle).
 #pragma once
 
+#include <nvtx3/nvToolsExt.h>
+
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -13,9 +15,19 @@ namespace moe {
 // ---------------------------------------------------------------- host side
 void set_error(const char *fmt, ...);
 int cuda_status(cudaError_t e, const char *what);   // MOE_OK or MOE_ECUDA (+ message)
+
 unsigned *device_error_word();                       // this device's error word, or nullptr
 int num_sms();                                       // SMs of the current device (cached)
 void count_launches(int n);                          // adds to the library's launch counter
+
+// Names the enclosing C-ABI call in profiler timelines (NVTX range; a no-op
+// when no tool is attached).
+struct NvtxRange {
+    explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange &) = delete;
+    NvtxRange &operator=(const NvtxRange &) = delete;
+};
 
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 

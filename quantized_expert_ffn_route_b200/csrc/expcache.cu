@@ -163,6 +163,7 @@ int expcache_lookup(moe_expcache *c, const int32_t *ids_host, int n, int32_t *sl
 
 int expcache_stage(moe_expcache *c, const int32_t *ids_host, int n, moe_stream_t compute, int32_t *hit_out,
                    int32_t *slot_out, int32_t *victim_out) {
+    moe::NvtxRange nvtx_range("expcache_stage");
     REQUIRE(c && (n == 0 || ids_host), "cache/ids are NULL");
     REQUIRE(n >= 0 && n <= 32, "n must be in [0, 32]");
     if (n > c->d.capacity) {
@@ -291,6 +292,7 @@ int expcache_join(moe_expcache *c, moe_stream_t s) {
 }
 
 int expcache_wait(moe_expcache *c, int64_t timeout_us) {
+    moe::NvtxRange nvtx_range("expcache_wait");
     REQUIRE(c != nullptr, "cache is NULL");
     const auto t0 = std::chrono::steady_clock::now();
     for (;;) {

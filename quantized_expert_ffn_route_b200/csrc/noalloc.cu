@@ -59,6 +59,7 @@ extern "C" int moe_expert_ffn_noalloc(int bits, const void *const *expert_blobs,
                                       const int32_t *active, const int32_t *perm_src, const void *x, int x_dtype,
                                       int T, int k, int H, int I, int E, const void *shared_blob, float *y_perm,
                                       float *y_shared, moe_stream_t s) {
+    moe::NvtxRange nvtx_range("moe_expert_ffn_noalloc");
     set_error("%s", "");
 #define NA_REQUIRE(cond, ...)      \
     do {                           \

@@ -76,7 +76,10 @@ class MoELayer:
         self.bits, self.H, self.I, self.E, self.k = bits, H, I, E, k
         self.device = torch.device(device)
         nb = moe_expert_blob_bytes(bits, H, I)
-        assert nb > 0 and tuple(blobs.shape) == (E, nb), (blobs.shape, nb)
+        if nb <= 0 or tuple(blobs.shape) != (E, nb):
+            raise ValueError(f"blobs must be uint8 [E={E}, {nb}] for bits={bits}, H={H}, I={I}; got {tuple(blobs.shape)}")
+        if shared is not None and int(np.asarray(shared).size) != nb:
+            raise ValueError(f"shared blob must hold {nb} bytes")
         self.blob_bytes = nb
         self.stride = _round_up(nb, slot_align)
         self.arena = torch.empty(E * self.stride, dtype=torch.uint8, device=self.device)

@@ -107,10 +107,72 @@ class ClockSampler:
 
 
 def src_hash(*names):
+    """Hash of the named kernel sources plus every header they can include
+    (the library's internal headers and the C ABI header), so a change to any
+    of them marks recorded DRAM counters as stale."""
+    csrc = ROOT / "quantized_expert_ffn_route_b200" / "csrc"
+    files = [csrc / n for n in names]
+    files += sorted(p for p in csrc.iterdir() if p.suffix in (".cuh", ".h"))
+    files.append(ROOT / "include" / "moe.h")
     h = hashlib.sha256()
-    for n in names:
-        h.update((ROOT / "quantized_expert_ffn_route_b200" / "csrc" / n).read_bytes())
+    for f in files:
+        h.update(f.name.encode())
+        h.update(f.read_bytes())
     return h.hexdigest()[:16]
+
+
+def fp32_peak_tflops(sm_mhz, sms=148):
+    """FP32 FMA roof derived from unit counts: SMs x 128 FP32 lanes x 2 FLOP
+    per FMA x SM clock."""
+    return sms * 128 * 2 * sm_mhz * 1e6 / 1e12
+
+
+def layer_roofline(kind, fused, H, I, E, k, T, n_act, blob, ms_launch, pk, sm_mhz):
+    """Roofline object of one expert-step launch.  Algorithmic bytes: the
+    distinct expert blobs + x read once + y written once (+ the router rows
+    and logits when the launch also routes); intermediates (x_perm, h, y_perm)
+    are not credited.  Algorithmic FLOPs: 2*3*H*I per (token, expert)
+    assignment including the shared expert (+ 2*H*E per token for a routing
+    launch)."""
+    if fused:
+        nbytes = (k + 1) * blob + E * H * 2 + H * 2 + E * 4 + H * 4
+        flops = 2 * 3 * H * I * (k + 1) + 2 * H * E
+    else:
+        nbytes = (n_act + 1) * blob + T * H * 2 + T * H * 4
+        flops = 2 * 3 * H * I * T * (k + 1)
+    sec = ms_launch / 1e3
+    gbs = nbytes / sec / 1e9
+    hbm = pk["hbm_gbs"]
+    if kind == "prefill":
+        peak_tf = pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+        tf = flops / sec / 1e12
+        if flops / nbytes > peak_tf * 1e12 / (hbm * 1e9):
+            roof = {"bound": "tensor", "achieved": round(tf, 2), "peak": peak_tf, "unit": "TFLOP/s",
+                    "frac": round(tf / peak_tf, 4)}
+        else:
+            roof = {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
+                    "frac": round(gbs / hbm, 4)}
+        roof["fp16_tensor_tflops_achieved"] = round(tf, 2)
+    else:
+        roof = {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
+                "frac": round(gbs / hbm, 4)}
+        if kind == "verify":
+            # the binding roof is the slower of the HBM and the FP32 ALU time
+            alu_peak = fp32_peak_tflops(sm_mhz)
+            tf = flops / sec / 1e12
+            t_hbm, t_alu = nbytes / (hbm * 1e9), flops / (alu_peak * 1e12)
+            roof["hbm_frac"] = round(gbs / hbm, 4)
+            roof["alu_achieved_tflops"] = round(tf, 3)
+            roof["alu_peak_tflops"] = round(alu_peak, 2)
+            roof["alu_frac"] = round(tf / alu_peak, 4)
+            roof["alu_peak_source"] = f"derived: 148 SMs x 128 FP32 lanes x 2 FLOP x {sm_mhz:.0f} MHz"
+            if t_alu > t_hbm:
+                roof.update({"bound": "alu", "achieved": round(tf, 3), "peak": round(alu_peak, 2),
+                             "unit": "TFLOP/s", "frac": round(tf / alu_peak, 4)})
+            roof["binding_roof_time_us"] = round(max(t_hbm, t_alu) * 1e6, 3)
+    roof["algorithmic_bytes_per_launch"] = int(nbytes)
+    roof["algorithmic_flops_per_launch"] = int(flops)
+    return roof
 
 
 def traffic_from_profiles(key: str, sha: str):
@@ -245,11 +307,10 @@ def bench_layer(args, world, rank, pk):
     layer = build_layer(kind)
     H, I, E, k, bits = layer.H, layer.I, layer.E, layer.k, layer.bits
     T = {"decode": 1, "verify": args.window, "prefill": args.chunk}[kind]
-    mode = M.MOE_MODE_GEMM if kind == "prefill" else M.MOE_MODE_AUTO
+    n_layers, mode, fused = workload_shape(kind, args)
     blob = M.moe_expert_blob_bytes(bits, H, I)
     # layer copies at distinct addresses: the steps of one sweep touch far more
     # than the 126 MB L2 (decode: 16 x 908 MB), so weights come from HBM
-    n_layers = args.layers or (2 if kind == "prefill" else 16)
     copies = gpu_copies(layer, n_layers)
     n_steps = args.warmup + args.steps
     seed = W.SEED[kind] + 7919 * rank
@@ -263,7 +324,6 @@ def bench_layer(args, world, rank, pk):
             return xs[j * T:(j + 1) * T]
         return xs[i * T:(i + 1) * T]
 
-    fused = kind == "decode" and not args.unfused
     dbuf = copies[0].decode_buffers() if fused else None
 
     def step(i, e0=None, e1=None):
@@ -345,34 +405,21 @@ def bench_layer(args, world, rank, pk):
     ffn_avg_ms = float(np.mean(ffn_ms))
     assert M.moe_device_error() == 0
 
-    # distinct experts actually touched in the last timed step (all routed + shared)
-    n_act = k if fused else int(bufs.active[0].item())
+    # distinct routed experts per launch: k for one token; for windows the
+    # mean over the windows that routing_stats reads back; for prefill the
+    # last chunk's active count
+    routing = routing_stats(step, bufs, T, k, n_steps) if kind == "verify" else None
+    if fused or kind == "decode":
+        n_act = k
+    elif routing and "distinct_experts_per_step" in routing:
+        n_act = routing["distinct_experts_per_step"]
+    else:
+        n_act = int(bufs.active[0].item())
     tokens_total = sum_over_ranks(args.steps * T, world)
     value = tokens_total / (ms_max / 1e3)
 
-    # algorithmic bytes/FLOPs of one expert-FFN launch
-    if kind == "prefill":
-        flops = 2 * 3 * H * I * T * (k + 1)
-        bytes_ffn = (n_act + 1) * blob + T * H * 2 + T * (k + 1) * H * 4
-        tf = flops / (ffn_avg_ms / 1e3) / 1e12
-        peak_tf = pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
-        gbs = bytes_ffn / (ffn_avg_ms / 1e3) / 1e9
-        if flops / bytes_ffn > peak_tf * 1e12 / (pk["hbm_gbs"] * 1e9):
-            roof = {"bound": "tensor", "achieved": round(tf, 2), "peak": peak_tf, "unit": "TFLOP/s",
-                    "frac": round(tf / peak_tf, 4)}
-        else:
-            roof = {"bound": "hbm", "achieved": round(gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
-                    "frac": round(gbs / pk["hbm_gbs"], 4)}
-    else:
-        # per-window distinct experts differ; average over the timed steps is not tracked on device,
-        # so credit the experts of the last window (decode: always k routed + 1 shared)
-        if fused:   # one kernel: router rows + k routed + shared expert blobs + x + logits + y
-            bytes_ffn = (k + 1) * blob + E * H * 2 + H * 2 + E * 4 + H * 4
-        else:
-            bytes_ffn = (n_act + 1) * blob + T * H * 2 + T * (k + 1) * H * 4
-        gbs = bytes_ffn / (ffn_avg_ms / 1e3) / 1e9
-        roof = {"bound": "hbm", "achieved": round(gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
-                "frac": round(gbs / pk["hbm_gbs"], 4)}
+    sm_mhz = (clk or {}).get("sm_mhz") or 1965.0
+    roof = layer_roofline(kind, fused, H, I, E, k, T, n_act, blob, ffn_avg_ms, pk, sm_mhz)
     sha = src_hash("decode.cu" if fused else ("gemv.cu" if kind != "prefill" else "gemm_tc.cu"))
     roof["traffic"] = traffic_from_profiles("k_decode" if fused else f"expert_ffn_{kind}_{T}", sha)
     roof["kernel"] = ("moe_layer_decode (k_dec_logits -> k_dec_gateup -> k_dec_down, chained by programmatic "
@@ -380,7 +427,6 @@ def bench_layer(args, world, rank, pk):
                       else "moe_expert_ffn (gate/up + down kernels)")
     roof["ms_per_launch"] = round(ffn_avg_ms, 5)
     roof["timing"] = ffn_timing
-    roof["algorithmic_bytes_per_launch"] = int(bytes_ffn)
     roof["peak_source"] = pk["source"]
 
     # end to end through the public API with host buffers
@@ -432,15 +478,9 @@ def bench_layer(args, world, rank, pk):
         cpu = {"value": round(ntok / dt, 3), "unit": "tokens/s", "cores": host_cores(), "kind": "oracle",
                "sample": f"{ntok} tokens of the {kind} workload through the fp64 oracle in batches of 8, {dt:.1f} s"}
 
-    cfg = {"workload": workload_name(kind, H, E, k, I, bits, T),
-           "tokens_per_step": T, "layer_copies": n_layers,
-           "l2": f"inputs larger than L2: {n_layers} layer copies x {E + 1} experts x {blob} B rotate per step",
-           "mode": "fused decode kernel" if fused else {0: "auto", 1: "gemv", 2: "gemm"}[mode],
-           "parallelism": f"replicas x{world}"}
-    if kind == "verify":
-        cfg["routing"] = routing_stats(step, bufs, T, k, n_steps)
+    cfg = layer_config(kind, H, E, k, I, bits, T, n_layers, blob, mode, fused, world)
     return dict(value=value, ms=ms_max, steps=args.steps, roofline=roof, e2e=e2e, cpu=cpu, clocks=clk,
-                launches=launches, config=cfg, dtype="fp32 (CUDA-core FMA on 4-bit codes)" if kind == "decode"
+                launches=launches, config=cfg, routing=routing, dtype="fp32 (CUDA-core FMA on 4-bit codes)" if kind == "decode"
                 else ("fp32 (CUDA-core FMA on 2-bit codes)" if kind == "verify" else "fp16 tensor cores, fp32 accum"))
 
 
@@ -581,11 +621,8 @@ def bench_paging(args, world, rank, pk):
         cpu = {"value": round(n / dt, 3), "unit": "tokens/s", "cores": host_cores(), "kind": "oracle",
                "sample": f"{n} paging steps (1 token, 10 of 24,576 experts) through the fp64 oracle, {dt:.1f} s"}
     cache.close()
-    cfg = {"workload": f"paging: {E} experts (2-bit, {nb} B each, {E * nb / 1e9:.1f} GB pinned host), "
-                       f"{cap} HBM slots, top-{k}, Zipf s={c['zipf_s']} with drift every {c['drift_every']} steps",
-           "tokens_per_step": 1, "cache": {"misses": st1["misses"] - st0["misses"],
-                                           "hits": st1["hits"] - st0["hits"]},
-           "l2": "weights paged from host; HBM slots 2 GB > L2", "parallelism": f"replicas x{world}"}
+    cfg = paging_config(E, k, nb, cap, c, world)
+    roof["cache"] = {"misses": st1["misses"] - st0["misses"], "hits": st1["hits"] - st0["hits"]}
     return dict(value=value, ms=ms, steps=args.steps, roofline=roof, e2e=e2e, cpu=cpu, clocks=clk,
                 launches=launches, config=cfg, dtype="fp32 (CUDA-core FMA on 2-bit codes)")
 
@@ -616,37 +653,81 @@ def routing_stats(step, bufs, T, k, n_steps, n=64):
         return {"error": str(e)[:200]}
 
 
+def layer_config(kind, H, E, k, I, bits, T, n_layers, blob, mode, fused, world):
+    """The `config` object of a resident-layer workload (both arms print it)."""
+    return {"workload": workload_name(kind, H, E, k, I, bits, T),
+            "tokens_per_step": T, "layer_copies": n_layers,
+            "l2": f"inputs larger than L2: {n_layers} layer copies x {E + 1} experts x {blob} B rotate per step",
+            "mode": "fused decode kernel" if fused else {0: "auto", 1: "gemv", 2: "gemm"}[mode],
+            "parallelism": f"replicas x{world}"}
+
+
+def paging_config(E, k, nb, cap, c, world):
+    """The `config` object of the paging workload (both arms print it)."""
+    return {"workload": f"paging: {E} experts (2-bit, {nb} B each, {E * nb / 1e9:.1f} GB pinned host), "
+                        f"{cap} HBM slots, top-{k}, Zipf s={c['zipf_s']} with drift every {c['drift_every']} steps",
+            "tokens_per_step": 1, "l2": "weights paged from host; HBM slots 2 GB > L2",
+            "parallelism": f"replicas x{world}"}
+
+
+def workload_shape(kind, args):
+    """(layer copies, FFN mode, fused) of a resident-layer workload as bench_layer runs it."""
+    n_layers = args.layers or (2 if kind == "prefill" else 16)
+    mode = 2 if kind == "prefill" else 0
+    fused = kind == "decode" and not args.unfused
+    return n_layers, mode, fused
+
+
 def workload_name(kind, H, E, k, I, bits, T):
     return (f"{kind}: hidden {H}, {E} experts + 1 shared, top-{k}, intermediate {I}, "
             f"{bits}-bit blocks of 32 + fp16 scale, {T} token(s)/step")
 
 
 def bench_reference(args, world, rank):
-    """The oracle on the host cores, each step a bounded sample (one token / window)."""
+    """The oracle on the host cores, as it stands; each step is a bounded
+    sample of the workload: one token (decode, verify, prefill) or one paging
+    step, so K steps take about K x 25-50 ms on 16 cores."""
     import oracle
     import workloads as W
     if rank != 0:
         return None
     oracle.set_threads(host_cores())
-    kind = args.workload if args.workload != "paging" else "decode"
-    layer = build_layer(kind)
-    T = {"decode": 1, "verify": args.window, "prefill": 8}[kind]
-    x = W.make_tokens(W.SEED[kind], (args.warmup + args.steps) * T, layer.H, "bf16")
+    kind = args.workload
+    n = args.warmup + args.steps
+    if kind == "paging":
+        c = W.PAGING
+        E, k, H, I, cap = c["E"], c["k"], c["H"], c["I"], c["capacity"]
+        base = W.make_layer(W.SEED["paging"], 2, H, I, 512, k, shared=False, w_dtype="bf16")
+        blob_list = [base.blobs[e % 512] for e in range(E)]     # the pool repeats 512 distinct blobs
+        trace = np.stack(list(W.paging_trace(W.SEED["paging"], E, k, n, s=c["zipf_s"],
+                                             drift_every=c["drift_every"], drift_prob=c["drift_prob"],
+                                             hot=c["hot"])))
+        x = W.make_tokens(W.SEED["paging"] + 1, n, H, "bf16")
 
-    def one(i):
-        oracle.moe_layer(layer.bits, x[i * T:(i + 1) * T], "bf16", layer.blobs, k=layer.k, H=layer.H, I=layer.I,
-                         E=layer.E, w_router=layer.w_router, w_dtype="bf16", bias=layer.bias,
-                         shared_blob=layer.shared)
+        def one(i):
+            oracle.moe_layer(2, x[i:i + 1], "bf16", blob_list, k=k, H=H, I=I, E=E, logits_in=trace[i:i + 1])
+        cfg = paging_config(E, k, oracle.blob_bytes(2, H, I), cap, c, world)
+        sample = "1 paging step (1 token, 10 of 24,576 experts)"
+    else:
+        layer = build_layer(kind)
+        x = W.make_tokens(W.SEED[kind], n, layer.H, "bf16")
+
+        def one(i):
+            oracle.moe_layer(layer.bits, x[i:i + 1], "bf16", layer.blobs, k=layer.k, H=layer.H, I=layer.I,
+                             E=layer.E, w_router=layer.w_router, w_dtype="bf16", bias=layer.bias,
+                             shared_blob=layer.shared)
+        Tw = {"decode": 1, "verify": args.window, "prefill": args.chunk}[kind]
+        n_layers, mode, fused = workload_shape(kind, args)
+        cfg = layer_config(kind, layer.H, layer.E, layer.k, layer.I, layer.bits, Tw, n_layers,
+                           oracle.blob_bytes(layer.bits, layer.H, layer.I), mode, fused, world)
+        sample = f"1 token of the {kind} workload"
     for i in range(args.warmup):
         one(i)
     t0 = time.perf_counter()
-    for i in range(args.warmup, args.warmup + args.steps):
+    for i in range(args.warmup, n):
         one(i)
     dt = time.perf_counter() - t0
-    v = args.steps * T / dt
-    name = workload_name(kind, layer.H, layer.E, layer.k, layer.I, layer.bits,
-                         {"decode": 1, "verify": args.window, "prefill": args.chunk}[kind])
-    return dict(value=v, ms=dt * 1e3, T=T, kind=kind, name=name)
+    return dict(value=args.steps / dt, ms=dt * 1e3, config=cfg, sample=sample)
 
 
 def main():
@@ -679,10 +760,10 @@ def main():
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(r["ms"] / args.steps, 3),
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
                 "data": "synthetic (seeded)", "impl": "reference",
-                "config": {"workload": r["name"], "tokens_per_step": r["T"], "parallelism": "replicas x1"},
+                "config": r["config"],
                 "cpu_baseline": {"value": round(r["value"], 4), "unit": "tokens/s", "cores": host_cores(),
                                  "kind": "oracle",
-                                 "sample": f"{args.steps} steps of {r['T']} token(s) of that workload"},
+                                 "sample": f"{args.steps} steps, each {r['sample']}"},
                 "e2e": {"value": round(r["value"], 4), "unit": "tokens/s", "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}}
         print(json.dumps(line), flush=True)
@@ -701,6 +782,8 @@ def main():
                 "data": "synthetic (seeded generators; no weights or datasets)", "config": r["config"],
                 "roofline": r["roofline"], "cpu_baseline": r["cpu"], "e2e": r["e2e"],
                 "gpu_launches": int(r["launches"]), "clocks": r["clocks"]}
+        if r.get("routing"):
+            line["routing"] = r["routing"]
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist

@@ -204,16 +204,17 @@ int moe_layer_decode(int bits, const void *x, int x_dtype, const void *w_router,
 
 /* ------------------------------------------------- allocation-free FFN
  * The pages have no counterpart of this call; it serves callers that cannot
- * allocate device memory when they run the step: code running while a
- * stream is captured into a CUDA graph (an allocation there breaks the
- * capture), engines held to a memory budget fixed at start-up, and C hosts
- * with no device allocator to hand out a workspace.
+ * allocate device memory when they run the step: engines held to a device
+ * memory budget fixed at start-up, C hosts with no device allocator to hand
+ * out a workspace, and latency-critical loops where an allocation could
+ * synchronise the device.
  * Same computation and arguments as moe_expert_ffn_q4/q2 in MOE_MODE_GEMV
  * (bits = 4 or 2 selects the blob format), but without ws/ws_bytes: the
  * scratch (the fp32 intermediate h, T*(k+1)*I*4 bytes) comes from one array
  * built into the library of moe_expert_ffn_noalloc_max_bytes() bytes (8 MiB),
  * which every GPU that loads the library holds until the process exits.
- *  - Calls needing more scratch than that, H/I outside [128, 2048], or an I
+ *  - Calls whose scratch, T*(k+1)*I*4 bytes, exceeds that size, H/I outside
+ *    [128, 2048], or an I
  *    that GEMV mode does not take (see above), are rejected with MOE_EINVAL
  *    before anything is launched.
  *  - It never calls cudaMalloc, cudaFree or any allocating routine.

@@ -50,6 +50,7 @@ def lib():
         _lib.oracle_blob_bytes.argtypes = [I32, I32, I32]
         _lib.oracle_expert_weights.argtypes = [I32, I32, I32, P, P, P, P]
         _lib.oracle_expert_ffn.argtypes = [I32, I32, I32, P, P, P, P]
+        _lib.oracle_expert_ffn_rows.argtypes = [I32, I32, I32, I32, P, P, P]
         _lib.oracle_router_logits.argtypes = [I32, I32, I32, P, I32, P, I32, P, P]
         _lib.oracle_topk.restype = I32
         _lib.oracle_topk.argtypes = [I32, I32, I32, P, P, P]
@@ -114,6 +115,19 @@ def expert_ffn(bits: int, H: int, I: int, blob: np.ndarray, x: np.ndarray):
     y = np.empty(H); h = np.empty(I)
     lib().oracle_expert_ffn(bits, H, I, _p(blob), _p(x), _p(y), _p(h))
     return y, h
+
+
+def expert_ffn_rows(bits: int, H: int, I: int, blobs, xs):
+    """Many independent (expert blob, token) pairs: y [n, H], row i = the FFN
+    of blobs[i] applied to xs[i] (fp64 rows)."""
+    blob_list = [np.ascontiguousarray(b, dtype=np.uint8) for b in blobs]
+    xs = _c(xs, np.float64)
+    n = len(blob_list)
+    assert xs.shape == (n, H)
+    ptrs = (C.c_void_p * max(1, n))(*[b.ctypes.data for b in blob_list])
+    y = np.empty((n, H))
+    lib().oracle_expert_ffn_rows(bits, H, I, n, C.cast(ptrs, C.c_void_p), _p(xs), _p(y))
+    return y
 
 
 # ------------------------------------------------------------------- router

@@ -182,6 +182,18 @@ void oracle_expert_ffn(int bits, int H, int I, const uint8_t *blob,
     free(h);
 }
 
+/* n independent (expert, token) pairs: y[i] = FFN of blobs[i] applied to
+ * x[i] (both [H] rows), one call of oracle_expert_ffn each, rows in
+ * parallel.  Used to check chosen rows of a large step without running the
+ * whole step. */
+void oracle_expert_ffn_rows(int bits, int H, int I, int n, const uint8_t *const *blobs,
+                            const double *x, double *y)
+{
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long i = 0; i < (long)n; ++i)
+        oracle_expert_ffn(bits, H, I, blobs[i], x + (size_t)i * H, y + (size_t)i * H, NULL);
+}
+
 /* -------------------------------------------------------------- router */
 
 void oracle_router_logits(int T, int H, int E, const void *x, int x_dtype,

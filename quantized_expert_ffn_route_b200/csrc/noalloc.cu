@@ -1,11 +1,10 @@
 // Allocation-free variant of the expert FFN (CUDA-core GEMV kernels).
 //
 // Some callers cannot allocate device memory at the point where they run the
-// expert step: code that runs while a stream is being captured into a CUDA
-// graph (allocation is not a stream operation and breaks the capture),
-// engines that must stay inside a memory budget fixed at start-up, and plain
-// C hosts that have no device allocator of their own to hand out a
-// workspace.  For them, this entry point takes its scratch (the SwiGLU
+// expert step: engines that must stay inside a device-memory budget fixed at
+// start-up, plain C hosts that have no device allocator of their own to hand
+// out a workspace, and latency-critical loops where an allocation could
+// synchronise the device.  For them, this entry point takes its scratch (the SwiGLU
 // intermediate h, fp32) from a fixed array compiled into the library instead
 // of a caller-provided workspace.
 //

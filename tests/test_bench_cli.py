@@ -45,3 +45,69 @@ def test_expert_stats():
     assert st["distinct_experts_per_step"] == 3.0          # {0,1,2} and {3,4,5}
     assert st["top2_share"] == 0.5                         # experts 1 and 3 take 4 of 8 selections
     assert st["steps"] == 2
+
+
+def _pk():
+    return {"hbm_gbs": 6557.4, "bf16_tflops": 1667.0, "source": "measured"}
+
+
+def test_roofline_bytes_exclude_intermediates():
+    """Algorithmic bytes: distinct blobs + x once + y once; y_perm, h and
+    x_perm are not credited.  FLOPs: 2*3*H*I per assignment incl. the shared expert."""
+    import bench
+    H, I, E, k, T, blob = 2048, 512, 512, 10, 8192, 1769472
+    r = bench.layer_roofline("prefill", False, H, I, E, k, T, 512, blob, 2.0, _pk(), 1965.0)
+    assert r["algorithmic_bytes_per_launch"] == 513 * blob + T * H * 2 + T * H * 4
+    assert r["algorithmic_flops_per_launch"] == 2 * 3 * H * I * T * (k + 1)
+    assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
+    r = bench.layer_roofline("prefill", False, H, I, E, k, 512, 512, blob, 0.2, _pk(), 1965.0)
+    assert r["bound"] == "hbm" and r["algorithmic_bytes_per_launch"] == 513 * blob + 512 * H * 6
+    # fused decode: 11 blobs + router rows + x + logits + y
+    r = bench.layer_roofline("decode", True, H, I, E, k, 1, k, blob, 0.01, _pk(), 1965.0)
+    assert r["algorithmic_bytes_per_launch"] == 11 * blob + E * H * 2 + H * 2 + E * 4 + H * 4
+
+
+def test_verify_roofline_names_the_binding_roof():
+    """Verify windows: max(HBM, FP32 ALU) with both fractions reported."""
+    import bench
+    H, I, k, blob = 2048, 512, 10, 983040
+    alu = bench.fp32_peak_tflops(1965.0)
+    assert abs(alu - 148 * 128 * 2 * 1.965e9 / 1e12) < 1e-9
+    # 16 tokens over 40 distinct experts: FLOPs 16 x 69.2 M vs 41 blobs
+    r = bench.layer_roofline("verify", False, H, I, 512, k, 16, 40, blob, 0.1, _pk(), 1965.0)
+    t_hbm = r["algorithmic_bytes_per_launch"] / (6557.4e9)
+    t_alu = r["algorithmic_flops_per_launch"] / (alu * 1e12)
+    assert r["bound"] == ("alu" if t_alu > t_hbm else "hbm")
+    assert "hbm_frac" in r and "alu_frac" in r
+    assert abs(r["binding_roof_time_us"] - max(t_hbm, t_alu) * 1e6) < 1e-2
+    # a window of 2 over 20 experts is HBM-bound
+    r = bench.layer_roofline("verify", False, H, I, 512, k, 2, 20, blob, 0.03, _pk(), 1965.0)
+    assert r["bound"] == "hbm"
+
+
+def test_both_arms_print_the_same_config():
+    import argparse
+    import bench
+    args = argparse.Namespace(layers=0, unfused=False)
+    for kind, T in (("decode", 1), ("verify", 16), ("prefill", 8192)):
+        n_layers, mode, fused = bench.workload_shape(kind, args)
+        bits = 2 if kind == "verify" else 4
+        blob = 983040 if bits == 2 else 1769472
+        a = bench.layer_config(kind, 2048, 512, 10, 512, bits, T, n_layers, blob, mode, fused, 1)
+        assert a["workload"].startswith(f"{kind}: hidden 2048, 512 experts + 1 shared, top-10")
+        assert a["layer_copies"] == (2 if kind == "prefill" else 16)
+
+
+def test_src_hash_covers_headers(tmp_path, monkeypatch):
+    """An edit to any internal header changes every kernel's source hash."""
+    import shutil
+    import bench
+    root = tmp_path
+    shutil.copytree(ROOT / "quantized_expert_ffn_route_b200" / "csrc", root / "quantized_expert_ffn_route_b200" / "csrc")
+    (root / "include").mkdir()
+    shutil.copy(ROOT / "include" / "moe.h", root / "include" / "moe.h")
+    monkeypatch.setattr(bench, "ROOT", root)
+    h0 = bench.src_hash("decode.cu")
+    p = root / "quantized_expert_ffn_route_b200" / "csrc" / "qdot.cuh"
+    p.write_text(p.read_text() + "\n// edit\n")
+    assert bench.src_hash("decode.cu") != h0

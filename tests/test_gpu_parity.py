@@ -162,12 +162,24 @@ def test_combine_against_oracle():
 
 
 # ------------------------------------------------------------ whole layer
+def _check_undecided(gpu_logits, gpu_ids, k):
+    """Tokens whose routing margin is within the logit error bound: their ids
+    must be the top-k of the GPU's own fp32 logits (same precision on both
+    sides)."""
+    if gpu_ids.shape[0] == 0:
+        return
+    ids_ref, _, _ = oracle.topk(np.ascontiguousarray(gpu_logits, np.float32), k)
+    assert np.array_equal(gpu_ids, ids_ref)
+
+
 def _check_layer(out, ref, layer, x, x_dtype, tol=TOL):
-    """ids/permutation bit-exact where the routing margin is decisive; y within tol."""
+    """ids/permutation bit-exact where the routing margin is decisive (the
+    rest: the top-k of the GPU's own logits); y within tol."""
     eps = logit_bound(layer, x, x_dtype) if layer.w_router is not None else np.zeros_like(ref["logits"])
     dec = decisive_tokens(ref["logits"], eps, layer.k)
     assert out["err"] == 0
     assert np.array_equal(out["ids"][dec], ref["ids"][dec])
+    _check_undecided(out["logits"][~dec], out["ids"][~dec], layer.k)
     if dec.all():
         assert np.array_equal(out["offsets"], ref["offsets"])
         assert np.array_equal(out["perm_src"], ref["perm_src"])
@@ -246,13 +258,50 @@ def test_decode_full_size(decode_layer, T):
     assert e < GEMV_TOL
 
 
-@pytest.mark.parametrize("T", [512, 2048])
+def _tile_edge_rows(n, tiles=(64, 256)):
+    """Local row positions that start or end a token tile of either size, plus the last row."""
+    pos = {0, n - 1}
+    for t in tiles:
+        for b in range(t, n, t):
+            pos.update((b - 1, b))
+    return sorted(p for p in pos if 0 <= p < n)
+
+
+def _check_expert_rows(out, layer, x, tol=TOL):
+    """y_perm rows at the first and last row of every active expert and at
+    every token-tile edge, and y_shared at the shared expert's tile edges,
+    each against the oracle's FFN of that expert on that token.  Covers every
+    expert group and every tile tail of the grouped GEMM."""
+    T, H, I = x.shape[0], layer.H, layer.I
+    offs, ps = out["offsets"], out["perm_src"]
+    xs = xd(x, "bf16")
+    rows, blobs = [], []
+    for e in range(layer.E):
+        r0, r1 = int(offs[e]), int(offs[e + 1])
+        for p in (_tile_edge_rows(r1 - r0) if r1 > r0 else []):
+            rows.append(r0 + p)
+            blobs.append(layer.blobs[e])
+    ref = oracle.expert_ffn_rows(layer.bits, H, I, blobs, xs[ps[rows]])
+    got = out["y_perm"][rows]
+    assert rel_err(got, ref) <= tol, f"y_perm rows: {rel_err(got, ref):.3e} x RMS over {len(rows)} rows"
+    if layer.shared is not None:
+        toks = _tile_edge_rows(T)
+        ref_s = oracle.expert_ffn_rows(layer.bits, H, I, [layer.shared] * len(toks), xs[toks])
+        assert rel_err(out["y_shared"][toks], ref_s) <= tol
+    return len(rows)
+
+
+@pytest.mark.parametrize("T", [512, 2048, 8192])
 def test_prefill_full_size_sampled(decode_layer, T):
-    """Prefill chunk in GEMM mode at full layer size; oracle on sampled tokens."""
+    """Prefill chunk in GEMM mode (the launch configuration the benchmark
+    times) at full layer size: every expert's edge rows against the oracle,
+    the combined output on sampled tokens, and the routing of every token."""
     layer, g = decode_layer
     x = W.make_tokens(W.SEED["prefill"] + T, T, layer.H, "bf16")
-    out = run_gpu(g, x, "bf16", mode=M.MOE_MODE_AUTO)
+    out = run_gpu(g, x, "bf16", mode=M.MOE_MODE_GEMM)
     assert out["err"] == 0
+    n_rows = _check_expert_rows(out, layer, x)
+    assert n_rows >= 2 * int(out["active"][0]) - 1
     rows = np.unique(np.concatenate([[0, T - 1], np.random.default_rng(T).choice(T, 6, replace=False)]))
     ref = _sampled_ref(layer, x, rows)
     eps = logit_bound(layer, x[rows], "bf16")
@@ -260,9 +309,38 @@ def test_prefill_full_size_sampled(decode_layer, T):
     assert np.array_equal(out["ids"][rows][dec], ref["ids"][dec])
     e = rel_err(out["y"][rows][dec], ref["y"][dec])
     assert e <= TOL, e
+    # every token: the ids are the top-k of the GPU's own fp32 logits, and
+    # the logits are within the fp32 error bound of the exact ones
+    _check_undecided(out["logits"], out["ids"], layer.k)
+    ref_l = oracle.router_logits(x[rows], "bf16", layer.w_router, "bf16", layer.bias)
+    assert np.all(np.abs(out["logits"][rows] - ref_l) <= eps)
     # whole-chunk invariants: every row of the permutation is used once
     assert sorted(out["perm_dst"].ravel().tolist()) == list(range(T * layer.k))
     assert out["offsets"][-1] == T * layer.k
+    assert np.array_equal(out["offsets"], oracle.permute(out["ids"], layer.E)["offsets"])
+
+
+@pytest.mark.parametrize("bits", [4, 2])
+def test_gemm_many_tiles_per_cta(bits):
+    """A shape whose 256-token tiles number several per CTA in both GEMMs
+    (gate/up: 8 experts x 16 token tiles x 4 row tiles + the shared expert's
+    128 = 640 tiles; down: 320), so each CTA reuses its TMEM accumulator
+    across tiles."""
+    H, I, E, k, T = 512, 512, 8, 4, 8192
+    layer = W.make_layer(90 + bits, bits, H, I, E, k, shared=True, w_dtype="bf16")
+    x = W.make_tokens(91 + bits, T, H, "bf16")
+    out = run_gpu(_layer_gpu(layer), x, "bf16", mode=M.MOE_MODE_GEMM)
+    assert out["err"] == 0
+    counts = np.diff(out["offsets"])
+    assert counts.min() > 256 * 2                     # several 256-token tiles per expert
+    _check_expert_rows(out, layer, x)
+    rows = np.unique(np.concatenate([[0, 255, 256, T - 1], np.random.default_rng(bits).choice(T, 8, replace=False)]))
+    ref = _sampled_ref(layer, x, rows)
+    eps = logit_bound(layer, x[rows], "bf16")
+    dec = decisive_tokens(ref["logits"], eps, k)
+    assert np.array_equal(out["ids"][rows][dec], ref["ids"][dec])
+    assert rel_err(out["y"][rows][dec], ref["y"][dec]) <= TOL
+    _check_undecided(out["logits"], out["ids"], k)
 
 
 @pytest.fixture(scope="module")

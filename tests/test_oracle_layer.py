@@ -197,3 +197,21 @@ def test_combine_matches_layer(oracle_lib):
             r = out["perm_dst"][t, j]
             ye, _ = oracle_lib.expert_ffn(4, layer.H, layer.I, layer.blobs[out["ids"][t, j]], x[t].astype(np.float64))
             assert np.array_equal(out["y_perm"][r], ye)
+
+
+@pytest.mark.parametrize("bits", [4, 2])
+def test_ffn_rows_is_the_single_row_ffn(oracle_lib, bits):
+    """The batched row helper is a parallel map of the pinned one-token FFN:
+    each of its rows equals that function's result bit for bit, whichever
+    expert and token it pairs (including repeated experts and a reversed order)."""
+    rng = np.random.default_rng(11 + bits)
+    H, I = 128, 64
+    blobs = [W.random_expert_blob(rng, bits, H, I, 0.02) for _ in range(3)]
+    xs = rng.standard_normal((7, H))
+    pick = [0, 2, 1, 1, 0, 2, 0]
+    got = oracle_lib.expert_ffn_rows(bits, H, I, [blobs[e] for e in pick], xs)
+    for i, e in enumerate(pick):
+        y, _ = oracle_lib.expert_ffn(bits, H, I, blobs[e], xs[i])
+        assert np.array_equal(got[i], y)
+    rev = oracle_lib.expert_ffn_rows(bits, H, I, [blobs[e] for e in pick[::-1]], xs[::-1])
+    assert np.array_equal(rev[::-1], got)

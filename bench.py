@@ -306,6 +306,9 @@ def bench_layer(args, world, rank, pk):
     kind = args.workload
     layer = build_layer(kind)
     H, I, E, k, bits = layer.H, layer.I, layer.E, layer.k, layer.bits
+    one_kernel = getattr(args, "decode_one_kernel", False)
+    if one_kernel:
+        M.moe_test_hook(M.MOE_HOOK_DECODE_ONE_KERNEL, 1)
     T = {"decode": 1, "verify": args.window, "prefill": args.chunk}[kind]
     n_layers, mode, fused = workload_shape(kind, args)
     blob = M.moe_expert_blob_bytes(bits, H, I)
@@ -364,7 +367,10 @@ def bench_layer(args, world, rank, pk):
     torch.cuda.synchronize()
     assert M.moe_device_error() == 0
     n0 = M.moe_kernel_launches()
-    graph, pairs = run_graph_steps(step, args.warmup, args.steps)
+    # the timed graph holds the K steps and nothing else: an event recorded
+    # inside a graph costs a few microseconds per node, which would be timed
+    # as part of the step
+    graph, _ = run_graph_steps(step, args.warmup, args.steps, time_ffn=False)
     launches = M.moe_kernel_launches() - n0
     graph.replay()                                     # first replay uploads the graph
     torch.cuda.synchronize()
@@ -385,12 +391,15 @@ def bench_layer(args, world, rank, pk):
     clk = clocks.stop()
     ms = ev0.elapsed_time(ev1)
     ms_max = max_over_ranks(ms, world)
-    try:
-        ffn_ms = [a.elapsed_time(b) for a, b in pairs]
-        ffn_timing = "event pairs recorded around every expert-FFN call inside the timed graph"
-    except Exception:
-        # events recorded inside the graph are not timeable here: time a graph of
-        # the same K FFN calls alone, bracketed by one event pair
+    if fused:
+        # the step is the one call: its average duration is the timed region
+        # over K (conservative: the gaps between calls are included)
+        ffn_ms = [ms / args.steps]
+        ffn_timing = ("timed region / K: the timed graph is K moe_layer_decode calls and nothing else, bracketed by "
+                      "one event pair on the launching stream")
+    else:
+        # a graph of the same K expert-FFN calls alone (same inputs and
+        # buffers as the timed steps), bracketed by one event pair
         torch.cuda.synchronize()
         g2, _ = run_graph_steps(lambda i, e0, e1: ffn_only(i), args.warmup, args.steps, time_ffn=False)
         g2.replay()
@@ -401,7 +410,8 @@ def bench_layer(args, world, rank, pk):
         z.record()
         torch.cuda.synchronize()
         ffn_ms = [a.elapsed_time(z) / args.steps]
-        ffn_timing = "graph of the K expert-FFN calls alone, one event pair / K"
+        ffn_timing = ("graph of the K expert-FFN calls alone (the timed steps' inputs and routing), one event pair "
+                      "on the launching stream / K")
     ffn_avg_ms = float(np.mean(ffn_ms))
     assert M.moe_device_error() == 0
 
@@ -420,11 +430,15 @@ def bench_layer(args, world, rank, pk):
 
     sm_mhz = (clk or {}).get("sm_mhz") or 1965.0
     roof = layer_roofline(kind, fused, H, I, E, k, T, n_act, blob, ffn_avg_ms, pk, sm_mhz)
-    sha = src_hash("decode.cu" if fused else ("gemv.cu" if kind != "prefill" else "gemm_tc.cu"))
+    sha = src_hash(*(("decode.cu", "decode_step.cu") if fused else (("gemv.cu",) if kind != "prefill" else ("gemm_tc.cu",))))
     roof["traffic"] = traffic_from_profiles("k_decode" if fused else f"expert_ffn_{kind}_{T}", sha)
-    roof["kernel"] = ("moe_layer_decode (k_dec_logits -> k_dec_gateup -> k_dec_down, chained by programmatic "
-                      "dependent launch; one call)" if fused
-                      else "moe_expert_ffn (gate/up + down kernels)")
+    if fused and one_kernel:
+        roof["kernel"] = "moe_layer_decode (k_dec_step: one persistent kernel, one CTA per SM, two grid barriers)"
+    elif fused:
+        roof["kernel"] = ("moe_layer_decode (k_dec_logits -> k_dec_gateup -> k_dec_down, chained by programmatic "
+                          "dependent launch; one call)")
+    else:
+        roof["kernel"] = "moe_expert_ffn (gate/up + down kernels)"
     roof["ms_per_launch"] = round(ffn_avg_ms, 5)
     roof["timing"] = ffn_timing
     roof["peak_source"] = pk["source"]
@@ -539,20 +553,62 @@ def bench_paging(args, world, rank, pk):
     xs = torch.from_numpy(x_host.view(np.int16)).view(torch.bfloat16).cuda()
     b = M.alloc_step_buffers(1, H, I, E, k, 2, M.MOE_MODE_GEMV, torch.device("cuda"), False)
     ids_h = torch.empty(k, dtype=torch.int32).pin_memory()
+    # expert lists of the two FFN calls of a step: [count, ids...] for the
+    # hits (resident: computed at once) and for the misses (after their copies)
+    act_h = torch.zeros(64, dtype=torch.int32).pin_memory()
+    act_d = torch.zeros(64, dtype=torch.int32, device="cuda")
     s = torch.cuda.current_stream()
     misses_per_step = []
+    ev_hit = [None, None]
 
     def step(i, x=None):
         M.moe_route_topk(None, 0, None, 0, logits[i], None, 1, H, E, k, b.ids, b.w)
         M.moe_permute(b.ids, 1, k, E, b.offsets, b.perm_src, b.perm_dst, b.active, b.ws_perm, b.sizes["perm"])
         ids_h.copy_(b.ids[:k], non_blocking=True)
         s.synchronize()                                  # the ids cross to the host
-        hit, _, _ = cache.stage(ids_h.numpy())
-        misses_per_step.append(int(k - hit.sum()))
-        cache.join()                                     # compute waits for copies + table patch
-        M.moe_expert_ffn_q2(table, b.offsets, b.active, b.perm_src, xs[i] if x is None else x, M.MOE_BF16, 1, k,
-                            H, I, E, None, b.y_perm, None, M.MOE_MODE_GEMV, b.ws_ffn, b.sizes["ffn"])
+        ids = ids_h.numpy().copy()
+        hit, _, _ = cache.stage(ids)
+        hits, miss = np.sort(ids[hit == 1]), np.sort(ids[hit == 0])
+        misses_per_step.append(int(miss.size))
+        a = act_h.numpy()
+        a[0], a[1:1 + hits.size] = hits.size, hits
+        a[32], a[33:33 + miss.size] = miss.size, miss
+        act_d.copy_(act_h, non_blocking=True)
+        xi = xs[i] if x is None else x
+        ffn = M.moe_expert_ffn_q2
+        if ev_hit[0] is not None:
+            ev_hit[0].record()
+        if hits.size:                                    # resident experts: at once, overlapping the copies
+            ffn(table, b.offsets, act_d[0:], b.perm_src, xi, M.MOE_BF16, 1, k, H, I, E, None, b.y_perm, None,
+                M.MOE_MODE_GEMV, b.ws_ffn, b.sizes["ffn"])
+        if ev_hit[1] is not None:
+            ev_hit[1].record()
+        cache.join()                                     # the rest waits for its copies + table patch
+        if miss.size:
+            ffn(table, b.offsets, act_d[32:], b.perm_src, xi, M.MOE_BF16, 1, k, H, I, E, None, b.y_perm, None,
+                M.MOE_MODE_GEMV, b.ws_ffn, b.sizes["ffn"])
         M.moe_combine(b.y_perm, b.perm_dst, b.w, None, 1, k, H, b.y)
+
+    def overlap_pass(first, n):
+        """Untimed pass over n more steps: the share of each step's copy time
+        (first copy issued -> table patched) during which the hit experts'
+        FFN ran on the compute stream."""
+        ref = torch.cuda.Event(enable_timing=True)
+        ev_hit[0], ev_hit[1] = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ref.record()
+        copy_ms = hidden_ms = 0.0
+        for i in range(first, first + n):
+            m0 = len(misses_per_step)
+            step(i)
+            torch.cuda.synchronize()
+            if misses_per_step[m0] == 0:
+                continue
+            c0, c1 = cache.copy_times(ref)
+            h0, h1 = ref.elapsed_time(ev_hit[0]), ref.elapsed_time(ev_hit[1])
+            copy_ms += c1 - c0
+            hidden_ms += max(0.0, min(c1, h1) - max(c0, h0))
+        ev_hit[0] = ev_hit[1] = None
+        return (hidden_ms / copy_ms if copy_ms > 0 else None), copy_ms
 
     for i in range(args.warmup):
         step(i)
@@ -573,10 +629,11 @@ def bench_paging(args, world, rank, pk):
     assert M.moe_device_error() == 0
     ms = max_over_ranks(a.elapsed_time(z), world)
     st1 = cache.stats()
+    mps = misses_per_step[args.warmup:n_steps]
+    overlap, copy_ms = overlap_pass(n_steps, min(200, 64))
     staged = st1["bytes_staged"] - st0["bytes_staged"]
     value = sum_over_ranks(args.steps, world) / (ms / 1e3)
     link_ach = staged / (ms / 1e3) / 1e9
-    mps = misses_per_step[args.warmup:]
     steady = mps[500:] if len(mps) > 600 else mps
     roof = {"bound": "host_link", "achieved": round(link_ach, 2), "peak": round(link, 2), "unit": "GB/s",
             "frac": round(link_ach / link, 4), "traffic": None,
@@ -584,7 +641,11 @@ def bench_paging(args, world, rank, pk):
             "peak_source": "pinned 1 GiB host->device copy measured in this run",
             "misses_per_step": round(float(np.mean(mps)), 3),
             "misses_per_step_steady": round(float(np.mean(steady)), 3),
-            "hbm_bytes_per_step": k * nb}
+            "hbm_bytes_per_step": k * nb,
+            "overlap": None if overlap is None else round(overlap, 4),
+            "overlap_definition": ("share of each step's copy interval (first copy issued -> device table "
+                                   "patched) during which the resident experts' FFN ran on the compute stream, "
+                                   "from CUDA events over an untimed pass of 64 further steps")}
 
     e2e = None
     if not args.no_e2e:
@@ -744,6 +805,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--unfused", action="store_true", help="decode through the four separate calls")
+    ap.add_argument("--decode-one-kernel", action="store_true",
+                    help="fused decode through the one-kernel persistent step instead of the three-kernel chain")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:

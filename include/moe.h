@@ -78,6 +78,7 @@ typedef struct CUstream_st *moe_stream_t;   /* same type as cudaStream_t */
 #define MOE_DEVERR_NONFINITE 4u      /* a selected logit was NaN or +inf */
 #define MOE_DEVERR_BAD_ROW 8u        /* offsets/perm_src inconsistent */
 #define MOE_DEVERR_TIMEOUT 16u       /* a bounded in-kernel wait ran out */
+#define MOE_DEVERR_MISALIGNED 32u    /* an expert blob pointer was not 16-byte aligned */
 
 /* Thread-local message of the last failing call ("" if none). */
 const char *moe_last_error(void);
@@ -93,6 +94,28 @@ uint64_t moe_kernel_launches(void);
  * `clear` != 0.  *bits_out receives MOE_DEVERR_* bits.  Returns MOE_OK, or
  * MOE_EDEVICE if any bit was set, or MOE_ECUDA. */
 int moe_device_error(uint32_t *bits_out, int clear, moe_stream_t s);
+
+/* Test hooks: settings that only tests change, to drive bounded in-kernel
+ * waits into their timeout path without a GPU fault.  Process-wide; read
+ * when a call launches its kernels; 0 restores the default.  Returns
+ * MOE_EINVAL for an unknown hook or a negative value.
+ *  MOE_HOOK_WAIT_LIMIT_NS         time limit of the fused decode kernel's
+ *                                 waits (grid barriers, copies); default 1 s.
+ *  MOE_HOOK_DECODE_EXTRA_ARRIVALS arrivals the fused decode kernel's grid
+ *                                 barriers wait for beyond its own CTAs, so
+ *                                 a value > 0 makes every barrier time out.
+ *  MOE_HOOK_GEMM_SPIN             polls before a grouped-GEMM mbarrier wait
+ *                                 gives up; default 4,194,304 (about a
+ *                                 second).
+ *  MOE_HOOK_DECODE_ONE_KERNEL     1: moe_layer_decode runs the one-kernel
+ *                                 persistent step where it applies instead
+ *                                 of the three-kernel chain (to test and
+ *                                 time both). */
+#define MOE_HOOK_WAIT_LIMIT_NS 1
+#define MOE_HOOK_DECODE_EXTRA_ARRIVALS 2
+#define MOE_HOOK_GEMM_SPIN 3
+#define MOE_HOOK_DECODE_ONE_KERNEL 4
+int moe_test_hook(int which, int64_t value);
 
 /* Bytes of one expert blob (see layout above). */
 size_t moe_expert_blob_bytes(int bits, int H, int I);
@@ -180,16 +203,24 @@ int moe_expert_ffn_q2(const void *const *expert_blobs, const int32_t *expert_off
  * with the same definitions as moe_route_topk -> moe_permute ->
  * moe_expert_ffn_q4/q2 (GEMV mode) -> moe_combine (Strata article, section 2
  * item 2: only the experts the router picks are computed; at one token the
- * step is bound by streaming those experts' weights).  Three kernels chained
- * with programmatic dependent launch (logits over E/4 CTAs; gate/up, whose
- * routed CTAs each select the top-k; down + combine); no in-kernel waits
- * spin.
+ * step is bound by streaming those experts' weights).
+ * When H and I are multiples of 256, H <= 2048, I / (32 for 4-bit, 64 for
+ * 2-bit) is 4, 8, 16 or 32 and the per-SM share of the weights fits in shared
+ * memory, the step is ONE persistent kernel (one CTA per SM, launched
+ * cooperatively so all CTAs are resident) with two grid-wide barriers kept in
+ * the workspace; each CTA copies its share of every selected expert with the
+ * bulk-copy engine as soon as the ids are known.  Other supported shapes run
+ * three kernels chained with programmatic dependent launch.
  *  x [H] (x_dtype), w_router [E,H] (w_dtype) or NULL with logits_in [E];
- *  expert_blobs device [E] blob pointers; shared_blob or NULL;
- *  topk_ids [k] int32 out, topk_w [k] fp32 out, logits_out [E] or NULL
+ *  expert_blobs device [E] blob pointers (16-byte aligned; a misaligned one
+ *  sets MOE_DEVERR_MISALIGNED and that expert is left out); shared_blob or
+ *  NULL; topk_ids [k] int32 out, topk_w [k] fp32 out, logits_out [E] or NULL
  *  (written only when the logits are computed here), y [H] fp32 out.
- *  ws: moe_layer_decode_ws_size() bytes of scratch (no initialisation
- *  needed).  Calls sharing one ws must not overlap.
+ *  ws: moe_layer_decode_ws_size() bytes of scratch.  It must be zero-filled
+ *  before its first use (cudaMemsetAsync once); every call leaves it ready
+ *  for the next.  After a call that set MOE_DEVERR_TIMEOUT (a grid barrier or
+ *  copy wait ran out, after 1 s) zero it again.  Calls sharing one ws must
+ *  not overlap.
  * Supported shapes (else MOE_EINVAL: use the separate calls): E <= 1024,
  * k <= 32, H <= 2048 and a multiple of 128, I a multiple of 128 with I/32
  * (4-bit) or I/64 (2-bit) in {4, 8, 16, 32}, and the down kernel's tasks,
@@ -306,6 +337,14 @@ int expcache_stats(moe_expcache *c, moe_expcache_stats *out);
 
 /* Host copy of the per-expert counters and slots (n_experts entries each; either may be NULL). */
 int expcache_snapshot(moe_expcache *c, int64_t *counts_out, int32_t *slot_of_out);
+
+/* Timing of the most recent step that staged copies: milliseconds from
+ * `ref_event` (a cudaEvent_t the caller recorded with timing enabled, on the
+ * cache's device) to the start of that step's first copy (*start_ms) and to
+ * the end of its table update (*end_ms).  Both events must have completed
+ * (synchronize first): MOE_ECUDA otherwise.  MOE_EINVAL before any step has
+ * staged a copy.  Used to measure how much copy time compute hides. */
+int expcache_copy_times(moe_expcache *c, const void *ref_event, float *start_ms, float *end_ms);
 
 /* Test hook: the next `n` copies report failure before being issued (MOE_EIO). */
 int expcache_inject_copy_failures(moe_expcache *c, int n);

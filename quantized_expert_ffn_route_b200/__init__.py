@@ -24,6 +24,8 @@ MOE_F32, MOE_BF16 = 0, 1
 MOE_MODE_AUTO, MOE_MODE_GEMV, MOE_MODE_GEMM = 0, 1, 2
 DEVERR_BAD_EXPERT, DEVERR_NULL_BLOB, DEVERR_NONFINITE, DEVERR_BAD_ROW = 1, 2, 4, 8
 MOE_DEVERR_TIMEOUT = 16
+DEVERR_MISALIGNED = 32
+MOE_HOOK_WAIT_LIMIT_NS, MOE_HOOK_DECODE_EXTRA_ARRIVALS, MOE_HOOK_GEMM_SPIN, MOE_HOOK_DECODE_ONE_KERNEL = 1, 2, 3, 4
 
 _STATUS = {1: "MOE_EINVAL", 2: "MOE_ENOMEM", 3: "MOE_ECUDA", 4: "MOE_EBUSY", 5: "MOE_ETIMEDOUT",
            6: "MOE_EIO", 7: "MOE_EDEVICE"}
@@ -64,6 +66,7 @@ def lib():
     sig = {
         "moe_last_error": (C.c_char_p, []),
         "moe_version": (I, []),
+        "moe_test_hook": (I, [I, C.c_int64]),
         "moe_kernel_launches": (C.c_uint64, []),
         "moe_device_error": (I, [P, I, S]),
         "moe_expert_blob_bytes": (Z, [I, I, I]),
@@ -90,6 +93,7 @@ def lib():
         "expcache_stats": (I, [P, C.POINTER(ExpCacheStats)]),
         "expcache_snapshot": (I, [P, P, P]),
         "expcache_inject_copy_failures": (I, [P, I]),
+        "expcache_copy_times": (I, [P, P, C.POINTER(C.c_float), C.POINTER(C.c_float)]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -130,6 +134,11 @@ def _check(rc: int):
 # ----------------------------------------------------------------- the ABI
 def moe_version() -> int:
     return lib().moe_version()
+
+
+def moe_test_hook(which: int, value: int) -> None:
+    """Sets a test hook (MOE_HOOK_*); 0 restores the default."""
+    _check(lib().moe_test_hook(which, int(value)))
 
 
 def moe_kernel_launches() -> int:
@@ -293,3 +302,10 @@ class ExpCache:
 
     def inject_copy_failures(self, n: int):
         _check(lib().expcache_inject_copy_failures(self.h, n))
+
+    def copy_times(self, ref_event):
+        """(start_ms, end_ms) of the last step's copies, measured from `ref_event`
+        (a torch.cuda.Event with timing, recorded earlier and completed)."""
+        a, b = C.c_float(0.0), C.c_float(0.0)
+        _check(lib().expcache_copy_times(self.h, C.c_void_p(ref_event.cuda_event), C.byref(a), C.byref(b)))
+        return a.value, b.value

@@ -61,6 +61,11 @@ int num_sms() {
     return g_sms[dev];
 }
 
+static std::atomic<long long> g_hooks[5];
+long long test_hook_value(int which) {
+    return which >= 1 && which <= 4 ? g_hooks[which].load(std::memory_order_relaxed) : 0;
+}
+
 static std::atomic<uint64_t> g_launches{0};
 void count_launches(int n) { g_launches.fetch_add(static_cast<uint64_t>(n), std::memory_order_relaxed); }
 
@@ -106,6 +111,14 @@ int moe_device_error(uint32_t *bits_out, int clear, moe_stream_t s) {
         set_error("device error word 0x%x", v);
         return MOE_EDEVICE;
     }
+    return MOE_OK;
+}
+
+int moe_test_hook(int which, int64_t value) {
+    t_err.clear();
+    REQUIRE(which >= 1 && which <= 4, "unknown test hook %d", which);
+    REQUIRE(value >= 0, "test hook value must be >= 0");
+    g_hooks[which].store(value, std::memory_order_relaxed);
     return MOE_OK;
 }
 

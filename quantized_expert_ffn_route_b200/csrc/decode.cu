@@ -37,8 +37,9 @@ __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.lau
 __host__ __device__ inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
 // Workspace layout (bytes): ids [32] int32 @0 | gates [32] fp32 @128 |
-// logits [E] @512 | h [(k+1) * I] fp32 (256-aligned).  Nothing in it needs
-// to start at any value.
+// grid-barrier arrival count (uint64) @256 (used by the one-kernel step;
+// zero before the first call) | logits [E] @512 | h [(k+1) * I] fp32
+// (256-aligned).
 struct DecodeWs {
     int32_t *ids;
     float *gates;
@@ -72,83 +73,6 @@ struct DecodeArgs {
     DecodeWs ws;
     unsigned *err;
 };
-
-// ------------------------------------------------------------ top-k
-// k best of N keys per lane by one warp.  Each lane first sorts its keys
-// (descending, a bitonic network on registers); then every round the warp
-// takes the largest head: a max reduction of the value halves, and only when
-// several heads share that value a second one of the low words (the larger
-// low word is the lower id).  The winning lane pops its head.  dst[r]
-// receives the rank-r key.
-template <int N>
-__device__ __forceinline__ void warp_take(uint64_t (&keys)[N], int k, int lane, uint64_t *dst) {
-#pragma unroll
-    for (int k2 = 2; k2 <= N; k2 <<= 1)
-#pragma unroll
-        for (int j = k2 >> 1; j > 0; j >>= 1)
-#pragma unroll
-            for (int i = 0; i < N; ++i) {
-                const int l = i ^ j;
-                if (l > i) {
-                    const bool desc = (i & k2) == 0;
-                    const uint64_t a = keys[i], b = keys[l];
-                    if (desc ? a < b : a > b) {
-                        keys[i] = b;
-                        keys[l] = a;
-                    }
-                }
-            }
-    for (int r = 0; r < k; ++r) {
-        const uint64_t head = keys[0];
-        const uint32_t hv = static_cast<uint32_t>(head >> 32);
-        const uint32_t hi = __reduce_max_sync(0xffffffffu, hv);
-        const unsigned tied = __ballot_sync(0xffffffffu, hv == hi);
-        int winner;
-        if (__popc(tied) == 1) {
-            winner = __ffs(tied) - 1;
-        } else {
-            const uint32_t lo = __reduce_max_sync(0xffffffffu, hv == hi ? static_cast<uint32_t>(head) : 0u);
-            winner = __ffs(__ballot_sync(0xffffffffu, hv == hi && static_cast<uint32_t>(head) == lo)) - 1;
-        }
-        const uint32_t wlo = __shfl_sync(0xffffffffu, static_cast<uint32_t>(head), winner);
-        if (lane == 0) dst[r] = (static_cast<uint64_t>(hi) << 32) | wlo;
-        if (lane == winner) {
-#pragma unroll
-            for (int q = 0; q + 1 < N; ++q) keys[q] = keys[q + 1];
-            keys[N - 1] = 0ull;
-        }
-    }
-}
-
-// Top-k (k <= 32) of E <= 1024 logits by one block of NW warps: each warp
-// takes the k best of its keys, then warp 0 the k best of the NW*k
-// candidates.  sel[0..k-1] receives the selection keys in rank order.
-template <int NW>
-__device__ void block_topk(const float *logits, int E, int k, uint64_t *cand, uint64_t *sel) {
-    constexpr int KPT = 1024 / (32 * NW);            // keys per thread
-    constexpr int CPL = NW;                          // candidates per lane in the second stage (NW*32/32)
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    {
-        uint64_t keys[KPT];
-#pragma unroll
-        for (int q = 0; q < KPT; ++q) {
-            const int e = threadIdx.x + 32 * NW * q;
-            keys[q] = e < E ? sel_key(__ldcg(logits + e), e) : 0ull;
-        }
-        warp_take(keys, k, lane, cand + warp * k);
-    }
-    __syncthreads();
-    if (warp == 0) {
-        uint64_t keys[CPL];
-#pragma unroll
-        for (int q = 0; q < CPL; ++q) {
-            const int i = lane + 32 * q;
-            keys[q] = i < NW * k ? cand[i] : 0ull;
-        }
-        warp_take(keys, k, lane, sel);
-    }
-    __syncthreads();
-}
 
 // ------------------------------------------------------------ 1. logits
 // One warp per router row, kLogitRows rows per CTA, so the E rows are read by
@@ -534,6 +458,14 @@ int launch_decode(int bits, const void *x, int x_dtype, const void *w_router, in
                   const float *logits_in, const uint8_t *const *blobs, const uint8_t *shared, int H, int I, int E,
                   int k, int32_t *ids, float *w, float *logits_out, float *y, void *ws, unsigned *err,
                   cudaStream_t s) {
+    if (test_hook_value(MOE_HOOK_DECODE_ONE_KERNEL) != 0 && decode_step_supported(bits, H, I, E, k, shared != nullptr)) {
+        // one persistent kernel (decode_step.cu); its grid-barrier count sits
+        // at byte 256 of the workspace, between the gates and the logits
+        const DecodeWs dw = decode_ws(ws, E);
+        return launch_decode_step(bits, x, x_dtype, w_router, w_dtype, bias, logits_in, blobs, shared, H, I, E, k, ids,
+                                  w, logits_out, y, dw.logits, dw.h,
+                                  reinterpret_cast<unsigned *>(static_cast<uint8_t *>(ws) + 256), err, s);
+    }
     DecodeArgs a;
     a.H = H; a.I = I; a.E = E; a.k = k;
     a.x = x; a.x_bf16 = x_dtype == MOE_BF16;

@@ -47,6 +47,8 @@ struct moe_expcache {
     cudaEvent_t ev_compute = nullptr;     // compute stream position at the last stage call
     cudaEvent_t ev_done = nullptr;        // all copies + table patch issued so far
     cudaEvent_t ev_stage[2] = {nullptr, nullptr};   // staging halves free again
+    cudaEvent_t ev_t0 = nullptr, ev_t1 = nullptr;     // timed: start / end of the last step's copies
+    bool timed = false;                               // ev_t0/ev_t1 have been recorded
     int stage_next = 0;
     std::vector<int32_t> slot_of, expert_in;
     std::vector<int64_t> cnt, last;
@@ -82,6 +84,8 @@ static void destroy_events(moe_expcache *c) {
     if (c->ev_done) cudaEventDestroy(c->ev_done);
     for (auto &e : c->ev_stage)
         if (e) cudaEventDestroy(e);
+    if (c->ev_t0) cudaEventDestroy(c->ev_t0);
+    if (c->ev_t1) cudaEventDestroy(c->ev_t1);
     if (c->copy) cudaStreamDestroy(c->copy);
 }
 
@@ -112,6 +116,8 @@ int expcache_create(const moe_expcache_desc *d, moe_expcache **out) {
     if (!rc) rc = cuda_status(cudaEventCreateWithFlags(&c->ev_done, cudaEventDisableTiming), "event");
     for (int i = 0; i < 2 && !rc; ++i)
         rc = cuda_status(cudaEventCreateWithFlags(&c->ev_stage[i], cudaEventDisableTiming), "event");
+    if (!rc) rc = cuda_status(cudaEventCreate(&c->ev_t0), "event");
+    if (!rc) rc = cuda_status(cudaEventCreate(&c->ev_t1), "event");
     if (!rc)
         rc = cuda_status(cudaMemsetAsync(d->dev_table, 0, sizeof(void *) * static_cast<size_t>(d->n_experts), c->copy),
                          "table clear");
@@ -242,6 +248,7 @@ int expcache_stage(moe_expcache *c, const int32_t *ids_host, int n, moe_stream_t
     // copies start after the compute work queued so far (it may still read victims' slots)
     int rc = cuda_status(cudaEventRecord(c->ev_compute, reinterpret_cast<cudaStream_t>(compute)), "event record");
     if (!rc) rc = cuda_status(cudaStreamWaitEvent(c->copy, c->ev_compute, 0), "stream wait");
+    if (!rc) rc = cuda_status(cudaEventRecord(c->ev_t0, c->copy), "event record");
     const size_t B = static_cast<size_t>(c->d.blob_bytes), S = static_cast<size_t>(c->d.slot_stride);
     auto *slab = static_cast<uint8_t *>(c->d.hbm_slab);
     auto *pool = static_cast<const uint8_t *>(c->d.host_pool);
@@ -283,7 +290,19 @@ int expcache_stage(moe_expcache *c, const int32_t *ids_host, int n, moe_stream_t
     }
     int rc2 = launch_table_patch(reinterpret_cast<const void **>(c->d.dev_table), patch, c->copy);
     if (!rc2) rc2 = cuda_status(cudaEventRecord(c->ev_done, c->copy), "event record");
+    if (!rc2) rc2 = cuda_status(cudaEventRecord(c->ev_t1, c->copy), "event record");
+    if (!rc2) c->timed = true;
     return rc ? rc : rc2;
+}
+
+int expcache_copy_times(moe_expcache *c, const void *ref_event, float *start_ms, float *end_ms) {
+    REQUIRE(c && ref_event && start_ms && end_ms, "cache/ref_event/start_ms/end_ms are NULL");
+    REQUIRE(c->timed, "no step has staged copies yet");
+    DeviceGuard guard(c->device);
+    cudaEvent_t ref = static_cast<cudaEvent_t>(const_cast<void *>(ref_event));
+    int rc = cuda_status(cudaEventElapsedTime(start_ms, ref, c->ev_t0), "elapsed time");
+    if (!rc) rc = cuda_status(cudaEventElapsedTime(end_ms, ref, c->ev_t1), "elapsed time");
+    return rc;
 }
 
 int expcache_join(moe_expcache *c, moe_stream_t s) {

@@ -37,7 +37,7 @@ constexpr int kDeq = 512;           // dequantising threads: 128 rows x 2 matric
 constexpr int kLoad = 64;           // token-row loader threads
 constexpr int kEpiWarp0 = 16, kMmaWarp = 20, kLoadWarp0 = 21;
 constexpr int kGemmThreads = 736;   // 16 dequant, 4 epilogue, 1 MMA, 2 loader warps
-constexpr long kSpin = 1L << 22;    // polls before a wait gives up (about a second)
+constexpr long kSpin = 1L << 22;    // polls before a wait gives up (about a second); the test hook may lower it
 constexpr int kMaxGroups = 4096;    // groups (active experts + shared) one launch may hold
 constexpr size_t kSmemLimit = 232448;
 
@@ -94,6 +94,7 @@ struct GemmArgs {
     float *y_shared;        // [T, H]
     int T, k, H, I, E;
     unsigned *err;
+    long spin;              // polls before a pipeline wait gives up (the drain before TMEM is freed keeps kSpin)
 };
 
 struct GroupInfo {
@@ -329,7 +330,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(GemmArgs a, int tile_c
                 // contents (slot u + 1 - R), then copy
                 int ok = 1;
                 if (lane == 0 && u + 1 >= R)
-                    ok = mbar_wait(rawEmpty + (u + 1) % R, static_cast<uint32_t>(((u + 1 - R) / R) & 1), kSpin);
+                    ok = mbar_wait(rawEmpty + (u + 1) % R, static_cast<uint32_t>(((u + 1 - R) / R) & 1), a.spin);
                 if (!__shfl_sync(0xffffffffu, ok, 0)) {
                     fail();
                     break;
@@ -340,7 +341,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(GemmArgs a, int tile_c
                 __syncwarp();
                 if (lane == 0) {
                     mbar_arrive(rawFull + slot);
-                    ok = mbar_wait(rawFull + slot, static_cast<uint32_t>((u / R) & 1), kSpin);
+                    ok = mbar_wait(rawFull + slot, static_cast<uint32_t>((u / R) & 1), a.spin);
                 }
                 if (!__shfl_sync(0xffffffffu, ok, 0)) {
                     fail();
@@ -351,7 +352,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(GemmArgs a, int tile_c
             const int sa = static_cast<int>(j % SA);
             // one lane per warp polls the stage barrier; the warp follows it
             int ok = 1;
-            if (lane == 0) ok = mbar_wait(emptyA + sa, static_cast<uint32_t>(((j / SA) & 1) ^ 1), kSpin);
+            if (lane == 0) ok = mbar_wait(emptyA + sa, static_cast<uint32_t>(((j / SA) & 1) ^ 1), a.spin);
             if (!__shfl_sync(0xffffffffu, ok, 0)) {
                 fail();
                 break;
@@ -411,7 +412,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(GemmArgs a, int tile_c
                 }
                 const int sb = static_cast<int>(j % SB);
                 int ok = 1;
-                if (lane == 0) ok = mbar_wait(emptyB + sb, static_cast<uint32_t>(((j / SB) & 1) ^ 1), kSpin);
+                if (lane == 0) ok = mbar_wait(emptyB + sb, static_cast<uint32_t>(((j / SB) & 1) ^ 1), a.spin);
                 if (!__shfl_sync(0xffffffffu, ok, 0)) {
                     fail();
                     break;
@@ -444,7 +445,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(GemmArgs a, int tile_c
             const TileEntry te = tiles[i];
             const int b = i % ACC;
             int ok = 1;
-            if (lane == 0) ok = mbar_wait(accF + b, static_cast<uint32_t>((i / ACC) & 1), kSpin);
+            if (lane == 0) ok = mbar_wait(accF + b, static_cast<uint32_t>((i / ACC) & 1), a.spin);
             if (!__shfl_sync(0xffffffffu, ok, 0)) {
                 fail();
                 break;
@@ -498,13 +499,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(GemmArgs a, int tile_c
             const int nmat = (GATEUP || te.m0 + kBM < a.H) ? 2 : 1;
             const int b = i % ACC;
             if (lane == 0) {
-                if (!mbar_wait(accE + b, static_cast<uint32_t>(((i / ACC) & 1) ^ 1), kSpin)) fail();
+                if (!mbar_wait(accE + b, static_cast<uint32_t>(((i / ACC) & 1) ^ 1), a.spin)) fail();
                 tc_fence_after();
                 for (int s = 0; s < nk && !abort_s; ++s) {
                     const long j = static_cast<long>(i) * nk + s;
                     const int sa = static_cast<int>(j % SA), sb = static_cast<int>(j % SB);
-                    if (!mbar_spin(fullA + sa, static_cast<uint32_t>((j / SA) & 1), kSpin * 16) ||
-                        !mbar_spin(fullB + sb, static_cast<uint32_t>((j / SB) & 1), kSpin * 16)) {
+                    if (!mbar_spin(fullA + sa, static_cast<uint32_t>((j / SA) & 1), a.spin * 16) ||
+                        !mbar_spin(fullB + sb, static_cast<uint32_t>((j / SB) & 1), a.spin * 16)) {
                         fail();
                         break;
                     }
@@ -644,6 +645,8 @@ int launch_gemm(int bits, const uint8_t *const *blobs, const int32_t *offsets, c
     a.I = I;
     a.E = E;
     a.err = err;
+    const long hook = test_hook_value(MOE_HOOK_GEMM_SPIN);
+    a.spin = hook > 0 ? hook : kSpin;
     {
         const long n = static_cast<long>(T) * H;
         long blocks = (n / 4 + 255) / 256;

@@ -37,6 +37,15 @@ int launch_decode(int bits, const void *x, int x_dtype, const void *w_router, in
                   int k, int32_t *ids, float *w, float *logits_out, float *y, void *ws, unsigned *err,
                   cudaStream_t s);
 
+bool decode_step_supported(int bits, int H, int I, int E, int k, bool shared);
+int launch_decode_step(int bits, const void *x, int x_dtype, const void *w_router, int w_dtype, const float *bias,
+                       const float *logits_in, const uint8_t *const *blobs, const uint8_t *shared, int H, int I,
+                       int E, int k, int32_t *ids, float *w, float *logits_out, float *y, float *logits_ws,
+                       float *h_ws, unsigned *bar, unsigned *err, cudaStream_t s);
+
+// Test hooks (moe_test_hook): the current value of a hook, 0 when unset.
+long long test_hook_value(int which);
+
 int launch_combine(const float *y_perm, const int32_t *perm_dst, const float *w, const float *y_shared, int T, int k,
                    int H, float *y, unsigned *err, cudaStream_t s);
 

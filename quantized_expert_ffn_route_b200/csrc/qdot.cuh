@@ -107,18 +107,20 @@ __device__ __forceinline__ void chunk_fx(const uint4 &code, const float4 (&xp)[Q
     // with the neighbouring x values of one float4, so operands sit in
     // register pairs as loaded.
     if constexpr (BITS == 4) {
-        float2 lo = make_float2(0.f, 0.f);
+        // four independent accumulators (one per code word), so consecutive
+        // packed FMAs do not wait on each other
+        float2 acc[4];
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
             const uint32_t L = (words[m] & 0x0F0F0F0Fu) | 0x80808080u;
             const uint32_t Hh = ((words[m] >> 4) & 0x0F0F0F0Fu) | 0x80808080u;
             const float4 a = xp[m], b = xp[4 + m];   // elements 4m..4m+3 (low nibbles), 16+4m.. (high)
-            lo = __ffma2_rn(make_float2(magic(L, 0), magic(L, 1)), make_float2(a.x, a.y), lo);
-            lo = __ffma2_rn(make_float2(magic(L, 2), magic(L, 3)), make_float2(a.z, a.w), lo);
-            lo = __ffma2_rn(make_float2(magic(Hh, 0), magic(Hh, 1)), make_float2(b.x, b.y), lo);
-            lo = __ffma2_rn(make_float2(magic(Hh, 2), magic(Hh, 3)), make_float2(b.z, b.w), lo);
+            acc[m] = __fmul2_rn(make_float2(magic(L, 0), magic(L, 1)), make_float2(a.x, a.y));
+            acc[m] = __ffma2_rn(make_float2(magic(L, 2), magic(L, 3)), make_float2(a.z, a.w), acc[m]);
+            acc[m] = __ffma2_rn(make_float2(magic(Hh, 0), magic(Hh, 1)), make_float2(b.x, b.y), acc[m]);
+            acc[m] = __ffma2_rn(make_float2(magic(Hh, 2), magic(Hh, 3)), make_float2(b.z, b.w), acc[m]);
         }
-        out[0] = lo.x + lo.y;
+        out[0] = ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) + ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
     } else {
         float2 acc[2][2] = {{make_float2(0.f, 0.f), make_float2(0.f, 0.f)},
                             {make_float2(0.f, 0.f), make_float2(0.f, 0.f)}};

@@ -142,3 +142,12 @@ def test_ffn_mode_shape_rules_on_host():
     # the allocation-free call takes the GEMV shapes only
     rc = L.moe_expert_ffn_noalloc(4, p, p, p, p, p, 1, 1, 2, 256, 2048, 16, None, p, None, None)
     assert rc == M.MOE_EINVAL and "I/32" in M.moe_last_error()
+
+
+def test_test_hooks_validate_arguments():
+    import quantized_expert_ffn_route_b200 as M
+    L = M.lib()
+    assert L.moe_test_hook(99, 1) == M.MOE_EINVAL
+    assert L.moe_test_hook(M.MOE_HOOK_GEMM_SPIN, -1) == M.MOE_EINVAL
+    for h in (M.MOE_HOOK_WAIT_LIMIT_NS, M.MOE_HOOK_DECODE_EXTRA_ARRIVALS, M.MOE_HOOK_GEMM_SPIN, M.MOE_HOOK_DECODE_ONE_KERNEL):
+        assert L.moe_test_hook(h, 0) == M.MOE_OK

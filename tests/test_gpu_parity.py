@@ -380,6 +380,22 @@ def test_null_blob_sets_error(decode_layer):
 
 
 # ------------------------------------------------------ fused decode step
+@pytest.fixture(params=["chain", "one_kernel"])
+def decode_path(request):
+    """Runs a test on both fused decode paths: the three-kernel chain (the
+    default) and the one-kernel persistent step (test hook)."""
+    M.moe_test_hook(M.MOE_HOOK_DECODE_ONE_KERNEL, 1 if request.param == "one_kernel" else 0)
+    yield request.param
+    M.moe_test_hook(M.MOE_HOOK_DECODE_ONE_KERNEL, 0)
+
+
+@pytest.fixture
+def one_kernel():
+    M.moe_test_hook(M.MOE_HOOK_DECODE_ONE_KERNEL, 1)
+    yield
+    M.moe_test_hook(M.MOE_HOOK_DECODE_ONE_KERNEL, 0)
+
+
 def _run_fused(g, x, x_dtype, logits_in=None):
     import quantized_expert_ffn_route_b200 as MM
     xdev = dev_x(x, x_dtype)
@@ -390,7 +406,7 @@ def _run_fused(g, x, x_dtype, logits_in=None):
                 w=b["w"][:g.k].cpu().numpy(), logits=b["logits"].cpu().numpy(), y=b["y"].cpu().numpy())
 
 
-def test_prepared_decode_matches_forward_decode():
+def test_prepared_decode_matches_forward_decode(decode_path):
     """The prepared one-token call runs the same kernels on the same buffers."""
     layer = W.make_layer(430, 4, 256, 256, 24, 4, shared=True, w_dtype="bf16")
     x = W.make_tokens(431, 3, 256, "bf16")
@@ -408,7 +424,7 @@ def test_prepared_decode_matches_forward_decode():
         assert np.array_equal(y1.cpu().numpy(), f["y"])
 
 
-def test_fused_decode_full_size(decode_layer):
+def test_fused_decode_full_size(decode_layer, decode_path):
     layer, g = decode_layer
     x = W.make_tokens(W.SEED["decode"] + 500, 6, layer.H, "bf16")
     ref = _sampled_ref(layer, x, np.arange(6))
@@ -421,14 +437,20 @@ def test_fused_decode_full_size(decode_layer):
         if dec[t]:
             assert np.array_equal(f["ids"], ref["ids"][t])
             assert rel_err(f["y"], ref["y"][t]) < GEMV_TOL
-        # same routing and outputs as the separate calls
+        # the gates are the softmax of the call's own selected logits (ids:
+        # the top-k of those logits, as the oracle selects them in fp32)
+        ids_own, w_own, _ = oracle.topk(f["logits"][None].astype(np.float32), layer.k)
+        assert np.array_equal(f["ids"], ids_own[0])
+        assert np.allclose(f["w"], w_own[0], rtol=4e-6, atol=1e-8)
+        # same routing and outputs as the separate calls (their logits are
+        # summed in another order: gates agree within the logit error bound)
         m = run_gpu(g, x[t:t + 1], "bf16", mode=M.MOE_MODE_GEMV)
         assert np.array_equal(f["ids"], m["ids"][0])
-        assert np.allclose(f["w"], m["w"][0], rtol=1e-6, atol=1e-7)
+        assert np.allclose(f["w"], m["w"][0], rtol=4 * float(eps[t].max()) + 4e-6, atol=1e-8)
         assert rel_err(f["y"], m["y"][0]) < 1e-4   # two fp32 orders of the same cancellation, each ~2e-5
 
 
-def test_fused_decode_q2_bias(verify_layer):
+def test_fused_decode_q2_bias(verify_layer, decode_path):
     layer, g = verify_layer
     x = W.make_tokens(W.SEED["verify"] + 900, 3, layer.H, "bf16")
     ref = _sampled_ref(layer, x, np.arange(3))
@@ -442,11 +464,15 @@ def test_fused_decode_q2_bias(verify_layer):
             assert rel_err(f["y"], ref["y"][t]) < GEMV_TOL
 
 
-@pytest.mark.parametrize("bits,dt,shared", [(4, "f32", False), (2, "bf16", True), (4, "bf16", True)])
-def test_fused_decode_small(bits, dt, shared):
-    layer = W.make_layer(400 + bits, bits, 256, 256, 24, 4, shared=shared, w_dtype=dt)
-    x = W.make_tokens(401 + bits, 3, 256, dt)
-    ref = oracle.moe_layer(bits, x, dt, layer.blobs, k=4, H=256, I=256, E=24, w_router=layer.w_router,
+@pytest.mark.parametrize("bits,dt,shared,H,I", [(4, "f32", False, 256, 256), (2, "bf16", True, 256, 256),
+                                               (4, "bf16", True, 256, 256), (4, "bf16", True, 256, 128),
+                                               (2, "f32", False, 384, 256)])
+def test_fused_decode_small(bits, dt, shared, H, I, decode_path):
+    """H and I multiples of 256: the one-kernel step; I = 128 or H = 384
+    (scale rows not 16-byte multiples): the three-kernel chain."""
+    layer = W.make_layer(400 + bits, bits, H, I, 24, 4, shared=shared, w_dtype=dt)
+    x = W.make_tokens(401 + bits, 3, H, dt)
+    ref = oracle.moe_layer(bits, x, dt, layer.blobs, k=4, H=H, I=I, E=24, w_router=layer.w_router,
                            w_dtype=dt, shared_blob=layer.shared)
     g = _layer_gpu(layer)
     eps = logit_bound(layer, x, dt)
@@ -459,7 +485,7 @@ def test_fused_decode_small(bits, dt, shared):
             assert rel_err(f["y"], ref["y"][t]) < GEMV_TOL
 
 
-def test_fused_decode_logits_in():
+def test_fused_decode_logits_in(decode_path):
     """Router logits given directly (the paging path), with exact ties."""
     layer = W.make_layer(410, 2, 256, 256, 64, 6, shared=False, w_dtype="bf16")
     x = W.make_tokens(411, 2, 256, "bf16")
@@ -472,3 +498,88 @@ def test_fused_decode_logits_in():
         assert f["err"] == 0
         assert np.array_equal(f["ids"], ref["ids"][t])
         assert rel_err(f["y"], ref["y"][t]) < GEMV_TOL
+
+
+def test_fused_decode_is_one_kernel_and_replays_from_a_graph(decode_layer, one_kernel):
+    """At full size the one-kernel step is a single kernel launch; captured in
+    a CUDA graph and replayed it gives the eager result bit for bit, call
+    after call; its grid-barrier arrival count moves on by exactly two
+    arrivals per CTA per call."""
+    layer, g = decode_layer
+    x = W.make_tokens(W.SEED["decode"] + 700, 3, layer.H, "bf16")
+    b = g.decode_buffers()
+
+    def count():
+        return int(b["ws"][256:264].cpu().numpy().view(np.uint64)[0])
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    eager = []
+    for t in range(3):
+        n0, c0 = M.moe_kernel_launches(), count()
+        f = _run_fused(g, x[t:t + 1], "bf16")
+        assert f["err"] == 0 and M.moe_kernel_launches() - n0 == 1
+        assert count() - c0 == 2 * sms
+        eager.append(f)
+    xd = torch.empty(1, layer.H, dtype=torch.bfloat16, device="cuda")
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(graph, stream=s):
+            g.forward_decode(xd, M.MOE_BF16, stream=s)
+    torch.cuda.current_stream().wait_stream(s)
+    c0 = count()
+    for t in (2, 0, 1):
+        xd.copy_(dev_x(x[t:t + 1], "bf16"))
+        graph.replay()
+        torch.cuda.synchronize()
+        assert M.moe_device_error(clear=True) == 0
+        assert np.array_equal(b["ids"][:layer.k].cpu().numpy(), eager[t]["ids"])
+        assert np.array_equal(b["y"].cpu().numpy(), eager[t]["y"])
+    assert count() - c0 == 3 * 2 * sms
+
+
+def test_fused_decode_barrier_timeout_recovers(decode_layer, one_kernel):
+    """A grid barrier that can never complete (the test hook makes it wait
+    for one CTA more than the grid has) runs out after its 2 ms limit: the
+    call sets MOE_DEVERR_TIMEOUT and returns; with the hook cleared and the
+    workspace zeroed again, the next call is exact."""
+    layer, g = decode_layer
+    x = W.make_tokens(W.SEED["decode"] + 800, 1, layer.H, "bf16")
+    good = _run_fused(g, x, "bf16")
+    assert good["err"] == 0
+    b = g.decode_buffers()
+    M.moe_test_hook(M.MOE_HOOK_WAIT_LIMIT_NS, 2_000_000)
+    M.moe_test_hook(M.MOE_HOOK_DECODE_EXTRA_ARRIVALS, 1)
+    try:
+        g.forward_decode(dev_x(x, "bf16"), M.MOE_BF16)
+        torch.cuda.synchronize()
+        err = M.moe_device_error(clear=True)
+    finally:
+        M.moe_test_hook(M.MOE_HOOK_DECODE_EXTRA_ARRIVALS, 0)
+        M.moe_test_hook(M.MOE_HOOK_WAIT_LIMIT_NS, 0)
+    assert err & M.MOE_DEVERR_TIMEOUT
+    b["ws"].zero_()
+    again = _run_fused(g, x, "bf16")
+    assert again["err"] == 0
+    assert np.array_equal(again["ids"], good["ids"]) and np.array_equal(again["y"], good["y"])
+
+
+def test_gemm_wait_timeout_recovers():
+    """The grouped GEMM's pipeline waits limited to two polls (test hook) run
+    out: the call sets MOE_DEVERR_TIMEOUT, every role leaves its loop, TMEM is
+    freed (the kernel returns), and the next call with the normal limit is
+    exact."""
+    layer = W.make_layer(72, 4, 256, 256, 8, 2, shared=True, w_dtype="bf16")
+    x = W.make_tokens(73, 300, 256, "bf16")
+    g = _layer_gpu(layer)
+    M.moe_test_hook(M.MOE_HOOK_GEMM_SPIN, 2)
+    try:
+        out = run_gpu(g, x, "bf16", mode=M.MOE_MODE_GEMM)
+    finally:
+        M.moe_test_hook(M.MOE_HOOK_GEMM_SPIN, 0)
+    assert out["err"] & M.MOE_DEVERR_TIMEOUT
+    ref = oracle.moe_layer(4, x, "bf16", layer.blobs, k=2, H=256, I=256, E=8, w_router=layer.w_router,
+                           w_dtype="bf16", shared_blob=layer.shared)
+    for _ in range(2):
+        out = run_gpu(g, x, "bf16", mode=M.MOE_MODE_GEMM)
+        _check_layer(out, ref, layer, x, "bf16")

@@ -46,7 +46,7 @@ __device__ __forceinline__ bool group_of(int g, int n_act, const int32_t *active
 constexpr int kGvThreads = 256;
 constexpr int kGvWarps = kGvThreads / 32;
 constexpr int kGvRows = 16;      // gate/up rows per task (2 per warp)
-constexpr int kGvNT = 16;        // token rows staged per pass
+constexpr int kGvNT = 8;         // token rows staged per pass (8: two CTAs fit an SM)
 // down: row groups per warp (4-bit codes need more registers per chunk)
 template <int BITS>
 struct GvTPW { static constexpr int value = BITS == 4 ? 2 : 4; };

@@ -14,9 +14,10 @@
 //               copies are whole lines), then each thread dequantises one
 //               32-weight block per k-step to fp16 into a 128-byte-swizzled
 //               A stage;
-//   warps 21-22 gather the tile's token rows (fp16) into the B stages with
+//   warps 21-28 gather the tile's token rows (fp16) into the B stages with
 //               cp.async, a few k-steps ahead; each warp publishes a stage
-//               with one barrier arrival once its copies have landed;
+//               with one barrier arrival once its copies have landed (eight
+//               warps: with two, the gather set the pace of every k-step);
 //   warp  20    allocates TMEM and issues tcgen05.mma (one thread);
 //   warps 16-19 epilogue: tcgen05.ld the fp32 accumulators and write
 //               gate/up -> h = silu(g) * u (fp16) or down -> y rows (fp32).
@@ -34,9 +35,9 @@ using namespace sm100;
 constexpr int kBM = 128;            // weight rows per matrix of a tile (MMA M)
 constexpr int kBK = 64;             // K per stage: one 128-byte row of fp16
 constexpr int kDeq = 512;           // dequantising threads: 128 rows x 2 matrices x 2 blocks
-constexpr int kLoad = 64;           // token-row loader threads
+constexpr int kLoad = 256;          // token-row loader threads (8 warps: the token-row gather sets the pace)
 constexpr int kEpiWarp0 = 16, kMmaWarp = 20, kLoadWarp0 = 21;
-constexpr int kGemmThreads = 736;   // 16 dequant, 4 epilogue, 1 MMA, 2 loader warps
+constexpr int kGemmThreads = 672 + kLoad;   // 16 dequant, 4 epilogue, 1 MMA, kLoad / 32 loader warps
 constexpr long kSpin = 1L << 22;    // polls before a wait gives up (about a second); the test hook may lower it
 constexpr int kMaxGroups = 4096;    // groups (active experts + shared) one launch may hold
 constexpr size_t kSmemLimit = 232448;
@@ -373,10 +374,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(GemmArgs a, int tile_c
         cp_async_wait<0>();
     } else if (warp >= kLoadWarp0) {
         // --------------------------------------------------- token rows
-        // Loader warp lw copies rows lw*MAXN/2 .. of each tile: lane = 8 x row
+        // Loader warp lw copies rows lw * HALF .. of each tile: lane = 8 x row
         // + 16-byte chunk.  Its token indices live in a warp-private table.
         const int lw = warp - kLoadWarp0;
-        constexpr int HALF = MAXN / 2;
+        constexpr int HALF = MAXN / (kLoad / 32);       // rows of each tile this warp copies
         int32_t *tok = tok_s + lw * HALF;
         const uint8_t *bsrc = GATEUP ? reinterpret_cast<const uint8_t *>(a.x16)
                                      : reinterpret_cast<const uint8_t *>(a.h16);

@@ -14,7 +14,7 @@
 //               copies are whole lines), then each thread dequantises one
 //               32-weight block per k-step to fp16 into a 128-byte-swizzled
 //               A stage;
-//   warps 21-28 gather the tile's token rows (fp16) into the B stages with
+//   warps 21+ gather the tile's token rows (fp16) into the B stages with
 //               cp.async, a few k-steps ahead; each warp publishes a stage
 //               with one barrier arrival once its copies have landed (eight
 //               warps: with two, the gather set the pace of every k-step);
@@ -35,9 +35,12 @@ using namespace sm100;
 constexpr int kBM = 128;            // weight rows per matrix of a tile (MMA M)
 constexpr int kBK = 64;             // K per stage: one 128-byte row of fp16
 constexpr int kDeq = 512;           // dequantising threads: 128 rows x 2 matrices x 2 blocks
-constexpr int kLoad = 256;          // token-row loader threads (8 warps: the token-row gather sets the pace)
+// Token-row loader threads: 8 warps for 256-token tiles (there the gather
+// sets the pace of every k-step), 2 for 64-token tiles (there the weights do).
+__host__ __device__ constexpr int gemm_loaders(int maxn) { return maxn > 64 ? 256 : 64; }
+__host__ __device__ constexpr int gemm_threads(int maxn) { return 672 + gemm_loaders(maxn); }
 constexpr int kEpiWarp0 = 16, kMmaWarp = 20, kLoadWarp0 = 21;
-constexpr int kGemmThreads = 672 + kLoad;   // 16 dequant, 4 epilogue, 1 MMA, kLoad / 32 loader warps
+// threads: 16 dequant, 4 epilogue, 1 MMA and gemm_loaders / 32 loader warps
 constexpr long kSpin = 1L << 22;    // polls before a wait gives up (about a second); the test hook may lower it
 constexpr int kMaxGroups = 4096;    // groups (active experts + shared) one launch may hold
 constexpr size_t kSmemLimit = 232448;
@@ -165,7 +168,7 @@ __device__ __forceinline__ void dequant_block(const uint8_t *codes, __half2 d2, 
 }
 
 template <int BITS, bool GATEUP, int MAXN>
-__global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(GemmArgs a, int tile_cap) {
+__global__ void __launch_bounds__(gemm_threads(MAXN), 1) k_gemm(GemmArgs a, int tile_cap) {
     using Cfg = GemmCfg<BITS, GATEUP, MAXN>;
     constexpr int SA = Cfg::SA, SB = Cfg::SB, R = Cfg::R, ACC = Cfg::ACC;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -202,7 +205,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(GemmArgs a, int tile_c
             mbar_init(emptyA + i, 1);
         }
         for (int i = 0; i < SB; ++i) {
-            mbar_init(fullB + i, kLoad / 32);          // one arrival per loader warp
+            mbar_init(fullB + i, gemm_loaders(MAXN) / 32);   // one arrival per loader warp
             mbar_init(emptyB + i, 1);
         }
         for (int i = 0; i < 2; ++i) {
@@ -377,7 +380,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(GemmArgs a, int tile_c
         // Loader warp lw copies rows lw * HALF .. of each tile: lane = 8 x row
         // + 16-byte chunk.  Its token indices live in a warp-private table.
         const int lw = warp - kLoadWarp0;
-        constexpr int HALF = MAXN / (kLoad / 32);       // rows of each tile this warp copies
+        constexpr int HALF = MAXN / (gemm_loaders(MAXN) / 32);   // rows of each tile this warp copies
         int32_t *tok = tok_s + lw * HALF;
         const uint8_t *bsrc = GATEUP ? reinterpret_cast<const uint8_t *>(a.x16)
                                      : reinterpret_cast<const uint8_t *>(a.h16);
@@ -611,7 +614,7 @@ static int launch_k_gemm(const GemmArgs &a, int cap, cudaStream_t s) {
                                               static_cast<int>(smem)),
                          "gemm smem attribute");
     if (rc) return rc;
-    k_gemm<BITS, GATEUP, MAXN><<<num_sms(), kGemmThreads, smem, s>>>(a, cap);
+    k_gemm<BITS, GATEUP, MAXN><<<num_sms(), gemm_threads(MAXN), smem, s>>>(a, cap);
     count_launches(1);
     return cuda_status(cudaGetLastError(), "gemm launch");
 }

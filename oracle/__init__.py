@@ -64,6 +64,8 @@ def lib():
         _lib.oracle_combine.argtypes = [I32, I32, I32, P, P, P, P, P]
         _lib.oracle_cache_sim.restype = C.c_long
         _lib.oracle_cache_sim.argtypes = [I32, I32, I32, I32, I32, P, P, P, P, P]
+        _lib.oracle_cache_sim_prefetch.restype = C.c_long
+        _lib.oracle_cache_sim_prefetch.argtypes = [I32, I32, I32, I32, I32, P, I32, P, P, P, P, P, P, P, P]
     return _lib
 
 
@@ -219,3 +221,26 @@ def cache_sim(ids: np.ndarray, n_experts: int, capacity: int, decay_period: int)
     if m < 0:
         raise ValueError("invalid cache trace")
     return dict(slot=slot, hit=hit.astype(bool), victim=victim, misses=int(m), counts=counts)
+
+
+def cache_sim_prefetch(ids: np.ndarray, pf_ids: np.ndarray, n_experts: int, capacity: int, decay_period: int):
+    """ids [steps, n], pf_ids [steps, npf] (-1 = none, prefetched after each
+    step's stage) -> dict(slot, hit, victim, pf_slot, pf_victim, misses,
+    prefetched, counts)."""
+    ids = _c(ids, np.int32)
+    pf_ids = _c(pf_ids, np.int32)
+    steps, n = ids.shape
+    npf = pf_ids.shape[1] if pf_ids.ndim == 2 else 0
+    assert pf_ids.shape[0] == steps
+    slot = np.empty((steps, n), np.int32); hit = np.empty((steps, n), np.int8)
+    victim = np.empty((steps, n), np.int32)
+    pf_slot = np.empty((steps, max(1, npf)), np.int32); pf_victim = np.empty((steps, max(1, npf)), np.int32)
+    counts = np.empty(n_experts, np.int64)
+    adm = C.c_long(0)
+    m = lib().oracle_cache_sim_prefetch(n_experts, capacity, decay_period, steps, n, _p(ids), npf, _p(pf_ids),
+                                        _p(slot), _p(hit), _p(victim), _p(pf_slot), _p(pf_victim), _p(counts),
+                                        C.byref(adm))
+    if m < 0:
+        raise ValueError("invalid cache trace")
+    return dict(slot=slot, hit=hit.astype(bool), victim=victim, pf_slot=pf_slot[:, :npf], pf_victim=pf_victim[:, :npf],
+                misses=int(m), prefetched=int(adm.value), counts=counts)

@@ -508,3 +508,160 @@ bad:
     free(last);
     return -1;
 }
+
+/* The same policy with prefetch (reading: the pages keep hot experts resident
+ * and move the rest in; loading the next layer's likely experts ahead of
+ * their use is the cross-layer form of that).  After the stage of step s, the
+ * ids pf_ids[s][0..npf) (-1 = none) are prefetched in order:
+ *  - a resident id (or -1): nothing happens (pf_slot = pf_victim = -1);
+ *  - otherwise the id enters the lowest free slot, else the slot of the
+ *    resident expert smallest in (counter, last use, id) that is neither one
+ *    of step s's ids nor on the prefetch list (the list names the experts
+ *    expected next: none of them is evicted for another); if no such expert
+ *    exists the id is skipped (pf_slot = -1);
+ *  - a prefetch is not a use: counters and last uses do not change.
+ * Stage outputs as oracle_cache_sim; pf_slot_out / pf_victim_out [steps][npf].
+ * *pf_admitted_out (optional) = the number of ids prefetched into a slot.
+ * Returns the stage misses, or -1 on invalid input. */
+long oracle_cache_sim_prefetch(int n_experts, int capacity, int decay_period, int steps, int n,
+                               const int32_t *ids, int npf, const int32_t *pf_ids,
+                               int32_t *slot_out, int8_t *hit_out, int32_t *victim_out,
+                               int32_t *pf_slot_out, int32_t *pf_victim_out,
+                               int64_t *counts_out, long *pf_admitted_out)
+{
+    if (n > capacity || capacity <= 0 || npf < 0)
+        return -1;
+    int32_t *slot_of = (int32_t *)malloc(sizeof(int32_t) * (size_t)n_experts);
+    int32_t *expert_in = (int32_t *)malloc(sizeof(int32_t) * (size_t)capacity);
+    int64_t *cnt = (int64_t *)calloc((size_t)n_experts, sizeof(int64_t));
+    int64_t *last = (int64_t *)malloc(sizeof(int64_t) * (size_t)n_experts);
+    int8_t *guard = (int8_t *)calloc((size_t)n_experts, 1);   /* protected from eviction */
+    for (int e = 0; e < n_experts; ++e) {
+        slot_of[e] = -1;
+        last[e] = -1;
+    }
+    for (int s = 0; s < capacity; ++s)
+        expert_in[s] = -1;
+    long misses = 0, admitted = 0;
+    for (int s = 0; s < steps; ++s) {
+        const int32_t *step_ids = ids + (size_t)s * n;
+        for (int j = 0; j < n; ++j) {
+            if (step_ids[j] < 0 || step_ids[j] >= n_experts)
+                goto bad;
+            for (int i = 0; i < j; ++i)
+                if (step_ids[i] == step_ids[j])
+                    goto bad;
+        }
+        if (decay_period > 0 && s > 0 && s % decay_period == 0)
+            for (int e = 0; e < n_experts; ++e)
+                cnt[e] /= 2;
+        for (int j = 0; j < n; ++j)
+            guard[step_ids[j]] = 1;
+        /* stage: the policy of oracle_cache_sim */
+        for (int j = 0; j < n; ++j) {
+            int e = step_ids[j];
+            size_t o = (size_t)s * n + j;
+            cnt[e] += 1;
+            last[e] = s;
+            victim_out[o] = -1;
+            if (slot_of[e] >= 0) {
+                hit_out[o] = 1;
+                slot_out[o] = slot_of[e];
+                continue;
+            }
+            hit_out[o] = 0;
+            misses++;
+            int slot = -1;
+            for (int sl = 0; sl < capacity; ++sl)
+                if (expert_in[sl] < 0) {
+                    slot = sl;
+                    break;
+                }
+            if (slot < 0) {
+                int best = -1;
+                for (int sl = 0; sl < capacity; ++sl) {
+                    int c = expert_in[sl];
+                    if (guard[c])
+                        continue;
+                    if (best < 0 || cnt[c] < cnt[best] ||
+                        (cnt[c] == cnt[best] && (last[c] < last[best] ||
+                                                 (last[c] == last[best] && c < best))))
+                        best = c;
+                }
+                slot = slot_of[best];
+                slot_of[best] = -1;
+                victim_out[o] = best;
+            }
+            expert_in[slot] = e;
+            slot_of[e] = slot;
+            slot_out[o] = slot;
+        }
+        /* prefetch after the stage: the whole list is protected */
+        for (int j = 0; j < npf; ++j) {
+            int e = pf_ids[(size_t)s * npf + j];
+            if (e < -1 || e >= n_experts)
+                goto bad;
+            if (e >= 0)
+                guard[e] = 1;
+        }
+        for (int j = 0; j < npf; ++j) {
+            size_t o = (size_t)s * npf + j;
+            int e = pf_ids[o];
+            pf_slot_out[o] = -1;
+            pf_victim_out[o] = -1;
+            if (e < -1 || e >= n_experts)
+                goto bad;
+            if (e < 0 || slot_of[e] >= 0)
+                continue;
+            int slot = -1;
+            for (int sl = 0; sl < capacity; ++sl)
+                if (expert_in[sl] < 0) {
+                    slot = sl;
+                    break;
+                }
+            if (slot < 0) {
+                int best = -1;
+                for (int sl = 0; sl < capacity; ++sl) {
+                    int c = expert_in[sl];
+                    if (guard[c])
+                        continue;
+                    if (best < 0 || cnt[c] < cnt[best] ||
+                        (cnt[c] == cnt[best] && (last[c] < last[best] ||
+                                                 (last[c] == last[best] && c < best))))
+                        best = c;
+                }
+                if (best < 0)
+                    continue;                        /* everything resident is protected */
+                slot = slot_of[best];
+                slot_of[best] = -1;
+                pf_victim_out[o] = best;
+            }
+            expert_in[slot] = e;
+            slot_of[e] = slot;
+            pf_slot_out[o] = slot;
+            admitted++;
+        }
+        for (int j = 0; j < n; ++j)
+            guard[step_ids[j]] = 0;
+        for (int j = 0; j < npf; ++j)
+            if (pf_ids[(size_t)s * npf + j] >= 0)
+                guard[pf_ids[(size_t)s * npf + j]] = 0;
+    }
+    if (counts_out)
+        memcpy(counts_out, cnt, sizeof(int64_t) * (size_t)n_experts);
+    if (pf_admitted_out)
+        *pf_admitted_out = admitted;
+    free(slot_of);
+    free(expert_in);
+    free(cnt);
+    free(last);
+    free(guard);
+    return misses;
+bad:
+    free(slot_of);
+    free(expert_in);
+    free(cnt);
+    free(last);
+    free(guard);
+    return -1;
+}

@@ -127,3 +127,37 @@ def test_cache_rejects_oversubscription_and_bad_ids():
     slots, nm = cache.lookup(np.array([0, 1]))
     assert slots[0] == -1 and slots[1] >= 0 and nm == 1
     cache.close()
+
+
+def test_cache_events_full_paging_trace():
+    """The paging workload's whole trace (24,576 experts, 2048 HBM slots,
+    5000 steps of 10 Gumbel-top-k ids over a Zipf popularity that drifts every
+    200 steps, halving every 256 steps) through expcache_stage: every hit,
+    slot and victim equals the oracle simulator's.  Blobs are 16 bytes here:
+    the policy, not the copy size, is under test."""
+    c = W.PAGING
+    E, k, cap, steps, decay = c["E"], c["k"], c["capacity"], c["steps"], 256
+    # the k largest logits of each step (any k distinct ids serve: the cache
+    # and the simulator see the same ones)
+    ids = np.stack([np.argpartition(-l, k - 1)[:k] for l in
+                    W.paging_trace(W.SEED["paging"], E, k, steps, s=c["zipf_s"], drift_every=c["drift_every"],
+                                   drift_prob=c["drift_prob"], hot=c["hot"])]).astype(np.int32)
+    ref = oracle.cache_sim(ids, E, cap, decay)
+    stride = 256
+    host = torch.zeros(E * stride, dtype=torch.uint8, pin_memory=True)
+    slab = torch.zeros(cap * stride, dtype=torch.uint8, device="cuda")
+    table = torch.zeros(E, dtype=torch.int64, device="cuda")
+    cache = M.ExpCache(E, cap, 16, stride, host, slab, table, decay)
+    try:
+        for st in range(steps):
+            hit, slot, victim = cache.stage(ids[st])
+            assert np.array_equal(hit.astype(bool), ref["hit"][st]), st
+            assert np.array_equal(slot, ref["slot"][st]), st
+            assert np.array_equal(victim, ref["victim"][st]), st
+        assert cache.wait(10_000_000) == M.MOE_OK
+        st = cache.stats()
+        assert st["misses"] == ref["misses"] and st["hits"] == steps * k - ref["misses"]
+        cnt, _ = cache.snapshot()
+        assert np.array_equal(cnt, ref["counts"])
+    finally:
+        cache.close()

@@ -161,3 +161,116 @@ def test_cache_rejects_bad_trace(oracle_lib):
         oracle_lib.cache_sim(np.array([[1, 2, 3]], np.int32), 4, 2, 0)  # n > capacity
     with pytest.raises(ValueError):
         oracle_lib.cache_sim(np.array([[7]], np.int32), 4, 2, 0)      # id out of range
+
+
+# ------------------------------------------------------------ with prefetch
+def _prefetch_golden():
+    rows, out = [], {}
+    for line in (GOLDEN / "cache_prefetch_trace.txt").read_text().splitlines():
+        line = line.strip()
+        if not line or line.startswith("#"):
+            continue
+        if line.startswith("stage"):
+            head, rest = line.split(":", 1)
+            stage, pf = rest.split("|")
+            e, hit, slot, victim = (int(v) for v in stage.split())
+            pfi, pfo = pf.split("->")
+            pfs, pfv = pfo.split(";")
+            rows.append(dict(id=e, hit=hit, slot=slot, victim=victim, pf=[int(v) for v in pfi.split()],
+                             pf_slot=[int(v) for v in pfs.split()], pf_victim=[int(v) for v in pfv.split()]))
+        else:
+            f = line.split()
+            out[f[0]] = [int(v) for v in f[1:]]
+    return rows, out
+
+
+def test_prefetch_sim_hand_worked_trace(oracle_lib):
+    rows, out = _prefetch_golden()
+    ids = np.array([[r["id"]] for r in rows], np.int32)
+    pf = np.array([r["pf"] for r in rows], np.int32)
+    got = oracle_lib.cache_sim_prefetch(ids, pf, 6, 3, 0)
+    assert got["hit"][:, 0].astype(int).tolist() == [r["hit"] for r in rows]
+    assert got["slot"][:, 0].tolist() == [r["slot"] for r in rows]
+    assert got["victim"][:, 0].tolist() == [r["victim"] for r in rows]
+    assert got["pf_slot"].tolist() == [r["pf_slot"] for r in rows]
+    assert got["pf_victim"].tolist() == [r["pf_victim"] for r in rows]
+    assert got["misses"] == out["misses"][0] and got["prefetched"] == out["prefetched"][0]
+    assert got["counts"].tolist() == out["counts"]
+
+
+def test_prefetch_sim_without_prefetch_is_the_plain_policy(oracle_lib):
+    rng = np.random.default_rng(21)
+    for E, cap, decay, n in ((40, 10, 8, 4), (300, 32, 16, 10)):
+        ids = np.stack([rng.choice(E, n, replace=False) for _ in range(400)]).astype(np.int32)
+        a = oracle_lib.cache_sim(ids, E, cap, decay)
+        b = oracle_lib.cache_sim_prefetch(ids, np.full((400, 3), -1, np.int32), E, cap, decay)
+        for key in ("slot", "hit", "victim", "counts"):
+            assert np.array_equal(a[key], b[key]), key
+        assert a["misses"] == b["misses"] and b["prefetched"] == 0
+
+
+def _prefetch_sim_sorted(ids, pf, E, cap, decay):
+    """Independent restatement: the resident set as a dict, victims picked by
+    sorting the unprotected residents on (count, last use, id)."""
+    slot_of, free, cnt, last = {}, list(range(cap)), [0] * E, [-1] * E
+    ev, pev, misses = [], [], 0
+    for s in range(ids.shape[0]):
+        if decay and s and s % decay == 0:
+            cnt = [c // 2 for c in cnt]
+        step = [int(v) for v in ids[s]]
+        prot = set(step)
+
+        def place(e):
+            if free:
+                free.sort()
+                return free.pop(0), -1
+            cand = sorted((cnt[c], last[c], c) for c in slot_of if c not in prot)
+            if not cand:
+                return None, -1
+            v = cand[0][2]
+            return slot_of.pop(v), v
+        for e in step:
+            cnt[e] += 1
+            last[e] = s
+            if e in slot_of:
+                ev.append((1, slot_of[e], -1))
+                continue
+            misses += 1
+            sl, v = place(e)
+            slot_of[e] = sl
+            ev.append((0, sl, v))
+        prot |= {int(v) for v in pf[s] if v >= 0}
+        for e in (int(v) for v in pf[s]):
+            if e < 0 or e in slot_of:
+                pev.append((-1, -1))
+                continue
+            sl, v = place(e)
+            if sl is None:
+                pev.append((-1, -1))
+                continue
+            slot_of[e] = sl
+            pev.append((sl, v))
+    return ev, pev, misses, cnt
+
+
+def test_prefetch_sim_matches_an_independent_simulator(oracle_lib):
+    rng = np.random.default_rng(22)
+    E, cap, decay, n, npf, steps = 60, 12, 16, 4, 3, 300
+    ids = np.stack([rng.choice(E, n, replace=False) for _ in range(steps)]).astype(np.int32)
+    pf = rng.integers(-1, E, size=(steps, npf)).astype(np.int32)
+    got = oracle_lib.cache_sim_prefetch(ids, pf, E, cap, decay)
+    ev, pev, misses, cnt = _prefetch_sim_sorted(ids, pf, E, cap, decay)
+    assert [tuple(v) for v in zip(got["hit"].ravel().astype(int), got["slot"].ravel(), got["victim"].ravel())] == ev
+    assert list(zip(got["pf_slot"].ravel().tolist(), got["pf_victim"].ravel().tolist())) == pev
+    assert got["misses"] == misses and got["counts"].tolist() == cnt
+
+
+def test_prefetching_the_next_step_leaves_only_the_first_misses(oracle_lib):
+    """A prefetch of exactly the next step's ids (room for both steps) turns
+    every later access into a hit."""
+    rng = np.random.default_rng(23)
+    E, cap, n, steps = 200, 24, 8, 100
+    ids = np.stack([rng.choice(E, n, replace=False) for _ in range(steps)]).astype(np.int32)
+    pf = np.vstack([ids[1:], np.full((1, n), -1, np.int32)])
+    got = oracle_lib.cache_sim_prefetch(ids, pf, E, cap, 0)
+    assert got["misses"] == n and got["hit"][1:].all()

@@ -688,6 +688,141 @@ def bench_paging(args, world, rank, pk):
                 launches=launches, config=cfg, dtype="fp32 (CUDA-core FMA on 2-bit codes)")
 
 
+def bench_paging48(args, world, rank, pk):
+    """48 layers x 512 two-bit experts = the 24,576-expert pool in page-locked
+    host memory, one cache of 2048 HBM slots, 10 experts per layer per token,
+    the next layer's most used experts prefetched while a layer computes."""
+    import torch
+    import quantized_expert_ffn_route_b200 as M
+    import workloads as W
+    from quantized_expert_ffn_route_b200.paged import PagedExpertStack
+    c = W.PAGING48
+    L, El, k, H, I, cap = c["layers"], c["experts_per_layer"], c["k"], c["H"], c["I"], c["capacity"]
+    E = L * El
+    pf_n = c["prefetch"] if args.prefetch < 0 else args.prefetch
+    base = W.make_layer(W.SEED["paging48"], 2, H, I, El, k, shared=False, w_dtype="bf16")
+    nb = M.moe_expert_blob_bytes(2, H, I)
+    stride = (nb + 255) // 256 * 256
+    link = host_link_gbs()
+    pool = torch.empty(E * stride, dtype=torch.uint8, pin_memory=True)
+    pv = pool.view(E, stride)
+    bt = torch.from_numpy(base.blobs)
+    for l in range(L):                                   # every layer's blobs (bytes moved are what matter here)
+        pv[l * El:(l + 1) * El, :nb].copy_(bt)
+    slab = torch.empty(cap * stride, dtype=torch.uint8, device="cuda")
+    table = torch.zeros(E, dtype=torch.int64, device="cuda")
+    stack = PagedExpertStack(L, El, 2, H, I, k, pool, slab, table, cap, nb, stride, decay_period=256,
+                             prefetch=pf_n)
+    tokens_w, tokens_t = max(1, args.warmup // 3), min(args.steps, c["tokens"])
+    n_tok = tokens_w + tokens_t + 16
+    trace = np.stack(list(W.paging48_trace(W.SEED["paging48"] + 17 * rank, L, El, n_tok, s=c["zipf_s"],
+                                           drift_every=c["drift_every"], drift_prob=c["drift_prob"],
+                                           hot=c["hot_per_layer"])))
+    logits = torch.from_numpy(trace).cuda()
+    x_host = W.make_tokens(W.SEED["paging48"] + 1, n_tok, H, "bf16")
+    xs = torch.from_numpy(x_host.view(np.int16)).view(torch.bfloat16).cuda()
+
+    def token(t, x=None):
+        for l in range(L):
+            y = stack.layer_step(l, xs[t:t + 1] if x is None else x, M.MOE_BF16, logits[t, l])
+        return y
+
+    for t in range(tokens_w):
+        token(t)
+    torch.cuda.synchronize()
+    st0 = stack.cache.stats()
+    stack.record, stack.events = True, []
+    n0 = M.moe_kernel_launches()
+    clocks = ClockSampler(torch.cuda.current_device())
+    barrier(world)
+    a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for t in range(tokens_w, tokens_w + tokens_t):
+        token(t)
+    z.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    stack.record = False
+    launches = M.moe_kernel_launches() - n0
+    assert M.moe_device_error() == 0
+    ms = max_over_ranks(a.elapsed_time(z), world)
+    st1 = stack.cache.stats()
+    staged = st1["bytes_staged"] - st0["bytes_staged"]
+    misses = st1["misses"] - st0["misses"]
+    prefetched = st1["prefetched"] - st0["prefetched"]
+    # prefetched experts that a later stage found resident before they were evicted
+    pending, useful = set(), 0
+    for gids, hit, _, victim, pf, pf_slot, pf_victim in stack.events:
+        for e, h in zip(gids.tolist(), hit.tolist()):
+            if h and e in pending:
+                useful += 1
+                pending.discard(e)
+        pending.difference_update(v for v in victim.tolist() if v >= 0)
+        pending.difference_update(v for v in pf_victim.tolist() if v >= 0)
+        pending.update(e for e, sl in zip(pf.tolist(), pf_slot.tolist()) if sl >= 0)
+    value = sum_over_ranks(tokens_t, world) / (ms / 1e3)
+    link_ach = staged / (ms / 1e3) / 1e9
+    roof = {"bound": "host_link", "achieved": round(link_ach, 2), "peak": round(link, 2), "unit": "GB/s",
+            "frac": round(link_ach / link, 4), "traffic": None,
+            "kernel": "expcache_stage + expcache_prefetch copies (cudaMemcpyAsync pinned host -> HBM slot)",
+            "peak_source": "pinned 1 GiB host->device copy measured in this run",
+            "misses_per_token": round(misses / tokens_t, 2),
+            "prefetched_per_token": round(prefetched / tokens_t, 2),
+            "prefetched_used_share": round(useful / prefetched, 4) if prefetched else None,
+            "expert_accesses_per_token": L * k, "hbm_bytes_per_token": L * k * nb}
+
+    e2e = None
+    if not args.no_e2e:
+        n_e2e = min(tokens_t, 16)
+        xh = torch.from_numpy(x_host.view(np.int16)).view(torch.bfloat16).pin_memory()
+        yh = torch.empty(H, dtype=torch.float32).pin_memory()
+        xd = torch.empty(1, H, dtype=torch.bfloat16, device="cuda")
+        s = torch.cuda.current_stream()
+        barrier(world)
+        a.record()
+        for j in range(n_e2e):
+            t = tokens_w + tokens_t + (j % 16)
+            xd.copy_(xh[t:t + 1], non_blocking=True)
+            y = token(t, xd)
+            yh.copy_(y[:H], non_blocking=True)
+            s.synchronize()
+        z.record()
+        torch.cuda.synchronize()
+        e_ms = max_over_ranks(a.elapsed_time(z), world)
+        e2e = {"value": round(sum_over_ranks(n_e2e, world) / (e_ms / 1e3), 2), "unit": "tokens/s",
+               "h2d_bytes_per_step": H * 2, "d2h_bytes_per_step": H * 4 + L * k * 4, "steps": n_e2e,
+               "note": "one token through 48 layers per step; x copied in from page-locked host memory, the last "
+                       "layer's y read back"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        oracle.set_threads(host_cores())
+        blob_list = [pv[e % El, :nb].numpy() for e in range(El)]
+        t0, n = time.perf_counter(), 0
+        while time.perf_counter() - t0 < args.cpu_seconds or n < L:
+            t, l = (n // L) % n_tok, n % L
+            oracle.moe_layer(2, x_host[t:t + 1], "bf16", blob_list, k=k, H=H, I=I, E=El, logits_in=trace[t, l][None])
+            n += 1
+        dt = time.perf_counter() - t0
+        cpu = {"value": round(n / L / dt, 4), "unit": "tokens/s", "cores": host_cores(), "kind": "oracle",
+               "sample": f"{n} layer steps ({n / L:.1f} tokens of 48 layers) through the fp64 oracle, {dt:.1f} s"}
+    stack.close()
+    cfg = paging48_config(L, El, k, nb, cap, c, pf_n, world)
+    return dict(value=value, ms=ms, steps=tokens_t, roofline=roof, e2e=e2e, cpu=cpu, clocks=clk,
+                launches=launches, config=cfg, dtype="fp32 (CUDA-core FMA on 2-bit codes)")
+
+
+def paging48_config(L, El, k, nb, cap, c, pf_n, world):
+    """The `config` object of the model-scale paging workload (both arms print it)."""
+    return {"workload": f"paging48: {L} layers x {El} experts (2-bit, {nb} B each, {L * El * nb / 1e9:.1f} GB pinned "
+                        f"host), {cap} HBM slots, top-{k} per layer, Zipf s={c['zipf_s']} per layer with drift every "
+                        f"{c['drift_every']} tokens, prefetch of the next layer's {pf_n} most used experts",
+            "tokens_per_step": 1, "layers_per_token": L, "l2": "weights paged from host; HBM slots 2 GB > L2",
+            "parallelism": f"replicas x{world}"}
+
+
 def expert_stats(ids_per_step, hot=42):
     """Routing of some steps (one int array of selected ids per step): mean
     distinct experts per step and the share of selections that fall on the
@@ -755,6 +890,29 @@ def bench_reference(args, world, rank):
     oracle.set_threads(host_cores())
     kind = args.workload
     n = args.warmup + args.steps
+    if kind == "paging48":
+        c = W.PAGING48
+        L, El, k, H, I, cap = c["layers"], c["experts_per_layer"], c["k"], c["H"], c["I"], c["capacity"]
+        base = W.make_layer(W.SEED["paging48"], 2, H, I, El, k, shared=False, w_dtype="bf16")
+        n_tok = n // L + 2
+        trace = np.stack(list(W.paging48_trace(W.SEED["paging48"], L, El, n_tok, s=c["zipf_s"],
+                                               drift_every=c["drift_every"], drift_prob=c["drift_prob"],
+                                               hot=c["hot_per_layer"])))
+        x = W.make_tokens(W.SEED["paging48"] + 1, n_tok, H, "bf16")
+
+        def one(i):
+            t, l = i // L, i % L
+            oracle.moe_layer(2, x[t:t + 1], "bf16", base.blobs, k=k, H=H, I=I, E=El, logits_in=trace[t, l][None])
+        pf_n = c["prefetch"] if getattr(args, "prefetch", -1) < 0 else args.prefetch
+        cfg = paging48_config(L, El, k, oracle.blob_bytes(2, H, I), cap, c, pf_n, world)
+        sample = "1 layer step of a token (10 of 512 experts of one of 48 layers); tokens/s = steps / 48 / time"
+        for i in range(args.warmup):
+            one(i)
+        t0 = time.perf_counter()
+        for i in range(args.warmup, n):
+            one(i)
+        dt = time.perf_counter() - t0
+        return dict(value=args.steps / L / dt, ms=dt * 1e3, config=cfg, sample=sample)
     if kind == "paging":
         c = W.PAGING
         E, k, H, I, cap = c["E"], c["k"], c["H"], c["I"], c["capacity"]
@@ -796,7 +954,8 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--workload", default="decode", choices=["decode", "verify", "prefill", "paging"])
+    ap.add_argument("--workload", default="decode", choices=["decode", "verify", "prefill", "paging", "paging48"])
+    ap.add_argument("--prefetch", type=int, default=-1, help="paging48: experts prefetched per layer (-1: config)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--window", type=int, default=16)
     ap.add_argument("--chunk", type=int, default=8192)
@@ -836,6 +995,8 @@ def main():
     world, rank, local = dist_setup(args.gpus)
     if args.workload == "paging":
         r = bench_paging(args, world, rank, pk)
+    elif args.workload == "paging48":
+        r = bench_paging48(args, world, rank, pk)
     else:
         r = bench_layer(args, world, rank, pk)
     if rank == 0:

@@ -302,6 +302,7 @@ typedef struct {
 typedef struct {
     int64_t steps, hits, misses, evictions, bytes_staged;
     int32_t resident;
+    int64_t prefetched;     /* experts admitted by expcache_prefetch */
 } moe_expcache_stats;
 
 /* Creates the cache (empty).  Returns MOE_EINVAL on bad descriptors. */
@@ -313,14 +314,32 @@ int expcache_lookup(moe_expcache *c, const int32_t *ids_host, int n, int32_t *sl
 
 /* One step: policy bookkeeping for the n distinct ids (host array), then the
  * copies of the misses.  Outputs (host, optional, n entries each): hit[i]
- * 1/0, slot[i], victim[i] (-1 = none).  The compute stream's work queued so
+ * 1 = resident and usable at once, 2 = resident but admitted by
+ * expcache_prefetch since the last expcache_join (its copy may still be in
+ * flight: use it after expcache_join), 0 = miss; slot[i], victim[i] (-1 =
+ * none).  The compute stream's work queued so
  * far is ordered before any slot is overwritten.  Returns MOE_EBUSY if
  * n > capacity, MOE_EINVAL for bad or repeated ids, MOE_EIO/MOE_ECUDA if
  * issuing a copy failed (the step's bookkeeping is then rolled back). */
 int expcache_stage(moe_expcache *c, const int32_t *ids_host, int n, moe_stream_t compute,
                    int32_t *hit_out, int32_t *slot_out, int32_t *victim_out);
 
-/* Makes `s` wait (cudaStreamWaitEvent) for every copy and table update issued so far. */
+/* Loads experts expected soon (the next layer's likely experts) without a
+ * use: for each id of ids_host (-1 = none), in order, a resident id is left
+ * alone; otherwise it enters the lowest free slot, else the slot of the
+ * resident expert smallest in (counter, last use, id) that is neither one of
+ * the last expcache_stage call's ids nor on this list; if every resident
+ * expert is protected the id is skipped.  Counters and last uses do not
+ * change.  Copies and the table patch are queued like expcache_stage's (after
+ * the compute stream's queued work); expcache_join covers them.  Outputs
+ * (host, optional): slot_out[i] (-1 = not admitted), victim_out[i],
+ * *n_admitted.  MOE_EINVAL for an id outside [-1, n_experts) or n > 32. */
+int expcache_prefetch(moe_expcache *c, const int32_t *ids_host, int n, moe_stream_t compute,
+                      int32_t *slot_out, int32_t *victim_out, int *n_admitted);
+
+/* Makes `s` wait (cudaStreamWaitEvent) for every copy and table update issued
+ * so far; experts admitted by earlier prefetches count as settled from then on
+ * (expcache_stage reports them as hit 1). */
 int expcache_join(moe_expcache *c, moe_stream_t s);
 
 /* Host wait for the staged copies with a time limit; MOE_ETIMEDOUT if not done. */

@@ -46,7 +46,8 @@ class ExpCacheDesc(C.Structure):
 
 class ExpCacheStats(C.Structure):
     _fields_ = [("steps", C.c_int64), ("hits", C.c_int64), ("misses", C.c_int64),
-                ("evictions", C.c_int64), ("bytes_staged", C.c_int64), ("resident", C.c_int32)]
+                ("evictions", C.c_int64), ("bytes_staged", C.c_int64), ("resident", C.c_int32),
+                ("prefetched", C.c_int64)]
 
 
 _lib = None
@@ -94,6 +95,7 @@ def lib():
         "expcache_snapshot": (I, [P, P, P]),
         "expcache_inject_copy_failures": (I, [P, I]),
         "expcache_copy_times": (I, [P, P, C.POINTER(C.c_float), C.POINTER(C.c_float)]),
+        "expcache_prefetch": (I, [P, P, I, S, P, P, C.POINTER(C.c_int)]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -273,6 +275,17 @@ class ExpCache:
         victim = np.empty(ids.size, np.int32)
         _check(lib().expcache_stage(self.h, _p(ids), ids.size, _stream(stream), _p(hit), _p(slot), _p(victim)))
         return hit, slot, victim
+
+    def prefetch(self, ids, stream=None):
+        """Loads the given experts (-1 = none) without a use; returns (slot, victim, admitted)."""
+        import numpy as np
+        ids = np.ascontiguousarray(ids, dtype=np.int32)
+        slot = np.empty(ids.size, np.int32)
+        victim = np.empty(ids.size, np.int32)
+        adm = C.c_int(0)
+        _check(lib().expcache_prefetch(self.h, _p(ids), ids.size, _stream(stream), _p(slot), _p(victim),
+                                       C.byref(adm)))
+        return slot, victim, adm.value
 
     def join(self, stream=None):
         _check(lib().expcache_join(self.h, _stream(stream)))

@@ -12,6 +12,7 @@
 // (counter, last use, id) over the resident experts); each miss is one
 // cudaMemcpyAsync on the cache's own stream, after which one small kernel
 // patches the device table of blob pointers.
+#include <algorithm>
 #include <chrono>
 #include <cstring>
 #include <new>
@@ -55,6 +56,8 @@ struct moe_expcache {
     std::set<std::tuple<int64_t, int64_t, int32_t>> order;   // resident experts by (cnt, last, id)
     std::set<int32_t> free_slots;
     int64_t step = 0;
+    std::vector<int32_t> step_ids;                     // ids of the last stage call (protected from prefetch)
+    std::vector<uint8_t> inflight;                     // admitted by a prefetch not yet covered by a join
     moe_expcache_stats st{};
     int inject_fail = 0;
 };
@@ -87,6 +90,65 @@ static void destroy_events(moe_expcache *c) {
     if (c->ev_t0) cudaEventDestroy(c->ev_t0);
     if (c->ev_t1) cudaEventDestroy(c->ev_t1);
     if (c->copy) cudaStreamDestroy(c->copy);
+}
+
+// One copy per admitted expert on the cache's stream, after the compute
+// stream's work queued so far (it may still read the victims' slots), then
+// one table patch; copies that cannot be issued leave their experts out of
+// the cache again.
+struct PendingCopy {
+    int32_t id, slot;
+};
+
+static int issue_copies(moe_expcache *c, const PendingCopy *copies, int nc, TablePatch &patch, moe_stream_t compute) {
+    if (nc == 0 && patch.n == 0) return MOE_OK;
+    int rc = MOE_OK;
+    if (nc > 0) {
+        rc = cuda_status(cudaEventRecord(c->ev_compute, reinterpret_cast<cudaStream_t>(compute)), "event record");
+        if (!rc) rc = cuda_status(cudaStreamWaitEvent(c->copy, c->ev_compute, 0), "stream wait");
+        if (!rc) rc = cuda_status(cudaEventRecord(c->ev_t0, c->copy), "event record");
+    }
+    const size_t B = static_cast<size_t>(c->d.blob_bytes), S = static_cast<size_t>(c->d.slot_stride);
+    auto *slab = static_cast<uint8_t *>(c->d.hbm_slab);
+    auto *pool = static_cast<const uint8_t *>(c->d.host_pool);
+    int issued = 0;
+    for (int i = 0; i < nc && !rc; ++i) {
+        uint8_t *dst = slab + static_cast<size_t>(copies[i].slot) * S;
+        const uint8_t *src = pool + static_cast<size_t>(copies[i].id) * S;
+        if (c->d.use_staging) {
+            const int h = c->stage_next;
+            c->stage_next ^= 1;
+            rc = cuda_status(cudaEventSynchronize(c->ev_stage[h]), "stage wait");
+            uint8_t *buf = static_cast<uint8_t *>(c->d.stage_buffer) + static_cast<size_t>(h) * S;
+            if (!rc) std::memcpy(buf, src, B);
+            if (!rc) rc = cuda_status(cudaMemcpyAsync(dst, buf, B, cudaMemcpyHostToDevice, c->copy), "stage copy");
+            if (!rc) rc = cuda_status(cudaEventRecord(c->ev_stage[h], c->copy), "event record");
+        } else {
+            rc = cuda_status(cudaMemcpyAsync(dst, src, B, cudaMemcpyHostToDevice, c->copy), "expert copy");
+        }
+        if (rc) {
+            rc = MOE_EIO;
+        } else {
+            patch.ids[patch.n] = copies[i].id;
+            patch.ptrs[patch.n] = dst;
+            patch.n++;
+            issued++;
+            c->st.bytes_staged += static_cast<int64_t>(B);
+        }
+    }
+    // copies that could not be issued leave their experts out of the cache
+    for (int i = issued; i < nc; ++i) {
+        const int e = copies[i].id;
+        c->order.erase(std::make_tuple(c->cnt[e], c->last[e], e));
+        c->expert_in[copies[i].slot] = -1;
+        c->slot_of[e] = -1;
+        c->free_slots.insert(copies[i].slot);
+    }
+    int rc2 = launch_table_patch(reinterpret_cast<const void **>(c->d.dev_table), patch, c->copy);
+    if (!rc2) rc2 = cuda_status(cudaEventRecord(c->ev_done, c->copy), "event record");
+    if (!rc2 && nc > 0) rc2 = cuda_status(cudaEventRecord(c->ev_t1, c->copy), "event record");
+    if (!rc2 && nc > 0) c->timed = true;
+    return rc ? rc : rc2;
 }
 
 extern "C" {
@@ -130,6 +192,7 @@ int expcache_create(const moe_expcache_desc *d, moe_expcache **out) {
     }
     try {
         c->slot_of.assign(d->n_experts, -1);
+        c->inflight.assign(d->n_experts, 0);
         c->expert_in.assign(d->capacity, -1);
         c->cnt.assign(d->n_experts, 0);
         c->last.assign(d->n_experts, -1);
@@ -197,8 +260,7 @@ int expcache_stage(moe_expcache *c, const int32_t *ids_host, int n, moe_stream_t
             if (c->slot_of[e] >= 0) c->order.emplace(c->cnt[e], c->last[e], e);
     }
     TablePatch patch{};
-    struct Copy { int32_t id, slot; };
-    Copy copies[32];
+    PendingCopy copies[32];
     int nc = 0;
     for (int i = 0; i < n; ++i) {
         const int e = ids_host[i];
@@ -227,6 +289,7 @@ int expcache_stage(moe_expcache *c, const int32_t *ids_host, int n, moe_stream_t
                 c->order.erase(it);
                 slot = c->slot_of[victim];
                 c->slot_of[victim] = -1;
+                c->inflight[victim] = 0;
                 c->st.evictions++;
                 patch.ids[patch.n] = victim;
                 patch.ptrs[patch.n] = nullptr;
@@ -235,64 +298,73 @@ int expcache_stage(moe_expcache *c, const int32_t *ids_host, int n, moe_stream_t
             c->slot_of[e] = slot;
             c->expert_in[slot] = e;
             c->order.emplace(c->cnt[e], c->last[e], e);
-            copies[nc++] = Copy{e, slot};
+            copies[nc++] = PendingCopy{e, slot};
             c->st.misses++;
         }
-        if (hit_out) hit_out[i] = resident ? 1 : 0;
+        if (hit_out) hit_out[i] = resident ? (c->inflight[e] ? 2 : 1) : 0;
         if (slot_out) slot_out[i] = c->slot_of[e];
         if (victim_out) victim_out[i] = victim;
     }
     c->step++;
     c->st.steps++;
-    if (nc == 0) return MOE_OK;
-    // copies start after the compute work queued so far (it may still read victims' slots)
-    int rc = cuda_status(cudaEventRecord(c->ev_compute, reinterpret_cast<cudaStream_t>(compute)), "event record");
-    if (!rc) rc = cuda_status(cudaStreamWaitEvent(c->copy, c->ev_compute, 0), "stream wait");
-    if (!rc) rc = cuda_status(cudaEventRecord(c->ev_t0, c->copy), "event record");
-    const size_t B = static_cast<size_t>(c->d.blob_bytes), S = static_cast<size_t>(c->d.slot_stride);
-    auto *slab = static_cast<uint8_t *>(c->d.hbm_slab);
-    auto *pool = static_cast<const uint8_t *>(c->d.host_pool);
-    for (int i = 0; i < nc && !rc; ++i) {
-        uint8_t *dst = slab + static_cast<size_t>(copies[i].slot) * S;
-        const uint8_t *src = pool + static_cast<size_t>(copies[i].id) * S;
-        if (c->d.use_staging) {
-            const int h = c->stage_next;
-            c->stage_next ^= 1;
-            rc = cuda_status(cudaEventSynchronize(c->ev_stage[h]), "stage wait");
-            uint8_t *buf = static_cast<uint8_t *>(c->d.stage_buffer) + static_cast<size_t>(h) * S;
-            if (!rc) std::memcpy(buf, src, B);
-            if (!rc) rc = cuda_status(cudaMemcpyAsync(dst, buf, B, cudaMemcpyHostToDevice, c->copy), "stage copy");
-            if (!rc) rc = cuda_status(cudaEventRecord(c->ev_stage[h], c->copy), "event record");
+    c->step_ids.assign(ids_host, ids_host + n);
+    return issue_copies(c, copies, nc, patch, compute);
+}
+
+int expcache_prefetch(moe_expcache *c, const int32_t *ids_host, int n, moe_stream_t compute, int32_t *slot_out,
+                      int32_t *victim_out, int *n_admitted) {
+    moe::NvtxRange nvtx_range("expcache_prefetch");
+    REQUIRE(c && (n == 0 || ids_host), "cache/ids are NULL");
+    REQUIRE(n >= 0 && n <= 32, "n must be in [0, 32]");
+    for (int i = 0; i < n; ++i)
+        REQUIRE(ids_host[i] >= -1 && ids_host[i] < c->d.n_experts, "expert id %d out of range", ids_host[i]);
+    DeviceGuard guard(c->device);
+    // protected: the last step's ids and every id on this list
+    auto protected_id = [&](int v) {
+        for (int32_t q : c->step_ids)
+            if (q == v) return true;
+        for (int i = 0; i < n; ++i)
+            if (ids_host[i] == v) return true;
+        return false;
+    };
+    TablePatch patch{};
+    PendingCopy copies[32];
+    int nc = 0;
+    for (int i = 0; i < n; ++i) {
+        const int e = ids_host[i];
+        if (slot_out) slot_out[i] = -1;
+        if (victim_out) victim_out[i] = -1;
+        if (e < 0 || c->slot_of[e] >= 0) continue;
+        int slot = -1, victim = -1;
+        if (!c->free_slots.empty()) {
+            slot = *c->free_slots.begin();
+            c->free_slots.erase(c->free_slots.begin());
         } else {
-            rc = cuda_status(cudaMemcpyAsync(dst, src, B, cudaMemcpyHostToDevice, c->copy), "expert copy");
-        }
-        if (rc) rc = MOE_EIO;
-        else {
-            patch.ids[patch.n] = copies[i].id;
-            patch.ptrs[patch.n] = dst;
+            auto it = c->order.begin();
+            while (it != c->order.end() && protected_id(std::get<2>(*it))) ++it;
+            if (it == c->order.end()) continue;        // everything resident is protected
+            victim = std::get<2>(*it);
+            c->order.erase(it);
+            slot = c->slot_of[victim];
+            c->slot_of[victim] = -1;
+            c->inflight[victim] = 0;
+            c->st.evictions++;
+            patch.ids[patch.n] = victim;
+            patch.ptrs[patch.n] = nullptr;
             patch.n++;
-            c->st.bytes_staged += static_cast<int64_t>(B);
         }
+        // a prefetch is not a use: the counter and last use stay as they are
+        c->slot_of[e] = slot;
+        c->expert_in[slot] = e;
+        c->order.emplace(c->cnt[e], c->last[e], e);
+        c->inflight[e] = 1;
+        copies[nc++] = PendingCopy{e, slot};
+        if (slot_out) slot_out[i] = slot;
+        if (victim_out) victim_out[i] = victim;
     }
-    if (rc) {
-        // copies that could not be issued leave their experts out of the cache
-        for (int i = 0; i < nc; ++i) {
-            bool issued = false;
-            for (int j = 0; j < patch.n; ++j) issued |= patch.ids[j] == copies[i].id && patch.ptrs[j] != nullptr;
-            if (!issued) {
-                const int e = copies[i].id;
-                c->order.erase(std::make_tuple(c->cnt[e], c->last[e], e));
-                c->expert_in[copies[i].slot] = -1;
-                c->slot_of[e] = -1;
-                c->free_slots.insert(copies[i].slot);
-            }
-        }
-    }
-    int rc2 = launch_table_patch(reinterpret_cast<const void **>(c->d.dev_table), patch, c->copy);
-    if (!rc2) rc2 = cuda_status(cudaEventRecord(c->ev_done, c->copy), "event record");
-    if (!rc2) rc2 = cuda_status(cudaEventRecord(c->ev_t1, c->copy), "event record");
-    if (!rc2) c->timed = true;
-    return rc ? rc : rc2;
+    c->st.prefetched += nc;
+    if (n_admitted) *n_admitted = nc;
+    return issue_copies(c, copies, nc, patch, compute);
 }
 
 int expcache_copy_times(moe_expcache *c, const void *ref_event, float *start_ms, float *end_ms) {
@@ -307,7 +379,9 @@ int expcache_copy_times(moe_expcache *c, const void *ref_event, float *start_ms,
 
 int expcache_join(moe_expcache *c, moe_stream_t s) {
     REQUIRE(c != nullptr, "cache is NULL");
-    return cuda_status(cudaStreamWaitEvent(reinterpret_cast<cudaStream_t>(s), c->ev_done, 0), "stream wait");
+    const int rc = cuda_status(cudaStreamWaitEvent(reinterpret_cast<cudaStream_t>(s), c->ev_done, 0), "stream wait");
+    if (!rc) std::fill(c->inflight.begin(), c->inflight.end(), 0);   // every copy so far is ordered before `s`
+    return rc;
 }
 
 int expcache_wait(moe_expcache *c, int64_t timeout_us) {
@@ -316,7 +390,10 @@ int expcache_wait(moe_expcache *c, int64_t timeout_us) {
     const auto t0 = std::chrono::steady_clock::now();
     for (;;) {
         const cudaError_t e = cudaEventQuery(c->ev_done);
-        if (e == cudaSuccess) return MOE_OK;
+        if (e == cudaSuccess) {
+            std::fill(c->inflight.begin(), c->inflight.end(), 0);   // every copy so far has landed
+            return MOE_OK;
+        }
         if (e != cudaErrorNotReady) return cuda_status(e, "event query");
         const auto us =
             std::chrono::duration_cast<std::chrono::microseconds>(std::chrono::steady_clock::now() - t0).count();
@@ -339,6 +416,7 @@ int expcache_evict(moe_expcache *c, const int32_t *ids_host, int n) {
         if (s < 0) continue;
         c->order.erase(std::make_tuple(c->cnt[e], c->last[e], e));
         c->slot_of[e] = -1;
+        c->inflight[e] = 0;
         c->expert_in[s] = -1;
         c->free_slots.insert(s);
         c->st.evictions++;

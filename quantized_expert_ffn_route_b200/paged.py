@@ -1,0 +1,99 @@
+"""Model-scale expert paging: L layers of E_l experts each, all drawn from one
+pool of L * E_l expert blobs in page-locked host memory, served through one
+expert cache (HBM slots).  Expert e of layer l is pool entry l * E_l + e.
+
+Per layer of a token (Strata article, section 2 item 2: resident experts are
+computed at once, only the others must first be moved in):
+  route over the layer's E_l experts -> the selected ids cross to the host ->
+  expcache_stage -> the FFN of the resident (hit) experts, overlapping the
+  miss copies -> expcache_join -> expcache_prefetch of the next layer's most
+  frequently used experts (their copies overlap this layer's remaining work
+  and the next layer's routing) -> the FFN of the missed experts -> combine.
+
+Everything here is host-side orchestration and argument marshalling; every
+arithmetic step runs in libmoe's kernels.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+
+class PagedExpertStack:
+    """L layers x E_l experts of one blob format behind one expert cache.
+
+    pool: page-locked host tensor [L * E_l * stride] uint8; slab: device
+    [capacity * stride]; table: device int64 [L * E_l] (the cache's table);
+    the compute of layer l reads table[l * E_l : (l + 1) * E_l].
+    prefetch: experts of the next layer to prefetch per layer (0 = none),
+    chosen by the number of times each expert was selected so far (ties: the
+    lower id).
+    """
+
+    def __init__(self, layers, experts_per_layer, bits, H, I, k, pool, slab, table, capacity, blob_bytes, stride,
+                 decay_period=256, prefetch=10, device="cuda"):
+        import torch
+        from . import MOE_MODE_GEMV, ExpCache, alloc_step_buffers
+        self.L, self.El, self.bits, self.H, self.I, self.k = layers, experts_per_layer, bits, H, I, k
+        self.prefetch_n = prefetch
+        self.pool, self.slab, self.table = pool, slab, table
+        self.cache = ExpCache(layers * experts_per_layer, capacity, blob_bytes, stride, pool, slab, table,
+                              decay_period)
+        self.dev = torch.device(device)
+        self.b = alloc_step_buffers(1, H, I, experts_per_layer, k, bits, MOE_MODE_GEMV, self.dev, False)
+        self.ids_h = torch.empty(k, dtype=torch.int32).pin_memory()
+        self.act_h = torch.zeros(64, dtype=torch.int32).pin_memory()
+        self.act_d = torch.zeros(64, dtype=torch.int32, device=self.dev)
+        self.freq = np.zeros(layers * experts_per_layer, np.int64)
+        self.events = []          # per layer step: (global ids, hit, slot, victim, pf ids, pf slot, pf victim)
+        self.record = False
+
+    def close(self):
+        self.cache.close()
+
+    def predict(self, layer):
+        """The next layer's prefetch list: its most often selected experts."""
+        if self.prefetch_n <= 0:
+            return np.full(max(1, self.prefetch_n), -1, np.int32)
+        f = self.freq[layer * self.El:(layer + 1) * self.El]
+        order = np.lexsort((np.arange(self.El), -f))[:self.prefetch_n]
+        return (order + layer * self.El).astype(np.int32)
+
+    def layer_step(self, layer, x, x_dtype, logits, y_out=None, stream=None):
+        """One token through one layer: logits [E_l] fp32 device, x [H] device;
+        returns the output buffer (fp32 [H])."""
+        import torch
+        from . import moe_combine, moe_expert_ffn_q2, moe_expert_ffn_q4, moe_permute, moe_route_topk
+        b, k, El, H, I = self.b, self.k, self.El, self.H, self.I
+        s = torch.cuda.current_stream() if stream is None else stream
+        moe_route_topk(None, 0, None, 0, logits, None, 1, H, El, k, b.ids, b.w, stream=s)
+        moe_permute(b.ids, 1, k, El, b.offsets, b.perm_src, b.perm_dst, b.active, b.ws_perm, b.sizes["perm"],
+                    stream=s)
+        self.ids_h.copy_(b.ids[:k], non_blocking=True)
+        s.synchronize()                                   # the ids cross to the host
+        local = self.ids_h.numpy().copy()
+        gids = (local + layer * El).astype(np.int32)
+        hit, slot, victim = self.cache.stage(gids, stream=s)
+        np.add.at(self.freq, gids, 1)
+        # hit 1: resident and settled, computed at once; hit 2 (admitted by a
+        # prefetch whose copy may still be in flight) and misses after the join
+        hits, miss = np.sort(local[hit == 1]), np.sort(local[hit != 1])
+        a = self.act_h.numpy()
+        a[0], a[1:1 + hits.size] = hits.size, hits
+        a[32], a[33:33 + miss.size] = miss.size, miss
+        self.act_d.copy_(self.act_h, non_blocking=True)
+        ffn = moe_expert_ffn_q4 if self.bits == 4 else moe_expert_ffn_q2
+        tview = self.table[layer * El:(layer + 1) * El]
+        if hits.size:                                     # resident experts: at once, overlapping the copies
+            ffn(tview, b.offsets, self.act_d[0:], b.perm_src, x, x_dtype, 1, k, H, I, El, None, b.y_perm, None,
+                1, b.ws_ffn, b.sizes["ffn"], stream=s)
+        self.cache.join(stream=s)                         # the misses' and the prefetched experts' copies
+        pf = self.predict((layer + 1) % self.L)            # the next layer (of this or the next token)
+        pf_slot, pf_victim, _ = self.cache.prefetch(pf, stream=s)
+        if miss.size:
+            ffn(tview, b.offsets, self.act_d[32:], b.perm_src, x, x_dtype, 1, k, H, I, El, None, b.y_perm, None,
+                1, b.ws_ffn, b.sizes["ffn"], stream=s)
+        y = b.y if y_out is None else y_out
+        moe_combine(b.y_perm, b.perm_dst, b.w, None, 1, k, H, y, stream=s)
+        if self.record:
+            self.events.append((gids, hit, slot, victim, pf, pf_slot, pf_victim))
+        return y

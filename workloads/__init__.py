@@ -203,7 +203,12 @@ PAGING = dict(bits=2, H=2048, I=512, E=24576, k=10, capacity=2048, steps=5000,
               drift_every=200, drift_prob=0.1, hot=2048, zipf_s=1.1, shared=False,
               x_dtype="bf16", sigma_w=0.02)
 
-SEED = {"tiny": 1001, "decode": 1002, "verify": 1003, "prefill": 1004, "paging": 1005}
+# Model-scale paging: 48 layers x 512 experts = the 24,576-expert pool, 10
+# experts per layer per token (480 accesses per token), one HBM cache.
+PAGING48 = dict(bits=2, H=2048, I=512, layers=48, experts_per_layer=512, k=10, capacity=2048, tokens=100,
+                drift_every=50, drift_prob=0.1, hot_per_layer=42, zipf_s=1.1, prefetch=10)
+
+SEED = {"tiny": 1001, "decode": 1002, "verify": 1003, "prefill": 1004, "paging": 1005, "paging48": 1006}
 
 
 def tiny_case(seed: int = SEED["tiny"], **over):
@@ -244,4 +249,29 @@ def paging_trace(seed: int, E: int, k: int, steps: int, *, s: float = 1.1,
                     order[r], order[c] = order[c], order[r]
         lnp[order] = lnp_rank
         g = rng.gumbel(size=E)
+        yield (lnp + g).astype(np.float32)
+
+
+def paging48_trace(seed: int, layers: int, experts: int, tokens: int, *, s: float = 1.1, drift_every: int = 50,
+                   drift_prob: float = 0.1, hot: int = 42):
+    """Per-token router logits of every layer, [layers, experts] float32 per
+    token: ln p + G with G standard Gumbel, p a Zipf(s) popularity over a
+    seeded rank order of each layer's experts.  Every `drift_every` tokens
+    each of a layer's `hot` most popular ranks swaps its expert with a
+    uniformly drawn colder one with probability `drift_prob`."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    order = np.stack([rng.permutation(experts) for _ in range(layers)])
+    p = (np.arange(1, experts + 1, dtype=np.float64)) ** (-s)
+    lnp_rank = np.log(p / p.sum())
+    lnp = np.empty((layers, experts))
+    for t in range(tokens):
+        if t % drift_every == 0 and t > 0:
+            for l in range(layers):
+                for r in range(hot):
+                    if rng.random() < drift_prob:
+                        c = int(rng.integers(hot, experts))
+                        order[l, r], order[l, c] = order[l, c], order[l, r]
+        for l in range(layers):
+            lnp[l, order[l]] = lnp_rank
+        g = rng.gumbel(size=(layers, experts))
         yield (lnp + g).astype(np.float32)

@@ -24,6 +24,7 @@
 #include "common.cuh"
 #include "kernels.h"
 #include "qdot.cuh"
+#include "sm100.cuh"
 #include "topk.cuh"
 
 namespace moe {
@@ -165,6 +166,19 @@ __device__ __forceinline__ void stage_x(float4 *xs, float *cs, int H, const void
     __syncthreads();
 }
 
+// This CTA's share (1 / rblocks of the rows) of a blob's down matrix, codes
+// and scales, into L2: the down kernel's loads, which may only start once the
+// whole gate/up grid is done, then come from L2 instead of HBM.
+template <int BITS>
+__device__ __forceinline__ void prefetch_down_share(const uint8_t *blob, int H, int I, int rb, int rblocks) {
+    const BlobView bv = blob_view(blob, BITS, H, I);
+    const size_t r0 = static_cast<size_t>(rb) * H / rblocks, r1 = static_cast<size_t>(rb + 1) * H / rblocks;
+    const size_t drowb = static_cast<size_t>(I) * BITS / 8, srow = static_cast<size_t>(I) / 16;
+    sm100::prefetch_l2(bv.cd + r0 * drowb, static_cast<uint32_t>((r1 - r0) * drowb));
+    const size_t s0 = (r0 * srow) & ~size_t(15), s1 = (r1 * srow) & ~size_t(15);
+    sm100::prefetch_l2(reinterpret_cast<const uint8_t *>(bv.sd) + s0, static_cast<uint32_t>(s1 - s0));
+}
+
 // ----------------------------------------------------------- 2. gate/up
 // Block = 8 warps x 2 row pairs = 16 rows of one group; grid = groups x I/16.
 // The last group (when present) is the shared expert.  Each lane keeps the
@@ -211,10 +225,13 @@ __global__ void __launch_bounds__(kDecThreads, 3) k_dec_gateup(DecodeArgs a) {
     stage_x<BITS>(xs, cs, H, a.x, a.x_bf16);
     if (shared_group) {
         load_codes(a.shared);                            // independent of the routing
+        if (threadIdx.x == 0) prefetch_down_share<BITS>(a.shared, H, I, blockIdx.x - g * rblocks, rblocks);
     } else {
         pdl_wait();                                      // the logits are final from here on
         __shared__ uint64_t cand[kDecWarps * 32], sel[32];
-        block_topk<kDecWarps>(a.logits_in ? a.logits_in : a.ws.logits, a.E, k, cand, sel);
+        const float *lg = a.logits_in ? a.logits_in : a.ws.logits;
+        if (k <= 16 && a.E <= 64 * kDecWarps) block_topk_tree2<kDecWarps>(lg, a.E, k, cand, sel);
+        else block_topk<kDecWarps>(lg, a.E, k, cand, sel);
         if (blockIdx.x == 0 && warp == 0) {              // one CTA publishes ids and gates
             const uint64_t key = lane < k ? sel[lane] : 0ull;
             const float my_v = key_float(static_cast<uint32_t>(key >> 32));
@@ -241,6 +258,7 @@ __global__ void __launch_bounds__(kDecThreads, 3) k_dec_gateup(DecodeArgs a) {
             return;                                      // uniform over the CTA; no barrier follows
         }
         load_codes(blob);
+        if (threadIdx.x == 0) prefetch_down_share<BITS>(blob, H, I, blockIdx.x - g * rblocks, rblocks);
     }
     float dot[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll

@@ -77,6 +77,12 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t
                  : "memory");
 }
 
+// Hint: bring `bytes` (a multiple of 16, 16-byte aligned start) of global
+// memory into L2 ahead of use.
+__device__ __forceinline__ void prefetch_l2(const void *src, uint32_t bytes) {
+    if (bytes) asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 // ------------------------------------------------- gpu-scope sync words
 __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned *p) {
     unsigned v;

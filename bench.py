@@ -261,19 +261,42 @@ def gpu_copies(layer, n):
     return [base] + [base.clone() for _ in range(n - 1)]
 
 
-def cpu_baseline(layer, tokens, seconds, T_batch=8):
-    """The oracle, as it stands, on a bounded sample: token batches until `seconds` pass."""
+def timed_oracle(step, seconds, min_n):
+    """Calls step(i) for i = 0, 1, ... until `seconds` have passed and at least
+    min_n calls have run; returns (calls, seconds)."""
+    t0, n = time.perf_counter(), 0
+    while time.perf_counter() - t0 < seconds or n < min_n:
+        step(n)
+        n += 1
+    return n, time.perf_counter() - t0
+
+
+def oracle_baseline(step, seconds, min_n, tokens_per_call, what):
+    """The oracle, as it stands, on a bounded sample: on all host cores, then
+    on one thread (a shorter sample), each as tokens/s."""
     import oracle
-    n, t0 = 0, time.perf_counter()
-    while True:
-        i = (n // T_batch) % max(1, tokens.shape[0] // T_batch)
-        x = tokens[i * T_batch:(i + 1) * T_batch]
-        oracle.moe_layer(layer.bits, x, "bf16", layer.blobs, k=layer.k, H=layer.H, I=layer.I, E=layer.E,
-                         w_router=layer.w_router, w_dtype="bf16", bias=layer.bias, shared_blob=layer.shared)
-        n += x.shape[0]
-        dt = time.perf_counter() - t0
-        if dt >= seconds and n >= T_batch:
-            return n, dt
+    cores = host_cores()
+    oracle.set_threads(cores)
+    n, dt = timed_oracle(step, seconds, min_n)
+    oracle.set_threads(1)
+    n1, dt1 = timed_oracle(step, max(2.0, seconds / 3), min_n)
+    oracle.set_threads(cores)
+    return {"value": round(n * tokens_per_call / dt, 4), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{n} {what} through the fp64 oracle on {cores} threads, {dt:.1f} s",
+            "one_thread": {"value": round(n1 * tokens_per_call / dt1, 4), "unit": "tokens/s", "cores": 1,
+                           "sample": f"{n1} {what} on 1 thread, {dt1:.1f} s"}}
+
+
+def layer_oracle_step(layer, tokens, T_batch=8):
+    """One call of the oracle's layer on the next batch of T_batch tokens."""
+    import oracle
+
+    def step(n):
+        i = n % max(1, tokens.shape[0] // T_batch)
+        oracle.moe_layer(layer.bits, tokens[i * T_batch:(i + 1) * T_batch], "bf16", layer.blobs, k=layer.k,
+                         H=layer.H, I=layer.I, E=layer.E, w_router=layer.w_router, w_dtype="bf16", bias=layer.bias,
+                         shared_blob=layer.shared)
+    return step
 
 
 def run_graph_steps(step_fn, first, count, time_ffn=True):
@@ -486,11 +509,8 @@ def bench_layer(args, world, rank, pk):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        import oracle
-        oracle.set_threads(host_cores())
-        ntok, dt = cpu_baseline(layer, x_host, args.cpu_seconds, T_batch=8)
-        cpu = {"value": round(ntok / dt, 3), "unit": "tokens/s", "cores": host_cores(), "kind": "oracle",
-               "sample": f"{ntok} tokens of the {kind} workload through the fp64 oracle in batches of 8, {dt:.1f} s"}
+        cpu = oracle_baseline(layer_oracle_step(layer, x_host, 8), args.cpu_seconds, 1, 8,
+                              f"batches of 8 tokens of the {kind} workload")
 
     cfg = layer_config(kind, H, E, k, I, bits, T, n_layers, blob, mode, fused, world)
     return dict(value=value, ms=ms_max, steps=args.steps, roofline=roof, e2e=e2e, cpu=cpu, clocks=clk,
@@ -670,17 +690,12 @@ def bench_paging(args, world, rank, pk):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
-        oracle.set_threads(host_cores())
         blob_list = [pv[e, :nb].numpy() for e in range(E)]
-        t0, n = time.perf_counter(), 0
-        while time.perf_counter() - t0 < args.cpu_seconds or n < 2:
+
+        def step(n):
             i = n % n_steps
-            oracle.moe_layer(2, x_host[i:i + 1], "bf16", blob_list, k=k, H=H, I=I, E=E,
-                             logits_in=trace[i:i + 1])
-            n += 1
-        dt = time.perf_counter() - t0
-        cpu = {"value": round(n / dt, 3), "unit": "tokens/s", "cores": host_cores(), "kind": "oracle",
-               "sample": f"{n} paging steps (1 token, 10 of 24,576 experts) through the fp64 oracle, {dt:.1f} s"}
+            oracle.moe_layer(2, x_host[i:i + 1], "bf16", blob_list, k=k, H=H, I=I, E=E, logits_in=trace[i:i + 1])
+        cpu = oracle_baseline(step, args.cpu_seconds, 2, 1, "paging steps (1 token, 10 of 24,576 experts)")
     cache.close()
     cfg = paging_config(E, k, nb, cap, c, world)
     roof["cache"] = {"misses": st1["misses"] - st0["misses"], "hits": st1["hits"] - st0["hits"]}
@@ -798,16 +813,12 @@ def bench_paging48(args, world, rank, pk):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
-        oracle.set_threads(host_cores())
         blob_list = [pv[e % El, :nb].numpy() for e in range(El)]
-        t0, n = time.perf_counter(), 0
-        while time.perf_counter() - t0 < args.cpu_seconds or n < L:
+
+        def step(n):
             t, l = (n // L) % n_tok, n % L
             oracle.moe_layer(2, x_host[t:t + 1], "bf16", blob_list, k=k, H=H, I=I, E=El, logits_in=trace[t, l][None])
-            n += 1
-        dt = time.perf_counter() - t0
-        cpu = {"value": round(n / L / dt, 4), "unit": "tokens/s", "cores": host_cores(), "kind": "oracle",
-               "sample": f"{n} layer steps ({n / L:.1f} tokens of 48 layers) through the fp64 oracle, {dt:.1f} s"}
+        cpu = oracle_baseline(step, args.cpu_seconds, L, 1.0 / L, "layer steps (1 token through 1 of 48 layers)")
     stack.close()
     cfg = paging48_config(L, El, k, nb, cap, c, pf_n, world)
     return dict(value=value, ms=ms, steps=tokens_t, roofline=roof, e2e=e2e, cpu=cpu, clocks=clk,

@@ -66,6 +66,8 @@ def lib():
         _lib.oracle_cache_sim.argtypes = [I32, I32, I32, I32, I32, P, P, P, P, P]
         _lib.oracle_cache_sim_prefetch.restype = C.c_long
         _lib.oracle_cache_sim_prefetch.argtypes = [I32, I32, I32, I32, I32, P, I32, P, P, P, P, P, P, P, P]
+        _lib.oracle_set_threads.argtypes = [I32]
+        _lib.oracle_max_threads.restype = I32
     return _lib
 
 
@@ -78,8 +80,14 @@ def _c(a, dtype):
 
 
 def set_threads(n: int) -> None:
-    """OpenMP thread count for later calls (must be set before the first parallel region)."""
+    """OpenMP thread count for the oracle's later calls."""
     os.environ["OMP_NUM_THREADS"] = str(n)
+    lib().oracle_set_threads(int(n))
+
+
+def max_threads() -> int:
+    """The thread count the oracle's parallel loops use now."""
+    return int(lib().oracle_max_threads())
 
 
 # ------------------------------------------------------------------ formats

@@ -28,6 +28,7 @@
  * repository; each is marked "reading" below.
  */
 #include <math.h>
+#include <omp.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
@@ -35,6 +36,21 @@
 #define ORACLE_BLOCK 32
 
 enum { OR_F32 = 0, OR_BF16 = 1 };
+
+/* ------------------------------------------------------------- threading */
+
+/* OpenMP threads for the parallel loops that follow (n > 0); the arithmetic
+ * of every function is the same at any thread count. */
+void oracle_set_threads(int n)
+{
+    if (n > 0)
+        omp_set_num_threads(n);
+}
+
+int oracle_max_threads(void)
+{
+    return omp_get_max_threads();
+}
 
 /* ---------------------------------------------------------------- formats */
 

@@ -8,21 +8,22 @@
 // h -> down weights.  The kernel keeps that chain to two round trips of data
 // plus two grid barriers:
 //
-//   A  every CTA loads its share of the router rows (one warp per row) and
-//      copies its share of the shared expert's rows -- they do not depend on
-//      the routing -- then computes its router logits (x in registers) and
-//      publishes them;                                        grid barrier 1
-//   B  every CTA selects the top-k from the E logits itself (a two-stage
-//      warp tournament), looks the k blobs up in a copy of the expert table
-//      staged in shared memory, and issues copies of ALL its remaining
+//   A  every CTA stages x in shared memory (in natural order for the router
+//      and as the pieces the dequantising dot products read), issues bulk
+//      copies (cp.async.bulk, completion counted on an mbarrier) of its share
+//      of the shared expert's rows -- they do not depend on the routing --
+//      then computes its share of the router logits, eight warps per router
+//      row, each over one eighth of H, the eight partial sums added in a
+//      fixed order, and publishes them;                     grid barrier 1
+//   B  every CTA selects the top-k from the E logits itself (a merge tree:
+//      each warp sorts 32 keys with a bitonic network, sorted lists of 16
+//      merge pairwise), looks the k blobs up in a copy of the expert table
+//      staged in shared memory, and issues bulk copies of ALL its remaining
 //      weights at once: its slice of the routed gate/up rows (in chunks of 8
-//      rows, one mbarrier each) and its output rows of every routed down
-//      matrix.  Each CTA's share is ~130 KB, so the whole ~19.5 MB of expert
-//      weights is in flight together.  The copies are 16-byte cp.async spread
-//      over all warps (one warp per row span), each chunk's completion
-//      tracked by cp.async.mbarrier.arrive: a single thread issuing bulk
-//      copies serialises their issue, which costs microseconds at this
-//      copy count;
+//      rows, one mbarrier each, each chunk's copies issued by lane 0 of its
+//      own warp so that issue is spread over the CTA) and its output rows of
+//      every routed down matrix.  Each CTA's share is ~130 KB, so the whole
+//      ~19.5 MB of expert weights is in flight together;
 //   C  each warp takes gate/up units (one row of W_g and W_u of one group) as
 //      their chunk lands: h = silu(W_g x) * (W_u x), written to the
 //      workspace;                                             grid barrier 2
@@ -30,6 +31,11 @@
 //      computes the CTA's output rows of W_d,g . h_g from the down rows that
 //      arrived during C; y[r] = sum_j w_j (W_d,e_j[r] . h_j) + W_d,shared[r] .
 //      h_s is summed in slot order (the combine).
+//
+// This path is opt-in (moe_test_hook MOE_HOOK_DECODE_ONE_KERNEL): on B200 the
+// three-kernel chain of decode.cu, whose launches overlap through
+// programmatic dependent launch, is faster, because each grid barrier here
+// costs about as much as a dependent launch and phase C runs on 1 CTA per SM.
 //
 // The grid barriers share one monotonic 64-bit arrival count in the caller's
 // workspace (zero before the first call; every call adds two arrivals per

@@ -111,3 +111,15 @@ def test_src_hash_covers_headers(tmp_path, monkeypatch):
     p = root / "quantized_expert_ffn_route_b200" / "csrc" / "qdot.cuh"
     p.write_text(p.read_text() + "\n// edit\n")
     assert bench.src_hash("decode.cu") != h0
+
+
+def test_oracle_baseline_adds_a_one_thread_run():
+    import bench
+    import oracle
+    calls = []
+    r = bench.oracle_baseline(lambda n: calls.append(oracle.max_threads()), 0.05, 3, 2, "tiny calls")
+    assert r["kind"] == "oracle" and r["cores"] == bench.host_cores() and r["value"] > 0
+    one = r["one_thread"]
+    assert one["cores"] == 1 and one["value"] > 0 and "1 thread" in one["sample"]
+    assert 1 in calls and bench.host_cores() in calls           # both runs used their thread count
+    assert oracle.max_threads() == bench.host_cores()            # restored afterwards

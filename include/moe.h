@@ -86,6 +86,16 @@ const char *moe_last_error(void);
 /* Library version (major * 10000 + minor * 100 + patch). */
 int moe_version(void);
 
+/* Build variant of the loaded library: MOE_BUILD_DEBUG set for the MOE_DEBUG
+ * build (python -m quantized_expert_ffn_route_b200.build --debug, output in
+ * _build_debug/), in which every index read from a caller's buffer before it
+ * addresses memory (permutation entries, the active-expert count, expert ids
+ * and row ranges of the tensor-core path) also sets its MOE_DEVERR_* bit when
+ * it is out of range.  Every build keeps such an index in range (it becomes 0,
+ * or the group is skipped); only the debug build reports it. */
+#define MOE_BUILD_DEBUG 1
+int moe_build_flags(void);
+
 /* Number of kernel launches this library has issued in this process (host-side
  * count; launches recorded into a CUDA graph are counted once, at capture). */
 uint64_t moe_kernel_launches(void);

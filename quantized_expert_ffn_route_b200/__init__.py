@@ -11,12 +11,16 @@ torch is used only for device memory and streams.
 from __future__ import annotations
 
 import ctypes as C
+import os
 from pathlib import Path
 
 from .layer import MoELayer, alloc_step_buffers  # noqa: F401
 
 _PKG = Path(__file__).resolve().parent
-LIB_PATH = _PKG / "_build" / "libmoe.so"
+# MOE_LIBRARY=debug loads the MOE_DEBUG build (index checks report to the
+# device error word); the default is the release build.
+LIB_PATH = _PKG / ("_build_debug" if os.environ.get("MOE_LIBRARY") == "debug" else "_build") / "libmoe.so"
+MOE_BUILD_DEBUG = 1
 HEADER = _PKG.parent / "include" / "moe.h"
 
 MOE_OK, MOE_EINVAL, MOE_ENOMEM, MOE_ECUDA, MOE_EBUSY, MOE_ETIMEDOUT, MOE_EIO, MOE_EDEVICE = range(8)
@@ -67,6 +71,7 @@ def lib():
     sig = {
         "moe_last_error": (C.c_char_p, []),
         "moe_version": (I, []),
+        "moe_build_flags": (I, []),
         "moe_test_hook": (I, [I, C.c_int64]),
         "moe_kernel_launches": (C.c_uint64, []),
         "moe_device_error": (I, [P, I, S]),

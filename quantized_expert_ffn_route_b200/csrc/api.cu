@@ -89,6 +89,14 @@ const char *moe_last_error(void) { return t_err.c_str(); }
 
 int moe_version(void) { return 100; }
 
+int moe_build_flags(void) {
+#ifdef MOE_DEBUG
+    return MOE_BUILD_DEBUG;
+#else
+    return 0;
+#endif
+}
+
 uint64_t moe_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
 
 int moe_device_error(uint32_t *bits_out, int clear, moe_stream_t s) {

@@ -36,6 +36,33 @@ __device__ __forceinline__ void report(unsigned *err, unsigned bits) {
     if (err) atomicOr(err, bits);
 }
 
+// An index read from a caller's buffer (a permutation entry, an active-expert
+// count) before it addresses memory: every build keeps it inside [0, n) --
+// out-of-range values become 0 -- and a MOE_DEBUG build also sets `bits` in
+// the device error word, so that a corrupt buffer is reported instead of
+// silently folded onto row 0.
+__device__ __forceinline__ int guard_index(int v, int n, unsigned *err, unsigned bits) {
+    const bool bad = v < 0 || v >= n;
+#ifdef MOE_DEBUG
+    if (bad) report(err, bits);
+#else
+    (void)err;
+    (void)bits;
+#endif
+    return bad ? 0 : v;
+}
+
+// The active-expert count active[0], kept inside [0, cap]; MOE_DEBUG builds
+// report a count outside it.
+__device__ __forceinline__ int guard_count(int v, int cap, unsigned *err) {
+#ifdef MOE_DEBUG
+    if (v < 0 || v > cap) report(err, MOE_DEVERR_BAD_ROW);
+#else
+    (void)err;
+#endif
+    return min(max(v, 0), cap);
+}
+
 __device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
     return __uint_as_float(static_cast<uint32_t>(b) << 16);
 }

@@ -115,7 +115,13 @@ __device__ __forceinline__ GroupInfo group_info(const GemmArgs &a, int g, int n_
         G.row0 = ok ? a.offsets[e] : 0;
         G.n = ok ? a.offsets[e + 1] - G.row0 : 0;
         G.blob = ok ? a.blobs[e] : nullptr;
-        if (G.row0 < 0 || G.n < 0 || G.row0 + G.n > a.T * a.k) G.n = 0;
+        const bool rows_ok = G.row0 >= 0 && G.n >= 0 && G.row0 + G.n <= a.T * a.k;
+#ifdef MOE_DEBUG
+        if (!ok) report(a.err, MOE_DEVERR_BAD_EXPERT);
+        else if (!rows_ok) report(a.err, MOE_DEVERR_BAD_ROW);
+        else if (!G.blob) report(a.err, MOE_DEVERR_NULL_BLOB);
+#endif
+        if (!rows_ok) G.n = 0;
     } else {
         G.row0 = -1;
         G.n = a.T;
@@ -195,7 +201,7 @@ __global__ void __launch_bounds__(gemm_threads(MAXN), 1) k_gemm(GemmArgs a, int 
     // k-steps per raw-code slot: the largest of KSMAX, 2, 1 dividing nk (a
     // slot never spans two tiles)
     const int KS = nk % Cfg::KSMAX == 0 ? Cfg::KSMAX : (nk % 2 == 0 ? 2 : 1);
-    const int n_act = min(max(a.active[0], 0), min(a.E, a.T * a.k));
+    const int n_act = guard_count(a.active[0], min(a.E, a.T * a.k), a.err);
     const int ng = min(n_act + (a.shared ? 1 : 0), kMaxGroups);
 
     if (tid == 0) {
@@ -406,7 +412,8 @@ __global__ void __launch_bounds__(gemm_threads(MAXN), 1) k_gemm(GemmArgs a, int 
                         int v = 0;
                         if (n < nvalid) {
                             if (GATEUP)
-                                v = min(max(te.row0 >= 0 ? a.perm_src[te.row0 + te.n0 + n] : te.n0 + n, 0), a.T - 1);
+                                v = te.row0 >= 0 ? guard_index(a.perm_src[te.row0 + te.n0 + n], a.T, a.err, MOE_DEVERR_BAD_ROW)
+                                                 : te.n0 + n;
                             else
                                 v = (te.row0 >= 0 ? te.row0 : a.T * a.k) + te.n0 + n;
                         }

@@ -69,7 +69,7 @@ __global__ void __launch_bounds__(kGvThreads, 2) k_gemv_gateup(const uint8_t *co
     float4 *xs = smem;
     float *cs = reinterpret_cast<float *>(smem + static_cast<size_t>(kGvNT) * (H / 4));
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int n_act = min(max(active[0], 0), min(E, T * k));   // a corrupt count cannot run past `active`
+    const int n_act = guard_count(active[0], min(E, T * k), err);   // a corrupt count cannot run past `active`
     const int n_groups = n_act + (shared_blob ? 1 : 0);
     const int row_blocks = I / kGvRows;
     const int nch = H / Q::EPC, nblk = H / 32, nsc = H / 32;
@@ -107,8 +107,7 @@ __global__ void __launch_bounds__(kGvThreads, 2) k_gemv_gateup(const uint8_t *co
                 xs, cs, nt, nt, H,
                 [=](int t) {
                     const int r = sub + t;
-                    int tok = row0 >= 0 ? perm_src[row0 + r] : r;
-                    tok = tok < 0 || tok >= T ? 0 : tok;
+                    const int tok = row0 >= 0 ? guard_index(perm_src[row0 + r], T, err, MOE_DEVERR_BAD_ROW) : r;
                     return static_cast<const void *>(static_cast<const uint8_t *>(x) + static_cast<size_t>(tok) * xrow);
                 },
                 x_bf16);
@@ -167,7 +166,7 @@ __global__ void __launch_bounds__(kGvThreads, 2) k_gemv_down(const uint8_t *cons
     float *hcs = reinterpret_cast<float *>(smem + static_cast<size_t>(kGvNT) * (IL / 4));
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int seg = lane % LPR, subr = lane / LPR;
-    const int n_act = min(max(active[0], 0), min(E, T * k));
+    const int n_act = guard_count(active[0], min(E, T * k), err);
     const int n_groups = n_act + (shared_blob ? 1 : 0);
     const int row_blocks = (H + RB - 1) / RB;
     for (int task = blockIdx.x; task < n_groups * row_blocks; task += gridDim.x) {

@@ -2,13 +2,18 @@
 that include/moe.h declares, sizes workspaces, and rejects bad arguments on
 the host before touching the device."""
 import ctypes as C
+import os
 import re
 import subprocess
+import sys
+from pathlib import Path
 
 import numpy as np
 import pytest
 
 import quantized_expert_ffn_route_b200 as M
+
+ROOT = Path(__file__).resolve().parents[1]
 
 
 def _declared():
@@ -151,3 +156,20 @@ def test_test_hooks_validate_arguments():
     assert L.moe_test_hook(M.MOE_HOOK_GEMM_SPIN, -1) == M.MOE_EINVAL
     for h in (M.MOE_HOOK_WAIT_LIMIT_NS, M.MOE_HOOK_DECODE_EXTRA_ARRIVALS, M.MOE_HOOK_GEMM_SPIN, M.MOE_HOOK_DECODE_ONE_KERNEL):
         assert L.moe_test_hook(h, 0) == M.MOE_OK
+
+
+def test_debug_build_exports_every_symbol_and_reports_its_flag():
+    """The MOE_DEBUG variant (build --debug) links the same ABI and says so."""
+    from quantized_expert_ffn_route_b200.build import build as build_lib
+    path = build_lib(debug=True)
+    assert path.parent.name == "_build_debug"
+    out = subprocess.run(["nm", "-D", "--defined-only", str(path)], capture_output=True, text=True).stdout
+    exported = set(re.findall(r" T ((?:moe|expcache)_\w+)$", out, flags=re.M))
+    assert set(_declared()) <= exported
+    code = ("import quantized_expert_ffn_route_b200 as M; "
+            "print(M.LIB_PATH.parent.name, M.lib().moe_build_flags(), M.MOE_BUILD_DEBUG)")
+    for variant, want in (("debug", "_build_debug 1 1"), ("release", "_build 0 1")):
+        env = dict(os.environ, MOE_LIBRARY=variant)
+        r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, env=env, cwd=ROOT)
+        assert r.returncode == 0, r.stderr
+        assert r.stdout.split() == want.split()

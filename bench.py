@@ -458,7 +458,7 @@ def bench_layer(args, world, rank, pk):
     if fused and one_kernel:
         roof["kernel"] = "moe_layer_decode (k_dec_step: one persistent kernel, one CTA per SM, two grid barriers)"
     elif fused:
-        roof["kernel"] = ("moe_layer_decode (k_dec_logits -> k_dec_gateup -> k_dec_down, chained by programmatic "
+        roof["kernel"] = ("moe_layer_decode (k_dec_route -> k_dec_gateup -> k_dec_down, chained by programmatic "
                           "dependent launch; one call)")
     else:
         roof["kernel"] = "moe_expert_ffn (gate/up + down kernels)"

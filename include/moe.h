@@ -214,23 +214,28 @@ int moe_expert_ffn_q2(const void *const *expert_blobs, const int32_t *expert_off
  * moe_expert_ffn_q4/q2 (GEMV mode) -> moe_combine (Strata article, section 2
  * item 2: only the experts the router picks are computed; at one token the
  * step is bound by streaming those experts' weights).
- * When H and I are multiples of 256, H <= 2048, I / (32 for 4-bit, 64 for
- * 2-bit) is 4, 8, 16 or 32 and the per-SM share of the weights fits in shared
- * memory, the step is ONE persistent kernel (one CTA per SM, launched
- * cooperatively so all CTAs are resident) with two grid-wide barriers kept in
- * the workspace; each CTA copies its share of every selected expert with the
- * bulk-copy engine as soon as the ids are known.  Other supported shapes run
- * three kernels chained with programmatic dependent launch.
+ * The step runs as three kernels chained with programmatic dependent launch:
+ * route (router logits, then the last of its CTAs selects the top-k, computes
+ * the gates and publishes the selected blob pointers), gate/up (the shared
+ * expert's CTAs start before the route kernel ends; every CTA prefetches its
+ * share of its expert's down matrix into L2) and down + combine.  With the
+ * test hook MOE_HOOK_DECODE_ONE_KERNEL set, shapes with H and I multiples of
+ * 256, H <= 2048, I / (32 for 4-bit, 64 for 2-bit) in {4, 8, 16, 32} and a
+ * per-SM share of the weights that fits in shared memory run instead as ONE
+ * persistent kernel (one CTA per SM, launched cooperatively so all CTAs are
+ * resident) with two grid-wide barriers kept in the workspace; on B200 it is
+ * the slower of the two.
  *  x [H] (x_dtype), w_router [E,H] (w_dtype) or NULL with logits_in [E];
  *  expert_blobs device [E] blob pointers (16-byte aligned; a misaligned one
  *  sets MOE_DEVERR_MISALIGNED and that expert is left out); shared_blob or
  *  NULL; topk_ids [k] int32 out, topk_w [k] fp32 out, logits_out [E] or NULL
  *  (written only when the logits are computed here), y [H] fp32 out.
  *  ws: moe_layer_decode_ws_size() bytes of scratch.  It must be zero-filled
- *  before its first use (cudaMemsetAsync once); every call leaves it ready
- *  for the next.  After a call that set MOE_DEVERR_TIMEOUT (a grid barrier or
- *  copy wait ran out, after 1 s) zero it again.  Calls sharing one ws must
- *  not overlap.
+ *  before its first use (cudaMemsetAsync once): it holds the route kernel's
+ *  ticket count and the one-kernel step's barrier count, which every call
+ *  leaves ready for the next.  After a call that set MOE_DEVERR_TIMEOUT (a
+ *  grid barrier or copy wait of the one-kernel step ran out) zero it again.
+ *  Calls sharing one ws must not overlap.
  * Supported shapes (else MOE_EINVAL: use the separate calls): E <= 1024,
  * k <= 32, H <= 2048 and a multiple of 128, I a multiple of 128 with I/32
  * (4-bit) or I/64 (2-bit) in {4, 8, 16, 32}, and the down kernel's tasks,

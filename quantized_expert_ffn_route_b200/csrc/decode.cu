@@ -2,14 +2,15 @@
 // programmatic dependent launch (each starts while its predecessor runs and
 // waits with griddepcontrol only where it reads the predecessor's results).
 //
-//   1. logits (one warp per router row, E/4 CTAs); skipped when the caller
-//      gives the logits.
+//   1. route: the logits (one warp per router row, E/4 CTAs; one CTA when
+//      the caller gives the logits), then the last CTA to finish selects the
+//      top-k, computes the gates and publishes ids, gates and the selected
+//      blob pointers.  Selecting once here rather than in every gate/up CTA
+//      keeps the selection off hundreds of CTAs' critical paths.
 //   2. gate/up (all selected experts + the shared expert, 16 rows per CTA):
-//      every routed CTA selects the top-k from the logits itself (a block
-//      top-k of well under a microsecond, cheaper than another kernel
-//      boundary or a grid-wide hand-off), then
-//      h_g[i] = silu(Wg_g[i] . x) * (Wu_g[i] . x); CTA 0 publishes ids and
-//      gates.  The shared expert's CTAs never wait for the logits.
+//      h_g[i] = silu(Wg_g[i] . x) * (Wu_g[i] . x).  The shared expert's CTAs
+//      never wait for the route kernel; every CTA prefetches its share of
+//      its expert's down rows into L2 for kernel 3.
 //   3. down + combine (a few output rows per CTA, all groups; each lane one
 //      chunk of one row): every code load is issued before h is staged, then
 //      y[r] = sum_j w_j (Wd_{e_j}[r] . h_j) + Wd_shared[r] . h_shared, summed
@@ -38,12 +39,16 @@ __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.lau
 __host__ __device__ inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
 // Workspace layout (bytes): ids [32] int32 @0 | gates [32] fp32 @128 |
-// grid-barrier arrival count (uint64) @256 (used by the one-kernel step;
-// zero before the first call) | logits [E] @512 | h [(k+1) * I] fp32
-// (256-aligned).
+// grid-barrier arrival count (uint64) @256 (used by the one-kernel step) |
+// route-CTA ticket count (uint32) @264 | selected blob pointers [32] @512 |
+// logits [E] @1024 | h [(k+1) * I] fp32 (256-aligned).  Both counts are zero
+// before the first call, and every call leaves them so.
+constexpr size_t kDecWsHeader = 1024;
 struct DecodeWs {
     int32_t *ids;
     float *gates;
+    unsigned *tickets;
+    const uint8_t **blob;
     float *logits;
     float *h;
 };
@@ -52,8 +57,10 @@ __host__ __device__ inline DecodeWs decode_ws(void *ws, int E) {
     DecodeWs w;
     w.ids = reinterpret_cast<int32_t *>(p);
     w.gates = reinterpret_cast<float *>(p + 128);
-    w.logits = reinterpret_cast<float *>(p + 512);
-    w.h = reinterpret_cast<float *>(p + 512 + ((static_cast<size_t>(E) * 4 + 255) / 256) * 256);
+    w.tickets = reinterpret_cast<unsigned *>(p + 264);
+    w.blob = reinterpret_cast<const uint8_t **>(p + 512);
+    w.logits = reinterpret_cast<float *>(p + kDecWsHeader);
+    w.h = reinterpret_cast<float *>(p + kDecWsHeader + ((static_cast<size_t>(E) * 4 + 255) / 256) * 256);
     return w;
 }
 
@@ -75,16 +82,21 @@ struct DecodeArgs {
     unsigned *err;
 };
 
-// ------------------------------------------------------------ 1. logits
+// ------------------------------------------------------------- 1. route
 // One warp per router row, kLogitRows rows per CTA, so the E rows are read by
 // E / kLogitRows SMs at once; every lane issues all of its weight loads
-// before it stages x.
-constexpr int kLogitRows = 4;
+// before it stages x.  Each CTA then takes a ticket; the CTA that takes the
+// last one sees every logit (each CTA fences its writes before its ticket)
+// and selects.
+constexpr int kLogitRows = 8;
 
-__global__ void __launch_bounds__(kLogitRows * 32) k_dec_logits(DecodeArgs a) {
+__global__ void __launch_bounds__(kLogitRows * 32) k_dec_route(DecodeArgs a) {
     __shared__ __align__(16) float xs[2048];
+    __shared__ uint64_t cand[kLogitRows * 32], sel[32];
+    __shared__ const uint8_t *tab_s[1024];
+    __shared__ int last;
     pdl_trigger();                                       // the gate/up kernel may start its prologue
-    const int H = a.H, E = a.E;
+    const int H = a.H, E = a.E, k = a.k;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     if (!a.logits_in) {
         const int e = blockIdx.x * kLogitRows + warp;
@@ -98,9 +110,21 @@ __global__ void __launch_bounds__(kLogitRows * 32) k_dec_logits(DecodeArgs a) {
                     w[j] = ldg_stream(static_cast<const __nv_bfloat16 *>(a.w_router) + static_cast<size_t>(e) * H + hh);
             }
         }
-        for (int i = threadIdx.x; i < H / 4; i += blockDim.x)
-            reinterpret_cast<float4 *>(xs)[i] = a.x_bf16 ? load4(static_cast<const __nv_bfloat16 *>(a.x) + 4 * i)
-                                                         : load4(static_cast<const float *>(a.x) + 4 * i);
+        {
+            float4 v[4];                                 // H <= 2048: at most 4 loads per thread, all in flight
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int i = threadIdx.x + u * kLogitRows * 32;
+                if (i < H / 4)
+                    v[u] = a.x_bf16 ? load4(static_cast<const __nv_bfloat16 *>(a.x) + 4 * i)
+                                    : load4(static_cast<const float *>(a.x) + 4 * i);
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int i = threadIdx.x + u * kLogitRows * 32;
+                if (i < H / 4) reinterpret_cast<float4 *>(xs)[i] = v[u];
+            }
+        }
         __syncthreads();
         if (e < E) {
             float s = 0.f;
@@ -138,6 +162,61 @@ __global__ void __launch_bounds__(kLogitRows * 32) k_dec_logits(DecodeArgs a) {
             }
         }
     }
+    __syncthreads();                                     // every row of this CTA written
+    if (threadIdx.x == 0) {                              // one fence per CTA on each side of the ticket
+        __threadfence();
+        last = atomicAdd(a.ws.tickets, 1u) == gridDim.x - 1;
+        if (last) __threadfence();
+    }
+    __syncthreads();
+    if (!last) return;
+    // the expert table (E <= 1024 pointers) is read together with the logits,
+    // so that the selected blob pointers need no further round trip
+    constexpr int kTabPerThread = 1024 / (kLogitRows * 32);
+    const uint8_t *tv[kTabPerThread];
+#pragma unroll
+    for (int u = 0; u < kTabPerThread; ++u) {
+        const int e = threadIdx.x + u * kLogitRows * 32;
+        tv[u] = e < E ? a.blobs[e] : nullptr;
+    }
+    const float *lg = a.logits_in ? a.logits_in : a.ws.logits;
+    if (k <= 16 && E <= 32 * 2 * kLogitRows) block_topk_tree_n<kLogitRows, 2>(lg, E, k, cand, sel);
+    else block_topk_merge<kLogitRows, 1024 / (32 * kLogitRows)>(lg, E, k, cand, sel);
+#pragma unroll
+    for (int u = 0; u < kTabPerThread; ++u) {
+        const int e = threadIdx.x + u * kLogitRows * 32;
+        if (e < E) tab_s[e] = tv[u];
+    }
+    __syncthreads();
+    if (warp == 0) {
+        const uint64_t key = lane < k ? sel[lane] : 0ull;
+        const float my_v = key_float(static_cast<uint32_t>(key >> 32));
+        const int my_id = static_cast<int>(0xffffffffu - static_cast<uint32_t>(key));
+        const float v0 = __shfl_sync(0xffffffffu, my_v, 0);
+        const bool bad = lane < k && (my_v != my_v || my_v == __int_as_float(0x7f800000));
+        const bool any_bad = __any_sync(0xffffffffu, bad);
+        const float ex = lane < k ? expf(my_v - v0) : 0.f;
+        float sum = 0.f;
+        for (int j = 0; j < k; ++j) sum += __shfl_sync(0xffffffffu, ex, j);   // slot order
+        if (lane < k) {
+            const float wj = any_bad ? __int_as_float(0x7fc00000) : ex / sum;
+            const bool id_ok = my_id >= 0 && my_id < E;
+            const uint8_t *b = id_ok ? tab_s[my_id] : nullptr;
+            if (!b) {
+                report(a.err, id_ok ? MOE_DEVERR_NULL_BLOB : MOE_DEVERR_BAD_EXPERT);
+            } else if (reinterpret_cast<uintptr_t>(b) & 15u) {   // 16-byte loads need an aligned blob
+                report(a.err, MOE_DEVERR_MISALIGNED);
+                b = nullptr;
+            }
+            a.ws.ids[lane] = my_id;
+            a.ws.gates[lane] = wj;
+            a.ws.blob[lane] = b;
+            a.ids_out[lane] = my_id;
+            a.w_out[lane] = wj;
+        }
+        if (lane == 0 && any_bad) report(a.err, MOE_DEVERR_NONFINITE);
+        if (lane == 0) *a.ws.tickets = 0u;               // ready for the next call
+    }
 }
 
 // x as fp32 pieces in the order the chunk loops read them (piece q of chunk
@@ -147,10 +226,21 @@ template <int BITS>
 __device__ __forceinline__ void stage_x(float4 *xs, float *cs, int H, const void *x, int bf16) {
     using Q = QT<BITS>;
     const int nch = H / Q::EPC;
-    for (int g4 = threadIdx.x; g4 < H / 4; g4 += blockDim.x) {
-        const int c = g4 / Q::PPC, q = g4 % Q::PPC;
-        xs[q * nch + c] = bf16 ? load4(static_cast<const __nv_bfloat16 *>(x) + 4 * g4)
-                               : load4(static_cast<const float *>(x) + 4 * g4);
+    constexpr int kB = 4;                                // loads of a thread in flight together
+    for (int base = threadIdx.x; base < H / 4; base += kB * blockDim.x) {
+        float4 v[kB];
+#pragma unroll
+        for (int u = 0; u < kB; ++u) {
+            const int g4 = base + u * blockDim.x;
+            if (g4 < H / 4)
+                v[u] = bf16 ? load4(static_cast<const __nv_bfloat16 *>(x) + 4 * g4)
+                            : load4(static_cast<const float *>(x) + 4 * g4);
+        }
+#pragma unroll
+        for (int u = 0; u < kB; ++u) {
+            const int g4 = base + u * blockDim.x;
+            if (g4 < H / 4) xs[(g4 % Q::PPC) * nch + g4 / Q::PPC] = v[u];
+        }
     }
     __syncthreads();
     for (int b = threadIdx.x; b < H / 32; b += blockDim.x) {
@@ -188,13 +278,17 @@ template <int BITS>
 __global__ void __launch_bounds__(kDecThreads, 3) k_dec_gateup(DecodeArgs a) {
     using Q = QT<BITS>;
     extern __shared__ __align__(16) float4 gsm[];
-    pdl_trigger();                                       // the down kernel may start (it waits for us)
     const int H = a.H, I = a.I, k = a.k;
     constexpr int RPB = kDecWarps * 2;
     const int rblocks = I / RPB;
     const int g = blockIdx.x / rblocks;
     const int i0 = (blockIdx.x - g * rblocks) * RPB;
     const bool shared_group = g == k;
+    // The down kernel is launched once every CTA here has triggered: the
+    // shared expert's CTAs trigger at once, the routed ones only after their
+    // wait on the route kernel, so that the down kernel may read the route
+    // kernel's outputs (gates, blob pointers) before its own wait on h.
+    if (shared_group) pdl_trigger();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     float4 *xs = gsm;
     float *cs = reinterpret_cast<float *>(gsm + H / 4);
@@ -227,36 +321,11 @@ __global__ void __launch_bounds__(kDecThreads, 3) k_dec_gateup(DecodeArgs a) {
         load_codes(a.shared);                            // independent of the routing
         if (threadIdx.x == 0) prefetch_down_share<BITS>(a.shared, H, I, blockIdx.x - g * rblocks, rblocks);
     } else {
-        pdl_wait();                                      // the logits are final from here on
-        __shared__ uint64_t cand[kDecWarps * 32], sel[32];
-        const float *lg = a.logits_in ? a.logits_in : a.ws.logits;
-        if (k <= 16 && a.E <= 64 * kDecWarps) block_topk_tree2<kDecWarps>(lg, a.E, k, cand, sel);
-        else block_topk<kDecWarps>(lg, a.E, k, cand, sel);
-        if (blockIdx.x == 0 && warp == 0) {              // one CTA publishes ids and gates
-            const uint64_t key = lane < k ? sel[lane] : 0ull;
-            const float my_v = key_float(static_cast<uint32_t>(key >> 32));
-            const int my_id = static_cast<int>(0xffffffffu - static_cast<uint32_t>(key));
-            const float v0 = __shfl_sync(0xffffffffu, my_v, 0);
-            const bool bad = lane < k && (my_v != my_v || my_v == __int_as_float(0x7f800000));
-            const bool any_bad = __any_sync(0xffffffffu, bad);
-            const float ex = lane < k ? expf(my_v - v0) : 0.f;
-            float sum = 0.f;
-            for (int j = 0; j < k; ++j) sum += __shfl_sync(0xffffffffu, ex, j);   // slot order
-            if (lane < k) {
-                const float wj = any_bad ? __int_as_float(0x7fc00000) : ex / sum;
-                a.ws.ids[lane] = my_id;
-                a.ws.gates[lane] = wj;
-                a.ids_out[lane] = my_id;
-                a.w_out[lane] = wj;
-            }
-            if (lane == 0 && any_bad) report(a.err, MOE_DEVERR_NONFINITE);
-        }
-        const int e = static_cast<int>(0xffffffffu - static_cast<uint32_t>(sel[g]));
-        const uint8_t *blob = (e >= 0 && e < a.E) ? a.blobs[e] : nullptr;
-        if (!blob) {
-            if (threadIdx.x == 0) report(a.err, (e >= 0 && e < a.E) ? MOE_DEVERR_NULL_BLOB : MOE_DEVERR_BAD_EXPERT);
-            return;                                      // uniform over the CTA; no barrier follows
-        }
+        pdl_wait();                                      // ids, gates and blob pointers are final from here on
+        pdl_trigger();
+        const uint8_t *blob = reinterpret_cast<const uint8_t *>(
+            __ldcg(reinterpret_cast<const unsigned long long *>(a.ws.blob) + g));
+        if (!blob) return;                               // reported by the route kernel; uniform over the CTA
         load_codes(blob);
         if (threadIdx.x == 0) prefetch_down_share<BITS>(blob, H, I, blockIdx.x - g * rblocks, rblocks);
     }
@@ -310,14 +379,14 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_dec_down(DecodeArgs a, int n
     float4 *hs = dsm;                                    // [ng][PPC][LPR] pieces
     float *hcs = reinterpret_cast<float *>(dsm + static_cast<size_t>(ng) * (IL / 4));
     float *part = hcs + static_cast<size_t>(ng) * dnsc;
-    pdl_wait();                                          // ids (route) and h (gate/up) are final
+    // The route kernel's gates and blob pointers are final already (see the
+    // gate/up kernel's trigger), so the code loads go out before the wait on h.
     if (threadIdx.x < ng) {
         const int g = threadIdx.x;
         const uint8_t *b = a.shared;
         float gw = 1.0f;
         if (g < k) {
-            const int e = __ldcg(a.ws.ids + g);
-            b = (e >= 0 && e < a.E) ? a.blobs[e] : nullptr;
+            b = reinterpret_cast<const uint8_t *>(__ldcg(reinterpret_cast<const unsigned long long *>(a.ws.blob) + g));
             gw = __ldcg(a.ws.gates + g);
         }
         blobs_s[g] = b;
@@ -339,11 +408,27 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_dec_down(DecodeArgs a, int n
         if (valid) code[t] = ldg_stream(bv.cd + static_cast<size_t>(r) * drowb + static_cast<size_t>(seg) * 16);
         load_scales<BITS>(bv.sd + static_cast<size_t>(valid ? r : 0) * dnsc, seg, valid, dsc[t]);
     }
+    pdl_wait();                                          // h (gate/up) is final
     // stage h of every group (gate/up's fp32 output) as pieces + block sums
-    for (int g4 = threadIdx.x; g4 < ng * (IL / 4); g4 += kDecThreads) {
-        const int t = g4 / (IL / 4), rem = g4 % (IL / 4);
-        const int c = rem / Q::PPC, q = rem % Q::PPC;
-        hs[(t * Q::PPC + q) * LPR + c] = __ldcg(reinterpret_cast<const float4 *>(a.ws.h) + g4);
+    {
+        constexpr int kB = 8;                            // loads of a thread in flight together
+        const int n4 = ng * (IL / 4);
+        for (int base = threadIdx.x; base < n4; base += kB * kDecThreads) {
+            float4 v[kB];
+#pragma unroll
+            for (int u = 0; u < kB; ++u) {
+                const int g4 = base + u * kDecThreads;
+                if (g4 < n4) v[u] = __ldcg(reinterpret_cast<const float4 *>(a.ws.h) + g4);
+            }
+#pragma unroll
+            for (int u = 0; u < kB; ++u) {
+                const int g4 = base + u * kDecThreads;
+                if (g4 < n4) {
+                    const int t = g4 / (IL / 4), rem = g4 % (IL / 4);
+                    hs[(t * Q::PPC + rem % Q::PPC) * LPR + rem / Q::PPC] = v[u];
+                }
+            }
+        }
     }
     __syncthreads();
     for (int b = threadIdx.x; b < ng * dnsc; b += kDecThreads) {
@@ -387,7 +472,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_dec_down(DecodeArgs a, int n
 
 // ------------------------------------------------------------------ host
 size_t decode_ws_bytes(int E, int k, int I) {
-    return 512 + ((static_cast<size_t>(E) * 4 + 255) / 256) * 256 + static_cast<size_t>(k + 1) * I * 4;
+    return kDecWsHeader + ((static_cast<size_t>(E) * 4 + 255) / 256) * 256 + static_cast<size_t>(k + 1) * I * 4;
 }
 
 static int down_lpr(int bits, int I) { return I / (bits == 4 ? 32 : 64); }
@@ -438,13 +523,13 @@ static int launch_decode_t(DecodeArgs a, int groups, cudaStream_t s) {
     cudaLaunchAttribute pdl;
     pdl.id = cudaLaunchAttributeProgrammaticStreamSerialization;
     pdl.val.programmaticStreamSerializationAllowed = 1;
-    // 1. router logits (skipped when the caller supplies them)
-    if (!a.logits_in) {
+    // 1. route (one CTA that only selects when the caller supplies the logits)
+    {
         cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(ceil_div(E, kLogitRows));
+        cfg.gridDim = dim3(a.logits_in ? 1 : ceil_div(E, kLogitRows));
         cfg.blockDim = dim3(kLogitRows * 32);
         cfg.stream = s;
-        int rc = cuda_status(cudaLaunchKernelEx(&cfg, k_dec_logits, a), "decode logits launch");
+        int rc = cuda_status(cudaLaunchKernelEx(&cfg, k_dec_route, a), "decode route launch");
         count_launches(1);
         if (rc) return rc;
     }
@@ -458,7 +543,7 @@ static int launch_decode_t(DecodeArgs a, int groups, cudaStream_t s) {
         cfg.dynamicSmemBytes = smem;
         cfg.stream = s;
         cfg.attrs = &pdl;
-        cfg.numAttrs = a.logits_in ? 0 : 1;              // x and given logits come from earlier work: no overlap
+        cfg.numAttrs = 1;
         int rc = cuda_status(cudaLaunchKernelEx(&cfg, k_dec_gateup<BITS>, a), "decode gate/up launch");
         count_launches(1);
         if (rc) return rc;

@@ -217,42 +217,51 @@ __device__ void block_topk_tree(const float *logits, int E, int k, uint64_t *lis
     __syncthreads();
 }
 
-// Sorts 64 keys, two per lane (element lane in v[0], element lane + 32 in
-// v[1]), in descending order across the warp: a bitonic network of 21 steps,
-// the stride-32 ones inside each lane.
-__device__ __forceinline__ void warp_sort64_desc(uint64_t (&v)[2], int lane) {
+// Sorts 32 * N keys, N per lane (element lane + 32 q in v[q]), in descending
+// order across the warp: a bitonic network whose compare-exchanges at
+// strides of 32 and more pair two keys of the same lane.
+template <int N>
+__device__ __forceinline__ void warp_sort_desc_n(uint64_t (&v)[N], int lane) {
 #pragma unroll
-    for (int k2 = 2; k2 <= 64; k2 <<= 1)
+    for (int k2 = 2; k2 <= 32 * N; k2 <<= 1)
 #pragma unroll
         for (int j = k2 >> 1; j > 0; j >>= 1) {
-            if (j == 32) {                               // partner in the same lane
-                const bool desc = k2 == 64 || (lane & k2) == 0;
-                const uint64_t hi = v[0] > v[1] ? v[0] : v[1], lo = v[0] > v[1] ? v[1] : v[0];
-                v[0] = desc ? hi : lo;
-                v[1] = desc ? lo : hi;
+            if (j >= 32) {                               // partner in the same lane
+#pragma unroll
+                for (int q = 0; q < N; ++q) {
+                    const int p = q ^ (j >> 5);
+                    if (p > q) {
+                        const bool desc = k2 == 32 * N || ((lane + 32 * q) & k2) == 0;
+                        const uint64_t lo_i = v[q], hi_i = v[p];
+                        const bool swap = desc ? lo_i < hi_i : lo_i > hi_i;
+                        v[q] = swap ? hi_i : lo_i;
+                        v[p] = swap ? lo_i : hi_i;
+                    }
+                }
             } else {
 #pragma unroll
-                for (int q = 0; q < 2; ++q) {
+                for (int q = 0; q < N; ++q) {
                     const int i = lane + 32 * q;
-                    const bool desc = k2 == 64 || (i & k2) == 0;
+                    const bool desc = k2 == 32 * N || (i & k2) == 0;
                     v[q] = cmpx(v[q], j, desc == ((i & j) == 0));
                 }
             }
         }
 }
 
-// block_topk_tree with two keys per thread: E <= 64 * NW, k <= 16.
-template <int NW>
-__device__ void block_topk_tree2(const float *logits, int E, int k, uint64_t *lists, uint64_t *sel) {
+// block_topk_tree with N keys per thread: E <= 32 * N * NW, k <= 16.  Warp w
+// sorts the keys of experts [32 N w, 32 N (w + 1)); the merge levels follow.
+template <int NW, int N>
+__device__ void block_topk_tree_n(const float *logits, int E, int k, uint64_t *lists, uint64_t *sel) {
     static_assert((NW & (NW - 1)) == 0, "a power-of-two number of warps");
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    uint64_t v[2];
+    uint64_t v[N];
 #pragma unroll
-    for (int q = 0; q < 2; ++q) {
-        const int e = warp * 64 + lane + 32 * q;
+    for (int q = 0; q < N; ++q) {
+        const int e = warp * 32 * N + lane + 32 * q;
         v[q] = e < E ? sel_key(__ldcg(logits + e), e) : 0ull;
     }
-    warp_sort64_desc(v, lane);
+    warp_sort_desc_n<N>(v, lane);
     if (lane < 16) lists[warp * 16 + lane] = v[0];
     __syncthreads();
 #pragma unroll 1
@@ -263,7 +272,7 @@ __device__ void block_topk_tree2(const float *logits, int E, int k, uint64_t *li
 #pragma unroll
             for (int j = 16; j > 0; j >>= 1) m = cmpx(m, j, (lane & j) == 0);
         }
-        __syncthreads();
+        __syncthreads();                                 // every read of this level before the writes
         if (warp < n / 2 && lane < 16) lists[warp * 16 + lane] = m;
         __syncthreads();
     }

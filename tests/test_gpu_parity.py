@@ -538,6 +538,72 @@ def test_fused_decode_is_one_kernel_and_replays_from_a_graph(decode_layer, one_k
     assert count() - c0 == 3 * 2 * sms
 
 
+def test_fused_decode_chain_replays_from_a_graph_and_leaves_ws_ready(decode_layer):
+    """The default path at full size is three kernels (route, gate/up, down)
+    per call; replayed from a CUDA graph it gives the eager result bit for
+    bit, and every call returns the route kernel's ticket count to zero."""
+    layer, g = decode_layer
+    x = W.make_tokens(W.SEED["decode"] + 710, 3, layer.H, "bf16")
+    b = g.decode_buffers()
+
+    def tickets():
+        return int(b["ws"][264:268].cpu().numpy().view(np.uint32)[0])
+    eager = []
+    for t in range(3):
+        n0 = M.moe_kernel_launches()
+        f = _run_fused(g, x[t:t + 1], "bf16")
+        assert f["err"] == 0 and M.moe_kernel_launches() - n0 == 3
+        assert tickets() == 0
+        eager.append(f)
+    xd_ = torch.empty(1, layer.H, dtype=torch.bfloat16, device="cuda")
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(graph, stream=s):
+            g.forward_decode(xd_, M.MOE_BF16, stream=s)
+    torch.cuda.current_stream().wait_stream(s)
+    for t in (2, 0, 1, 2):
+        xd_.copy_(dev_x(x[t:t + 1], "bf16"))
+        graph.replay()
+        torch.cuda.synchronize()
+        assert M.moe_device_error(clear=True) == 0
+        assert np.array_equal(b["ids"][:layer.k].cpu().numpy(), eager[t]["ids"])
+        assert np.array_equal(b["y"].cpu().numpy(), eager[t]["y"])
+        assert tickets() == 0
+
+
+def test_fused_decode_leaves_out_null_and_misaligned_blobs(decode_path):
+    """A selected expert whose table entry is NULL (MOE_DEVERR_NULL_BLOB) or
+    not 16-byte aligned (MOE_DEVERR_MISALIGNED) is left out: the ids and
+    gates are unchanged, and y is the full step minus that slot's weighted
+    expert output (the oracle's FFN of that expert)."""
+    layer = W.make_layer(440, 4, 256, 256, 24, 4, shared=True, w_dtype="bf16")
+    x = W.make_tokens(441, 1, 256, "bf16")
+    g = _layer_gpu(layer)
+    full = _run_fused(g, x, "bf16")
+    assert full["err"] == 0
+    j = 1
+    e = int(full["ids"][j])
+    saved = int(g.table[e].item())
+    outs = {}
+    for name, val, bit in (("null", 0, M.DEVERR_NULL_BLOB), ("misaligned", saved + 8, M.DEVERR_MISALIGNED)):
+        g.table[e] = val
+        try:
+            r = _run_fused(g, x, "bf16")
+        finally:
+            g.table[e] = saved
+        assert r["err"] == bit, (name, r["err"])
+        assert np.array_equal(r["ids"], full["ids"]) and np.array_equal(r["w"], full["w"])
+        outs[name] = r["y"]
+    assert np.array_equal(outs["null"], outs["misaligned"])
+    ffn_j = oracle.expert_ffn_rows(4, 256, 256, [layer.blobs[e]], xd(x, "bf16")[:1])[0]
+    want = full["y"].astype(np.float64) - float(full["w"][j]) * ffn_j
+    assert rel_err(outs["null"], want) <= TOL
+    again = _run_fused(g, x, "bf16")                      # the table restored: the full step again
+    assert again["err"] == 0 and np.array_equal(again["y"], full["y"])
+
+
 def test_fused_decode_barrier_timeout_recovers(decode_layer, one_kernel):
     """A grid barrier that can never complete (the test hook makes it wait
     for one CTA more than the grid has) runs out after its 2 ms limit: the

@@ -163,11 +163,8 @@ __global__ void __launch_bounds__(kLogitRows * 32) k_dec_route(DecodeArgs a) {
         }
     }
     __syncthreads();                                     // every row of this CTA written
-    if (threadIdx.x == 0) {                              // one fence per CTA on each side of the ticket
-        __threadfence();
-        last = atomicAdd(a.ws.tickets, 1u) == gridDim.x - 1;
-        if (last) __threadfence();
-    }
+    if (threadIdx.x == 0)                                // release this CTA's rows; the last also acquires all
+        last = sm100::atom_add_acq_rel_gpu(a.ws.tickets, 1u) == gridDim.x - 1;
     __syncthreads();
     if (!last) return;
     // the expert table (E <= 1024 pointers) is read together with the logits,
@@ -318,16 +315,16 @@ __global__ void __launch_bounds__(kDecThreads, 3) k_dec_gateup(DecodeArgs a) {
     };
     stage_x<BITS>(xs, cs, H, a.x, a.x_bf16);
     if (shared_group) {
-        load_codes(a.shared);                            // independent of the routing
         if (threadIdx.x == 0) prefetch_down_share<BITS>(a.shared, H, I, blockIdx.x - g * rblocks, rblocks);
+        load_codes(a.shared);                            // independent of the routing
     } else {
         pdl_wait();                                      // ids, gates and blob pointers are final from here on
         pdl_trigger();
         const uint8_t *blob = reinterpret_cast<const uint8_t *>(
             __ldcg(reinterpret_cast<const unsigned long long *>(a.ws.blob) + g));
         if (!blob) return;                               // reported by the route kernel; uniform over the CTA
-        load_codes(blob);
         if (threadIdx.x == 0) prefetch_down_share<BITS>(blob, H, I, blockIdx.x - g * rblocks, rblocks);
+        load_codes(blob);
     }
     float dot[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll

@@ -64,6 +64,8 @@ def lib():
         _lib.oracle_combine.argtypes = [I32, I32, I32, P, P, P, P, P]
         _lib.oracle_cache_sim.restype = C.c_long
         _lib.oracle_cache_sim.argtypes = [I32, I32, I32, I32, I32, P, P, P, P, P]
+        _lib.oracle_cache_sim_admit.restype = C.c_long
+        _lib.oracle_cache_sim_admit.argtypes = [I32, I32, I32, I32, I32, I32, P, P, P, P, P]
         _lib.oracle_cache_sim_prefetch.restype = C.c_long
         _lib.oracle_cache_sim_prefetch.argtypes = [I32, I32, I32, I32, I32, P, I32, P, P, P, P, P, P, P, P]
         _lib.oracle_set_threads.argtypes = [I32]
@@ -229,6 +231,21 @@ def cache_sim(ids: np.ndarray, n_experts: int, capacity: int, decay_period: int)
     if m < 0:
         raise ValueError("invalid cache trace")
     return dict(slot=slot, hit=hit.astype(bool), victim=victim, misses=int(m), counts=counts)
+
+
+def cache_sim_admit(ids: np.ndarray, n_experts: int, capacity: int, decay_period: int, admit_min: int):
+    """cache_sim with the admission threshold: ids [steps, n] -> dict(slot,
+    hit (int8: 1 hit, 0 admitted miss, 3 computed in place), victim, misses,
+    in_place, counts)."""
+    ids = _c(ids, np.int32)
+    steps, n = ids.shape
+    slot = np.empty((steps, n), np.int32); hit = np.empty((steps, n), np.int8)
+    victim = np.empty((steps, n), np.int32); counts = np.empty(n_experts, np.int64)
+    m = lib().oracle_cache_sim_admit(n_experts, capacity, decay_period, admit_min, steps, n, _p(ids), _p(slot),
+                                     _p(hit), _p(victim), _p(counts))
+    if m < 0:
+        raise ValueError("invalid cache trace")
+    return dict(slot=slot, hit=hit, victim=victim, misses=int(m), in_place=int((hit == 3).sum()), counts=counts)
 
 
 def cache_sim_prefetch(ids: np.ndarray, pf_ids: np.ndarray, n_experts: int, capacity: int, decay_period: int):

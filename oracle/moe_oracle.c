@@ -434,13 +434,20 @@ void oracle_combine(int T, int k, int H, const double *y_perm, const int32_t *pe
  *    the lowest free slot if any, else the slot of the resident expert that
  *    is not among this step's ids and is smallest in (counter, last use, id).
  *
- * ids [steps][n].  Outputs per (step, j): slot, hit (1/0), victim (-1 none).
+ * With admit_min > 1 (reading: the zero-copy form of "only the others move
+ * in" for experts that are rarely used), a miss whose counter after this use
+ * is below admit_min does not enter: it is computed in place from host
+ * memory (hit 3, slot -1, no victim) and nothing else changes beyond its
+ * counter and last use.  admit_min 0 or 1 is the policy above;
+ * oracle_cache_sim is that case.
+ *
+ * ids [steps][n].  Outputs per (step, j): slot, hit (1/0/3), victim (-1 none).
  * counts_out [n_experts] (optional): the counters after the last step.
- * Returns the number of misses, or -1 on invalid input (id out of range,
- * repeated id within a step, n > capacity). */
-long oracle_cache_sim(int n_experts, int capacity, int decay_period, int steps, int n,
-                      const int32_t *ids, int32_t *slot_out, int8_t *hit_out,
-                      int32_t *victim_out, int64_t *counts_out)
+ * Returns the number of misses (admitted or not), or -1 on invalid input (id
+ * out of range, repeated id within a step, n > capacity). */
+long oracle_cache_sim_admit(int n_experts, int capacity, int decay_period, int admit_min, int steps,
+                            int n, const int32_t *ids, int32_t *slot_out, int8_t *hit_out,
+                            int32_t *victim_out, int64_t *counts_out)
 {
     if (n > capacity || capacity <= 0)
         return -1;
@@ -478,8 +485,13 @@ long oracle_cache_sim(int n_experts, int capacity, int decay_period, int steps, 
                 slot_out[o] = slot_of[e];
                 continue;
             }
-            hit_out[o] = 0;
             misses++;
+            if (admit_min > 1 && cnt[e] < admit_min) {
+                hit_out[o] = 3;                      /* computed in place, not admitted */
+                slot_out[o] = -1;
+                continue;
+            }
+            hit_out[o] = 0;
             int slot = -1;
             for (int sl = 0; sl < capacity; ++sl)
                 if (expert_in[sl] < 0) {
@@ -523,6 +535,14 @@ bad:
     free(cnt);
     free(last);
     return -1;
+}
+
+long oracle_cache_sim(int n_experts, int capacity, int decay_period, int steps, int n,
+                      const int32_t *ids, int32_t *slot_out, int8_t *hit_out,
+                      int32_t *victim_out, int64_t *counts_out)
+{
+    return oracle_cache_sim_admit(n_experts, capacity, decay_period, 0, steps, n, ids, slot_out, hit_out,
+                                  victim_out, counts_out);
 }
 
 /* The same policy with prefetch (reading: the pages keep hot experts resident

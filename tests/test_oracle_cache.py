@@ -274,3 +274,61 @@ def test_prefetching_the_next_step_leaves_only_the_first_misses(oracle_lib):
     pf = np.vstack([ids[1:], np.full((1, n), -1, np.int32)])
     got = oracle_lib.cache_sim_prefetch(ids, pf, E, cap, 0)
     assert got["misses"] == n and got["hit"][1:].all()
+
+
+def _admit_golden():
+    rows, out = [], {}
+    for line in (GOLDEN / "cache_admit_trace.txt").read_text().splitlines():
+        line = line.strip()
+        if not line or line.startswith("#"):
+            continue
+        if line.startswith("step"):
+            ev = [[int(v) for v in part.split()] for part in line.split(":", 1)[1].split(";")]
+            rows.append(ev)
+        else:
+            f = line.split()
+            out[f[0]] = [int(v) for v in f[1:]]
+    return rows, out
+
+
+def test_admit_sim_hand_worked_trace(oracle_lib):
+    rows, out = _admit_golden()
+    ids = np.array([[ev[0] for ev in r] for r in rows], np.int32)
+    got = oracle_lib.cache_sim_admit(ids, 5, 2, 0, 2)
+    assert got["hit"].astype(int).tolist() == [[ev[1] for ev in r] for r in rows]
+    assert got["slot"].tolist() == [[ev[2] for ev in r] for r in rows]
+    assert got["victim"].tolist() == [[ev[3] for ev in r] for r in rows]
+    assert got["misses"] == out["misses"][0] and got["in_place"] == out["in_place"][0]
+    assert got["counts"].tolist() == out["counts"]
+
+
+@pytest.mark.parametrize("admit_min", [0, 1])
+def test_admit_sim_without_threshold_is_the_base_policy(oracle_lib, admit_min):
+    rng = np.random.default_rng(77 + admit_min)
+    ids = np.stack([rng.choice(40, 4, replace=False) for _ in range(300)]).astype(np.int32)
+    a = oracle_lib.cache_sim_admit(ids, 40, 9, 16, admit_min)
+    b = oracle_lib.cache_sim(ids, 40, 9, 16)
+    assert np.array_equal(a["slot"], b["slot"]) and np.array_equal(a["victim"], b["victim"])
+    assert np.array_equal(a["hit"].astype(bool), b["hit"]) and a["misses"] == b["misses"] and a["in_place"] == 0
+    assert np.array_equal(a["counts"], b["counts"])
+
+
+def test_admit_sim_invariants(oracle_lib):
+    """A threshold no counter reaches admits nothing.  With a cache as large
+    as the pool and no decay (nothing is ever evicted), each expert is
+    computed in place for its first admit_min - 1 uses, enters at use
+    admit_min and hits afterwards."""
+    rng = np.random.default_rng(5)
+    ids = np.stack([rng.choice(30, 3, replace=False) for _ in range(200)]).astype(np.int32)
+    never = oracle_lib.cache_sim_admit(ids, 30, 6, 0, 10 ** 6)
+    assert (never["hit"] == 3).all() and (never["slot"] == -1).all() and (never["victim"] == -1).all()
+    assert never["misses"] == ids.size == never["in_place"]
+    big = oracle_lib.cache_sim_admit(ids, 30, 30, 0, 3)
+    uses = np.zeros(30, int)
+    for s in range(ids.shape[0]):
+        for j in range(ids.shape[1]):
+            e = ids[s, j]
+            uses[e] += 1
+            want = 3 if uses[e] < 3 else (0 if uses[e] == 3 else 1)
+            assert big["hit"][s, j] == want, (s, j, e, uses[e])
+    assert (big["victim"] == -1).all()

@@ -299,6 +299,21 @@ def layer_oracle_step(layer, tokens, T_batch=8):
     return step
 
 
+def graph_upload(graph):
+    """Uploads an instantiated CUDA graph to the device (cuGraphUpload) so
+    that its first replay runs only its work.  A graph whose replay changes
+    state (the expert cache of the paging workloads) cannot be replayed once
+    beforehand just to upload it."""
+    import ctypes
+    import torch
+    drv = ctypes.CDLL("libcuda.so.1")
+    drv.cuGraphUpload.argtypes = [ctypes.c_void_p, ctypes.c_void_p]
+    rc = drv.cuGraphUpload(ctypes.c_void_p(graph.raw_cuda_graph_exec()),
+                           ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    if rc != 0:
+        raise RuntimeError(f"cuGraphUpload failed ({rc})")
+
+
 def run_graph_steps(step_fn, first, count, time_ffn=True):
     """Captures `count` steps in one CUDA graph; returns (graph, ffn event pairs)."""
     import torch
@@ -563,7 +578,14 @@ def bench_paging(args, world, rank, pk):
         pv[e0:e0 + 512, :nb].copy_(bt)
     slab = torch.empty(cap * stride, dtype=torch.uint8, device="cuda")
     table = torch.zeros(E, dtype=torch.int64, device="cuda")
-    cache = M.ExpCache(E, cap, nb, stride, pool, slab, table, decay_period=256)
+    dev_mode = args.device_staging
+    if dev_mode:                                         # policy and copies on the device (devcache_*)
+        from quantized_expert_ffn_route_b200.paged import DevicePagedExpertStack
+        stack = DevicePagedExpertStack(1, E, 2, H, I, k, pool, slab, table, cap, nb, stride, decay_period=256,
+                                       admit_min=args.admit_min)
+        cache = stack.cache
+    else:
+        cache = M.ExpCache(E, cap, nb, stride, pool, slab, table, decay_period=256)
     n_steps = args.warmup + args.steps
     trace = np.stack(list(W.paging_trace(W.SEED["paging"] + 17 * rank, E, k, n_steps + 64, s=c["zipf_s"],
                                          drift_every=c["drift_every"], drift_prob=c["drift_prob"],
@@ -571,7 +593,8 @@ def bench_paging(args, world, rank, pk):
     logits = torch.from_numpy(trace).cuda()
     x_host = W.make_tokens(W.SEED["paging"] + 1, n_steps + 64, H, "bf16")
     xs = torch.from_numpy(x_host.view(np.int16)).view(torch.bfloat16).cuda()
-    b = M.alloc_step_buffers(1, H, I, E, k, 2, M.MOE_MODE_GEMV, torch.device("cuda"), False)
+    b = stack.b if dev_mode else M.alloc_step_buffers(1, H, I, E, k, 2, M.MOE_MODE_GEMV, torch.device("cuda"),
+                                                         False)
     ids_h = torch.empty(k, dtype=torch.int32).pin_memory()
     # expert lists of the two FFN calls of a step: [count, ids...] for the
     # hits (resident: computed at once) and for the misses (after their copies)
@@ -582,7 +605,11 @@ def bench_paging(args, world, rank, pk):
     ev_hit = [None, None]
 
     def step(i, x=None):
-        M.moe_route_topk(None, 0, None, 0, logits[i], None, 1, H, E, k, b.ids, b.w)
+        if dev_mode:
+            stack.layer_step(0, xs[i] if x is None else x, M.MOE_BF16, logits[i])
+            return
+        M.moe_route_topk(None, 0, None, 0, logits[i], None, 1, H, E, k, b.ids, b.w, None, b.ws_route,
+                         b.sizes["route"])
         M.moe_permute(b.ids, 1, k, E, b.offsets, b.perm_src, b.perm_dst, b.active, b.ws_perm, b.sizes["perm"])
         ids_h.copy_(b.ids[:k], non_blocking=True)
         s.synchronize()                                  # the ids cross to the host
@@ -633,31 +660,51 @@ def bench_paging(args, world, rank, pk):
     for i in range(args.warmup):
         step(i)
     torch.cuda.synchronize()
+    graph = None
+    if dev_mode:
+        # nothing in a device-staged step waits for the host: the K steps are
+        # one CUDA graph, uploaded before the timed region and replayed once
+        nc0 = M.moe_kernel_launches()
+        graph, _ = run_graph_steps(lambda i, e0, e1: step(i), args.warmup, args.steps, time_ffn=False)
+        graph_launches = M.moe_kernel_launches() - nc0
+        graph_upload(graph)                              # the timed replay is the steps' only run
+        torch.cuda.synchronize()
     st0 = cache.stats()
     n0 = M.moe_kernel_launches()
     clocks = ClockSampler(torch.cuda.current_device())
     barrier(world)
     a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record()
-    for i in range(args.warmup, n_steps):
-        step(i)
+    if graph is not None:
+        graph.replay()
+    else:
+        for i in range(args.warmup, n_steps):
+            step(i)
     z.record()
     torch.cuda.synchronize()
     barrier(world)
     clk = clocks.stop()
-    launches = M.moe_kernel_launches() - n0
+    launches = graph_launches if graph is not None else M.moe_kernel_launches() - n0
     assert M.moe_device_error() == 0
     ms = max_over_ranks(a.elapsed_time(z), world)
     st1 = cache.stats()
-    mps = misses_per_step[args.warmup:n_steps]
-    overlap, copy_ms = overlap_pass(n_steps, min(200, 64))
-    staged = st1["bytes_staged"] - st0["bytes_staged"]
     value = sum_over_ranks(args.steps, world) / (ms / 1e3)
+    if dev_mode:
+        in_place = st1["in_place"] - st0["in_place"]
+        staged = st1["bytes_copied"] - st0["bytes_copied"] + in_place * nb     # every byte over the link
+        mps = [(st1["misses"] - st0["misses"]) / args.steps]
+        overlap = None
+    else:
+        mps = misses_per_step[args.warmup:n_steps]
+        overlap, copy_ms = overlap_pass(n_steps, min(200, 64))
+        staged = st1["bytes_staged"] - st0["bytes_staged"]
     link_ach = staged / (ms / 1e3) / 1e9
     steady = mps[500:] if len(mps) > 600 else mps
     roof = {"bound": "host_link", "achieved": round(link_ach, 2), "peak": round(link, 2), "unit": "GB/s",
             "frac": round(link_ach / link, 4), "traffic": None,
-            "kernel": "expcache_stage copies (cudaMemcpyAsync pinned host -> HBM slot)",
+            "kernel": ("devcache_stage (policy kernel on the device; copy kernel of SM loads from the mapped pinned "
+                       "pool; no host synchronisation per step)" if dev_mode
+                       else "expcache_stage copies (cudaMemcpyAsync pinned host -> HBM slot)"),
             "peak_source": "pinned 1 GiB host->device copy measured in this run",
             "misses_per_step": round(float(np.mean(mps)), 3),
             "misses_per_step_steady": round(float(np.mean(steady)), 3),
@@ -665,7 +712,11 @@ def bench_paging(args, world, rank, pk):
             "overlap": None if overlap is None else round(overlap, 4),
             "overlap_definition": ("share of each step's copy interval (first copy issued -> device table "
                                    "patched) during which the resident experts' FFN ran on the compute stream, "
-                                   "from CUDA events over an untimed pass of 64 further steps")}
+                                   "from CUDA events over an untimed pass of 64 further steps; not measured "
+                                   "with device staging, whose copies run in a kernel beside the hits' FFN")}
+    if dev_mode:
+        roof["in_place_per_step"] = round(in_place / args.steps, 3)
+        roof["admit_min"] = args.admit_min
 
     e2e = None
     if not args.no_e2e:
@@ -698,6 +749,8 @@ def bench_paging(args, world, rank, pk):
         cpu = oracle_baseline(step, args.cpu_seconds, 2, 1, "paging steps (1 token, 10 of 24,576 experts)")
     cache.close()
     cfg = paging_config(E, k, nb, cap, c, world)
+    if dev_mode:
+        cfg["staging"] = "device-initiated" + (f", admit_min {args.admit_min}" if args.admit_min > 1 else "")
     roof["cache"] = {"misses": st1["misses"] - st0["misses"], "hits": st1["hits"] - st0["hits"]}
     return dict(value=value, ms=ms, steps=args.steps, roofline=roof, e2e=e2e, cpu=cpu, clocks=clk,
                 launches=launches, config=cfg, dtype="fp32 (CUDA-core FMA on 2-bit codes)")
@@ -726,8 +779,15 @@ def bench_paging48(args, world, rank, pk):
         pv[l * El:(l + 1) * El, :nb].copy_(bt)
     slab = torch.empty(cap * stride, dtype=torch.uint8, device="cuda")
     table = torch.zeros(E, dtype=torch.int64, device="cuda")
-    stack = PagedExpertStack(L, El, 2, H, I, k, pool, slab, table, cap, nb, stride, decay_period=256,
-                             prefetch=pf_n)
+    dev_mode = args.device_staging
+    if dev_mode:                                         # policy and copies on the device; no prefetch
+        from quantized_expert_ffn_route_b200.paged import DevicePagedExpertStack
+        pf_n = 0
+        stack = DevicePagedExpertStack(L, El, 2, H, I, k, pool, slab, table, cap, nb, stride, decay_period=256,
+                                       admit_min=args.admit_min)
+    else:
+        stack = PagedExpertStack(L, El, 2, H, I, k, pool, slab, table, cap, nb, stride, decay_period=256,
+                                 prefetch=pf_n)
     tokens_w, tokens_t = max(1, args.warmup // 3), min(args.steps, c["tokens"])
     n_tok = tokens_w + tokens_t + 16
     trace = np.stack(list(W.paging48_trace(W.SEED["paging48"] + 17 * rank, L, El, n_tok, s=c["zipf_s"],
@@ -745,6 +805,14 @@ def bench_paging48(args, world, rank, pk):
     for t in range(tokens_w):
         token(t)
     torch.cuda.synchronize()
+    graph = None
+    if dev_mode:
+        # no layer waits for the host: the timed tokens are one CUDA graph
+        nc0 = M.moe_kernel_launches()
+        graph, _ = run_graph_steps(lambda t, e0, e1: token(t), tokens_w, tokens_t, time_ffn=False)
+        graph_launches = M.moe_kernel_launches() - nc0
+        graph_upload(graph)                              # the timed replay is the tokens' only run
+        torch.cuda.synchronize()
     st0 = stack.cache.stats()
     stack.record, stack.events = True, []
     n0 = M.moe_kernel_launches()
@@ -752,23 +820,31 @@ def bench_paging48(args, world, rank, pk):
     barrier(world)
     a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record()
-    for t in range(tokens_w, tokens_w + tokens_t):
-        token(t)
+    if graph is not None:
+        graph.replay()
+    else:
+        for t in range(tokens_w, tokens_w + tokens_t):
+            token(t)
     z.record()
     torch.cuda.synchronize()
     barrier(world)
     clk = clocks.stop()
     stack.record = False
-    launches = M.moe_kernel_launches() - n0
+    launches = graph_launches if graph is not None else M.moe_kernel_launches() - n0
     assert M.moe_device_error() == 0
     ms = max_over_ranks(a.elapsed_time(z), world)
     st1 = stack.cache.stats()
-    staged = st1["bytes_staged"] - st0["bytes_staged"]
     misses = st1["misses"] - st0["misses"]
-    prefetched = st1["prefetched"] - st0["prefetched"]
+    if dev_mode:
+        in_place = st1["in_place"] - st0["in_place"]
+        staged = st1["bytes_copied"] - st0["bytes_copied"] + in_place * nb     # every byte over the link
+        prefetched = 0
+    else:
+        staged = st1["bytes_staged"] - st0["bytes_staged"]
+        prefetched = st1["prefetched"] - st0["prefetched"]
     # prefetched experts that a later stage found resident before they were evicted
     pending, useful = set(), 0
-    for gids, hit, _, victim, pf, pf_slot, pf_victim in stack.events:
+    for gids, hit, _, victim, pf, pf_slot, pf_victim in (() if dev_mode else stack.events):
         for e, h in zip(gids.tolist(), hit.tolist()):
             if h and e in pending:
                 useful += 1
@@ -780,7 +856,9 @@ def bench_paging48(args, world, rank, pk):
     link_ach = staged / (ms / 1e3) / 1e9
     roof = {"bound": "host_link", "achieved": round(link_ach, 2), "peak": round(link, 2), "unit": "GB/s",
             "frac": round(link_ach / link, 4), "traffic": None,
-            "kernel": "expcache_stage + expcache_prefetch copies (cudaMemcpyAsync pinned host -> HBM slot)",
+            "kernel": ("devcache_stage (policy kernel on the device; copy kernel of SM loads from the mapped pinned "
+                       "pool; no host synchronisation per layer)" if dev_mode
+                       else "expcache_stage + expcache_prefetch copies (cudaMemcpyAsync pinned host -> HBM slot)"),
             "peak_source": "pinned 1 GiB host->device copy measured in this run",
             "misses_per_token": round(misses / tokens_t, 2),
             "prefetched_per_token": round(prefetched / tokens_t, 2),
@@ -821,6 +899,8 @@ def bench_paging48(args, world, rank, pk):
         cpu = oracle_baseline(step, args.cpu_seconds, L, 1.0 / L, "layer steps (1 token through 1 of 48 layers)")
     stack.close()
     cfg = paging48_config(L, El, k, nb, cap, c, pf_n, world)
+    if dev_mode:
+        cfg["staging"] = "device-initiated" + (f", admit_min {args.admit_min}" if args.admit_min > 1 else "")
     return dict(value=value, ms=ms, steps=tokens_t, roofline=roof, e2e=e2e, cpu=cpu, clocks=clk,
                 launches=launches, config=cfg, dtype="fp32 (CUDA-core FMA on 2-bit codes)")
 
@@ -967,6 +1047,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default="decode", choices=["decode", "verify", "prefill", "paging", "paging48"])
     ap.add_argument("--prefetch", type=int, default=-1, help="paging48: experts prefetched per layer (-1: config)")
+    ap.add_argument("--device-staging", action="store_true",
+                    help="paging, paging48: the cache policy and copies on the device (devcache_*)")
+    ap.add_argument("--admit-min", type=int, default=0,
+                    help="device staging: misses used fewer times are computed in place, not admitted")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--window", type=int, default=16)
     ap.add_argument("--chunk", type=int, default=8192)

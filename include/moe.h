@@ -146,7 +146,10 @@ size_t moe_expert_blob_bytes(int bits, int H, int I);
  *  bias     device [E] fp32 or NULL (added to logits from x, not to logits_in).
  *  topk_ids device [T,k] int32 out.  topk_w device [T,k] fp32 out.
  *  logits_out device [T,E] fp32 out, or NULL.
- *  ws       device workspace of at least moe_route_ws_size(T,E,k) bytes.
+ *  ws       device workspace of at least moe_route_ws_size(T,E,k) bytes:
+ *           the logits when they are computed here and logits_out is NULL,
+ *           and, when E > 1024, the chunked top-k's candidates (so with
+ *           E > 1024 ws is needed even with logits_in or logits_out).
  * Limits: 1 <= k <= min(E, 32), 1 <= E <= 32768, T >= 0.  T = 0 is a no-op.
  * A selected NaN/+inf logit sets MOE_DEVERR_NONFINITE and yields NaN gates. */
 size_t moe_route_ws_size(int T, int E, int k);
@@ -382,6 +385,91 @@ int expcache_copy_times(moe_expcache *c, const void *ref_event, float *start_ms,
 
 /* Test hook: the next `n` copies report failure before being issued (MOE_EIO). */
 int expcache_inject_copy_failures(moe_expcache *c, int n);
+
+/* ------------------------------------------ device-initiated expert staging
+ * The expert cache's policy and copies on the GPU (Strata article, section 2
+ * item 2: resident experts are computed at once, the others move in from
+ * host memory; the host-driven expcache_* calls above are the form that
+ * hands each step's ids to the host).  devcache_stage reads the step's ids
+ * from DEVICE memory and enqueues, with no host synchronisation:
+ *  1. one policy kernel on `compute`: the policy of expcache_stage (halving
+ *     decay every decay_period steps; count += 1 and last use = step for each
+ *     id in order; resident -> hit; a miss takes the lowest free slot, else
+ *     the slot of the resident expert outside this step with the smallest
+ *     (count, last use, id)), the device table patched at once (victims
+ *     NULL, admitted misses -> their slot), and the FFN lists written;
+ *  2. one copy kernel on `copy`, after the policy kernel: the admitted
+ *     misses' blobs from the host pool into their slots, read by the SMs
+ *     through the pool's device mapping (16-byte loads over the host link).
+ * devcache_join(c, s) makes `s` wait for the copy kernel.  The sequence is
+ * fixed by the host arguments alone, so a CUDA graph can hold whole steps.
+ * Zero-copy compute for cold experts: with admit_min > 1 a missed expert
+ * whose count (after this use) is below admit_min is not admitted; for this
+ * step its table entry points at its blob in the host pool, which the
+ * expert FFN in MOE_MODE_GEMV reads in place (only that mode: the other
+ * paths read blobs with bulk copies, which this build keeps off host
+ * memory); the next devcache_stage clears the entry.  admit_min 0 or 1:
+ * every miss is admitted (the policy of expcache_stage exactly).
+ */
+typedef struct moe_devcache moe_devcache;
+
+typedef struct {
+    int32_t n_experts;      /* experts in the host pool */
+    int32_t capacity;       /* HBM slots (<= n_experts) */
+    int64_t blob_bytes;     /* bytes per expert (multiple of 16, <= 1 GiB) */
+    int64_t slot_stride;    /* bytes between slots and pool entries (>= blob_bytes, multiple of 256) */
+    void *host_pool;        /* host [n_experts * slot_stride], page-locked and mapped (cudaHostAlloc, or
+                               cudaHostRegister with cudaHostRegisterMapped), caller-owned */
+    void *hbm_slab;         /* device [capacity * slot_stride], caller-owned */
+    void *dev_table;        /* device [n_experts] pointers, caller-owned; set to NULL at create */
+    int32_t decay_period;   /* steps between halvings; 0 = never */
+    int32_t admit_min;      /* see above; 0 or 1 = admit every miss */
+    int32_t log_steps;      /* steps of per-id events kept on the device (ring) for devcache_events; 0 = none */
+} moe_devcache_desc;
+
+typedef struct {
+    int64_t steps, hits, misses, evictions;
+    int64_t in_place;       /* misses computed in place (not admitted) */
+    int64_t bytes_copied;   /* bytes of admitted misses */
+    int64_t bad_steps;      /* steps whose ids were out of range or repeated (nothing changed) */
+} moe_devcache_stats;
+
+/* Creates the cache (empty, every table entry NULL); synchronises the device.
+ * MOE_EINVAL on a bad descriptor (including a host_pool the device cannot
+ * address), MOE_ENOMEM/MOE_ECUDA on allocation failures. */
+int devcache_create(const moe_devcache_desc *d, moe_devcache **out);
+void devcache_destroy(moe_devcache *c);
+
+/* One step.  ids_dev: device int32 [n] (n <= 32, n <= capacity, else
+ * MOE_EINVAL / MOE_EBUSY), the step's distinct ids, each offset by id_base
+ * into the pool (a layer's experts id_base .. id_base + E_l - 1).  act_dev:
+ * device int32 [66] out, two active-expert lists in the layout the expert
+ * FFN takes: act_dev[0] = n_a, act_dev[1..n_a] the ids (without id_base) of
+ * the hits and of experts computed in place -- usable at once; act_dev[33] =
+ * n_b, act_dev[34..33+n_b] the admitted misses -- usable on a stream after
+ * devcache_join.  Ids that are out of range or repeated set
+ * MOE_DEVERR_BAD_EXPERT and leave both lists empty and the cache unchanged.
+ * compute and copy may be the same stream; when they differ, the previous
+ * step must have been joined (devcache_join) first, else MOE_EINVAL. */
+int devcache_stage(moe_devcache *c, const int32_t *ids_dev, int n, int32_t id_base, int32_t *act_dev,
+                   moe_stream_t compute, moe_stream_t copy);
+
+/* Makes `s` wait for the copy kernel of the last devcache_stage. */
+int devcache_join(moe_devcache *c, moe_stream_t s);
+
+/* Host copies (after a device synchronisation) of the logged events of steps
+ * [first_step, first_step + n_steps): per step 32 entries, entry j for the
+ * step's j-th id: hit 1 = hit, 0 = admitted miss, 3 = computed in place;
+ * slot (-1 if none), victim (-1 if none).  The steps must still be in the
+ * log ring of log_steps steps, else MOE_EINVAL.  Any output may be NULL. */
+int devcache_events(moe_devcache *c, int64_t first_step, int n_steps, int8_t *hit_out, int32_t *slot_out,
+                    int32_t *victim_out);
+
+/* Counters (a synchronous copy from the device). */
+int devcache_stats(moe_devcache *c, moe_devcache_stats *out);
+
+/* Host copies of the per-expert counts and slots (n_experts entries each; either may be NULL). */
+int devcache_snapshot(moe_devcache *c, int64_t *counts_out, int32_t *slot_of_out);
 
 #ifdef __cplusplus
 }

@@ -54,6 +54,21 @@ class ExpCacheStats(C.Structure):
                 ("prefetched", C.c_int64)]
 
 
+class DevCacheDesc(C.Structure):
+    _fields_ = [("n_experts", C.c_int32), ("capacity", C.c_int32), ("blob_bytes", C.c_int64),
+                ("slot_stride", C.c_int64), ("host_pool", C.c_void_p), ("hbm_slab", C.c_void_p),
+                ("dev_table", C.c_void_p), ("decay_period", C.c_int32), ("admit_min", C.c_int32),
+                ("log_steps", C.c_int32)]
+
+
+class DevCacheStats(C.Structure):
+    _fields_ = [("steps", C.c_int64), ("hits", C.c_int64), ("misses", C.c_int64), ("evictions", C.c_int64),
+                ("in_place", C.c_int64), ("bytes_copied", C.c_int64), ("bad_steps", C.c_int64)]
+
+
+DEVCACHE_ACT_INTS = 66          # two active-expert lists: [0] n_a, [1..32] ids; [33] n_b, [34..65] ids
+DEVCACHE_HIT, DEVCACHE_MISS, DEVCACHE_IN_PLACE = 1, 0, 3
+
 _lib = None
 
 
@@ -101,6 +116,13 @@ def lib():
         "expcache_inject_copy_failures": (I, [P, I]),
         "expcache_copy_times": (I, [P, P, C.POINTER(C.c_float), C.POINTER(C.c_float)]),
         "expcache_prefetch": (I, [P, P, I, S, P, P, C.POINTER(C.c_int)]),
+        "devcache_create": (I, [C.POINTER(DevCacheDesc), C.POINTER(P)]),
+        "devcache_destroy": (None, [P]),
+        "devcache_stage": (I, [P, P, I, C.c_int32, P, S, S]),
+        "devcache_join": (I, [P, S]),
+        "devcache_events": (I, [P, C.c_int64, I, P, P, P]),
+        "devcache_stats": (I, [P, C.POINTER(DevCacheStats)]),
+        "devcache_snapshot": (I, [P, P, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -327,3 +349,59 @@ class ExpCache:
         a, b = C.c_float(0.0), C.c_float(0.0)
         _check(lib().expcache_copy_times(self.h, C.c_void_p(ref_event.cuda_event), C.byref(a), C.byref(b)))
         return a.value, b.value
+
+
+class DevCache:
+    """Handle around the devcache_* calls (device-initiated staging; the caller
+    owns pool, slab and table).  The pool must be page-locked and mapped
+    (torch's pin_memory() is)."""
+
+    def __init__(self, n_experts, capacity, blob_bytes, slot_stride, host_pool, hbm_slab, dev_table,
+                 decay_period=256, admit_min=0, log_steps=0):
+        d = DevCacheDesc(n_experts, capacity, blob_bytes, slot_stride, _p(host_pool), _p(hbm_slab), _p(dev_table),
+                         decay_period, admit_min, log_steps)
+        h = C.c_void_p()
+        _check(lib().devcache_create(C.byref(d), C.byref(h)))
+        self.h = h
+        self.n_experts = n_experts
+
+    def close(self):
+        if self.h:
+            lib().devcache_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def stage(self, ids_dev, n, act_dev, id_base=0, stream=None, copy_stream=None):
+        """One step from device ids; act_dev: device int32 [66] (DEVCACHE_ACT_INTS)."""
+        s = _stream(stream)
+        _check(lib().devcache_stage(self.h, _p(ids_dev), int(n), int(id_base), _p(act_dev), s,
+                                    s if copy_stream is None else _stream(copy_stream)))
+
+    def join(self, stream=None):
+        _check(lib().devcache_join(self.h, _stream(stream)))
+
+    def events(self, first_step, n_steps):
+        """(hit, slot, victim) numpy arrays [n_steps, 32] of logged steps."""
+        import numpy as np
+        hit = np.zeros((n_steps, 32), np.int8)
+        slot = np.zeros((n_steps, 32), np.int32)
+        victim = np.zeros((n_steps, 32), np.int32)
+        _check(lib().devcache_events(self.h, int(first_step), int(n_steps), _p(hit), _p(slot), _p(victim)))
+        return hit, slot, victim
+
+    def stats(self) -> dict:
+        st = DevCacheStats()
+        _check(lib().devcache_stats(self.h, C.byref(st)))
+        return {f: getattr(st, f) for f, _ in DevCacheStats._fields_}
+
+    def snapshot(self):
+        import numpy as np
+        cnt = np.empty(self.n_experts, np.int64)
+        slot = np.empty(self.n_experts, np.int32)
+        _check(lib().devcache_snapshot(self.h, _p(cnt), _p(slot)))
+        return cnt, slot

@@ -75,14 +75,6 @@ static bool check_dtype(int dt) { return dt == MOE_F32 || dt == MOE_BF16; }
 
 using namespace moe;
 
-#define REQUIRE(cond, ...)            \
-    do {                              \
-        if (!(cond)) {                \
-            set_error(__VA_ARGS__);   \
-            return MOE_EINVAL;        \
-        }                             \
-    } while (0)
-
 extern "C" {
 
 const char *moe_last_error(void) { return t_err.c_str(); }
@@ -137,9 +129,10 @@ size_t moe_expert_blob_bytes(int bits, int H, int I) {
 
 // ------------------------------------------------------------------ route
 size_t moe_route_ws_size(int T, int E, int k) {
-    (void)k;
     if (T <= 0 || E <= 0) return 0;
-    return static_cast<size_t>(T) * E * sizeof(float);
+    if (E <= 1024) return static_cast<size_t>(T) * E * sizeof(float);
+    k = k < 1 ? 1 : (k > 32 ? 32 : k);
+    return topk_chunk_ws_offset(T, E) + topk_chunk_ws_bytes(T, E, k);   // logits, then the chunk candidates
 }
 
 int moe_route_topk(const void *x, int x_dtype, const void *w_router, int w_dtype, const float *logits_in,
@@ -166,6 +159,9 @@ int moe_route_topk(const void *x, int x_dtype, const void *w_router, int w_dtype
         REQUIRE(logits_in != nullptr, "w_router and logits_in are both NULL");
         REQUIRE(aligned16(logits_in), "logits_in must be 16-byte aligned");
     }
+    REQUIRE(E <= 1024 || (ws && ws_bytes >= moe_route_ws_size(T, E, k) && aligned16(ws)),
+            "E > 1024 needs the workspace (the chunked top-k keeps its candidates there): need %zu bytes",
+            moe_route_ws_size(T, E, k));
     cudaStream_t st = reinterpret_cast<cudaStream_t>(s);
     unsigned *err = device_error_word();
     if (!err) return cuda_status(cudaErrorInvalidDevice, "device error word");
@@ -188,7 +184,8 @@ int moe_route_topk(const void *x, int x_dtype, const void *w_router, int w_dtype
             if (rc) return rc;
         }
     }
-    launch_topk(logits, T, E, k, topk_ids, topk_w, err, st);
+    launch_topk(logits, T, E, k, topk_ids, topk_w, err,
+                E > 1024 ? static_cast<uint8_t *>(ws) + topk_chunk_ws_offset(T, E) : nullptr, st);
     return cuda_status(cudaGetLastError(), "route launch");
 }
 

@@ -20,6 +20,27 @@ unsigned *device_error_word();                       // this device's error word
 int num_sms();                                       // SMs of the current device (cached)
 void count_launches(int n);                          // adds to the library's launch counter
 
+// Argument check of a C-ABI call: sets the error message, returns MOE_EINVAL.
+#define REQUIRE(cond, ...)            \
+    do {                              \
+        if (!(cond)) {                \
+            set_error(__VA_ARGS__);   \
+            return MOE_EINVAL;        \
+        }                             \
+    } while (0)
+
+// Makes a device current for the scope and restores the caller's.
+struct DeviceGuard {
+    int prev = -1;
+    explicit DeviceGuard(int dev) {
+        if (cudaGetDevice(&prev) == cudaSuccess && prev != dev) cudaSetDevice(dev);
+    }
+    ~DeviceGuard() {
+        int cur = -1;
+        if (prev >= 0 && cudaGetDevice(&cur) == cudaSuccess && cur != prev) cudaSetDevice(prev);
+    }
+};
+
 // Names the enclosing C-ABI call in profiler timelines (NVTX range; a no-op
 // when no tool is attached).
 struct NvtxRange {

@@ -62,26 +62,6 @@ struct moe_expcache {
     int inject_fail = 0;
 };
 
-#define REQUIRE(cond, ...)            \
-    do {                              \
-        if (!(cond)) {                \
-            set_error(__VA_ARGS__);   \
-            return MOE_EINVAL;        \
-        }                             \
-    } while (0)
-
-// Makes the cache's device current for the scope and restores the caller's.
-struct DeviceGuard {
-    int prev = -1;
-    explicit DeviceGuard(int dev) {
-        if (cudaGetDevice(&prev) == cudaSuccess && prev != dev) cudaSetDevice(dev);
-    }
-    ~DeviceGuard() {
-        int cur = -1;
-        if (prev >= 0 && cudaGetDevice(&cur) == cudaSuccess && cur != prev) cudaSetDevice(prev);
-    }
-};
-
 static void destroy_events(moe_expcache *c) {
     if (c->ev_compute) cudaEventDestroy(c->ev_compute);
     if (c->ev_done) cudaEventDestroy(c->ev_done);

@@ -12,7 +12,11 @@ void launch_router_logits(const void *x, int x_dtype, const void *w, int w_dtype
 bool router_mma_supported(int x_dtype, int w_dtype, int T, int H);
 int launch_router_mma(const void *x, const void *w, const float *bias, int T, int H, int E, float *out,
                       unsigned *err, cudaStream_t s);
-void launch_topk(const float *logits, int T, int E, int k, int32_t *ids, float *w, unsigned *err, cudaStream_t s);
+void launch_topk(const float *logits, int T, int E, int k, int32_t *ids, float *w, unsigned *err, void *cand_ws,
+                 cudaStream_t s);
+// E > 1024: the chunk candidates' place in the route workspace and their size
+size_t topk_chunk_ws_offset(int T, int E);
+size_t topk_chunk_ws_bytes(int T, int E, int k);
 
 size_t permute_ws_bytes(int T, int k, int E);
 int launch_permute(const int32_t *ids, int T, int k, int E, int32_t *offsets, int32_t *perm_src, int32_t *perm_dst,

@@ -96,6 +96,62 @@ __global__ void __launch_bounds__(1024) k_permute_small(const int32_t *__restric
     if (threadIdx.x < 32) warp_scatter(ids, 0, n, k, E, cnt, perm_src, perm_dst);
 }
 
+// Few pairs (n = T*k <= 32, e.g. one decode token) and any E: no counting
+// array over the experts.  Warp 0 holds the n ids; the row of a valid pair is
+// the number of valid pairs with a smaller id plus the earlier pairs with the
+// same id (the stable order), and each offset is the number of valid pairs
+// with a smaller id, counted directly -- O(E * n) comparisons spread over the
+// block instead of a scan over E counters.
+constexpr int kSparsePairs = 32;
+
+__global__ void __launch_bounds__(1024) k_permute_sparse(const int32_t *__restrict__ ids, int n, int k, int E,
+                                                          int32_t *__restrict__ offsets,
+                                                          int32_t *__restrict__ perm_src,
+                                                          int32_t *__restrict__ perm_dst,
+                                                          int32_t *__restrict__ active, int active_cap,
+                                                          unsigned *err) {
+    __shared__ int ids_s[kSparsePairs];
+    const int tid = threadIdx.x;
+    if (tid < 32) {
+        const int lane = tid;
+        const bool live = lane < n;
+        const int e = live ? ids[lane] : -1;
+        const bool ok = live && e >= 0 && e < E;
+        if (live && !ok) report(err, MOE_DEVERR_BAD_EXPERT);
+        ids_s[lane] = ok ? e : -1;                       // -1: no valid pair here
+        __syncwarp();
+        int r = 0, d = 0;
+        bool first = ok;
+        for (int q = 0; q < n; ++q) {
+            const int f = ids_s[q];
+            if (f < 0) continue;
+            r += f < e || (f == e && q < lane);
+            first &= !(f == e && q < lane);
+            if (ok && f < e) {                           // distinct ids below e: count first occurrences
+                bool fq = true;
+                for (int u = 0; u < q; ++u) fq &= ids_s[u] != f;
+                d += fq;
+            }
+        }
+        if (ok) {
+            perm_src[r] = lane / k;
+            perm_dst[lane] = r;
+            if (first && active && d < active_cap) active[1 + d] = e;
+        }
+        const unsigned firsts = __ballot_sync(0xffffffffu, first);
+        if (lane == 0 && active) active[0] = __popc(firsts);
+    }
+    __syncthreads();
+    for (int e = tid; e <= E; e += blockDim.x) {
+        int c = 0;
+        for (int q = 0; q < n; ++q) {
+            const int f = ids_s[q];
+            c += f >= 0 && f < e;
+        }
+        offsets[e] = c;
+    }
+}
+
 // General path, step 1: per-chunk counts (chunk c = pairs [c*P, (c+1)*P)).
 __global__ void k_permute_count(const int32_t *__restrict__ ids, int n, int E, int P, int32_t *__restrict__ cc,
                                 unsigned *err) {
@@ -153,7 +209,7 @@ static constexpr int kChunkPairs = 1024;
 
 size_t permute_ws_bytes(int T, int k, int E) {
     const long n = static_cast<long>(T) * k;
-    if (n <= kSmallPairs && E <= kSmallE) return 0;
+    if (n <= kSparsePairs || (n <= kSmallPairs && E <= kSmallE)) return 0;
     const long C = (n + kChunkPairs - 1) / kChunkPairs;
     return static_cast<size_t>((C + 1) * E) * sizeof(int32_t);
 }
@@ -162,6 +218,11 @@ int launch_permute(const int32_t *ids, int T, int k, int E, int32_t *offsets, in
                    int32_t *perm_dst, int32_t *active, void *ws, unsigned *err, cudaStream_t s) {
     const int n = T * k;
     const int active_cap = n < E ? n : E;
+    if (n <= kSparsePairs) {
+        k_permute_sparse<<<1, 1024, 0, s>>>(ids, n, k, E, offsets, perm_src, perm_dst, active, active_cap, err);
+        count_launches(1);
+        return cuda_status(cudaGetLastError(), "permute launch");
+    }
     if (n <= kSmallPairs && E <= kSmallE) {
         const size_t smem = static_cast<size_t>(E) * sizeof(int32_t);
         cudaFuncSetAttribute(k_permute_small, cudaFuncAttributeMaxDynamicSharedMemorySize, 32768 * 4);

@@ -86,52 +86,67 @@ __global__ void __launch_bounds__(256) k_topk_warp(const float *__restrict__ log
     write_gates(lane, k, my_v, my_id, ids + static_cast<size_t>(t) * k, w + static_cast<size_t>(t) * k, err);
 }
 
-// One 1024-thread block per token, E <= 1024 * NPT.  32-bit value keys are
-// kept in registers; the id half of the selection key is rebuilt on the fly.
-template <int NPT>
-__global__ void __launch_bounds__(1024) k_topk_block(const float *__restrict__ logits, int T, int E, int k,
-                                                      int32_t *__restrict__ ids, float *__restrict__ w,
-                                                      unsigned *err) {
-    __shared__ uint64_t red[32];
-    __shared__ uint64_t chosen[32];
-    const int t = blockIdx.x;
-    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-    const float *l = logits + static_cast<size_t>(t) * E;
-    uint32_t vkey[NPT];
-#pragma unroll
-    for (int i = 0; i < NPT; ++i) {
-        int e = threadIdx.x + 1024 * i;
-        vkey[i] = e < E ? float_key(l[e]) : 0u;
-    }
-    uint64_t last = ~0ull;
-    for (int j = 0; j < k; ++j) {
-        uint64_t m = 0ull;
-#pragma unroll
-        for (int i = 0; i < NPT; ++i) {
-            int e = threadIdx.x + 1024 * i;
-            uint64_t c = e < E ? ((static_cast<uint64_t>(vkey[i]) << 32) |
-                                  static_cast<uint32_t>(0xffffffffu - static_cast<uint32_t>(e)))
-                               : 0ull;
-            c = c < last ? c : 0ull;
-            m = c > m ? c : m;
+// E > 1024: the logits split into chunks of kTopkChunk; one 256-thread CTA
+// per (token, chunk) selects the chunk's best k (block_topk_merge) and writes
+// them, as selection keys re-based to global ids, to the workspace; then one
+// warp per token merges the sorted chunk lists (lane c holds the head of
+// chunk c's list; each round the best head wins and its lane reads on).  The
+// whole GPU shares the selection instead of one SM scanning every logit k
+// times.  Keys of missing entries (a chunk shorter than k) are 0, below every
+// real key.
+constexpr int kTopkChunk = 2048;
+
+__global__ void __launch_bounds__(256) k_topk_chunk(const float *__restrict__ logits, int E, int k,
+                                                    uint64_t *__restrict__ cand) {
+    __shared__ uint64_t c_s[8 * 32], sel[32];
+    const int t = blockIdx.x, c = blockIdx.y, C = gridDim.y;
+    const int e0 = c * kTopkChunk;
+    const int n = min(kTopkChunk, E - e0);
+    block_topk_merge<8, kTopkChunk / 256>(logits + static_cast<size_t>(t) * E + e0, n, k, c_s, sel);
+    if (threadIdx.x < k) {
+        uint64_t key = sel[threadIdx.x];
+        if (key) {
+            const uint32_t local = 0xffffffffu - static_cast<uint32_t>(key);
+            key = (key & 0xffffffff00000000ull) | (0xffffffffu - (local + static_cast<uint32_t>(e0)));
         }
-        m = shfl_max64(m);
-        if (lane == 0) red[wid] = m;
-        __syncthreads();
-        if (wid == 0) {
-            uint64_t v = red[lane];
-            v = shfl_max64(v);
-            if (lane == 0) chosen[j] = v;
+        cand[(static_cast<size_t>(t) * C + c) * k + threadIdx.x] = key;
+    }
+}
+
+__global__ void __launch_bounds__(32) k_topk_merge_chunks(const uint64_t *__restrict__ cand, int C, int k,
+                                                          int32_t *__restrict__ ids, float *__restrict__ w,
+                                                          unsigned *err) {
+    const int t = blockIdx.x, lane = threadIdx.x;
+    const uint64_t *cl = cand + static_cast<size_t>(t) * C * k;
+    int pos = 0;
+    uint64_t head = lane < C ? cl[static_cast<size_t>(lane) * k] : 0ull, mine = 0ull;
+    for (int r = 0; r < k; ++r) {
+        const uint32_t hv = static_cast<uint32_t>(head >> 32);
+        const uint32_t hi = __reduce_max_sync(0xffffffffu, hv);
+        const unsigned tied = __ballot_sync(0xffffffffu, hv == hi);
+        int winner;
+        if (__popc(tied) == 1) {
+            winner = __ffs(tied) - 1;
+        } else {
+            const uint32_t lo = __reduce_max_sync(0xffffffffu, hv == hi ? static_cast<uint32_t>(head) : 0u);
+            winner = __ffs(__ballot_sync(0xffffffffu, hv == hi && static_cast<uint32_t>(head) == lo)) - 1;
         }
-        __syncthreads();
-        last = chosen[j];
+        const uint64_t won = __shfl_sync(0xffffffffu, head, winner);
+        if (lane == r) mine = won;
+        if (lane == winner) {
+            ++pos;
+            head = pos < k ? cl[static_cast<size_t>(lane) * k + pos] : 0ull;
+        }
     }
-    if (wid == 0) {
-        uint64_t m = lane < k ? chosen[lane] : 0ull;
-        float my_v = key_float(static_cast<uint32_t>(m >> 32));
-        int my_id = static_cast<int>(0xffffffffu - static_cast<uint32_t>(m));
-        write_gates(lane, k, my_v, my_id, ids + static_cast<size_t>(t) * k, w + static_cast<size_t>(t) * k, err);
-    }
+    const float my_v = key_float(static_cast<uint32_t>(mine >> 32));
+    const int my_id = static_cast<int>(0xffffffffu - static_cast<uint32_t>(mine));
+    write_gates(lane, k, my_v, my_id, ids + static_cast<size_t>(t) * k, w + static_cast<size_t>(t) * k, err);
+}
+
+size_t topk_chunk_ws_offset(int T, int E) { return (static_cast<size_t>(T) * E * sizeof(float) + 255) / 256 * 256; }
+
+size_t topk_chunk_ws_bytes(int T, int E, int k) {
+    return static_cast<size_t>(T) * ((E + kTopkChunk - 1) / kTopkChunk) * k * sizeof(uint64_t);
 }
 
 // ------------------------------------------------------------- launchers
@@ -166,7 +181,7 @@ void launch_router_logits(const void *x, int x_dtype, const void *w, int w_dtype
         launch_logits_t<float, float>(x, w, bias, T, H, E, out, s);
 }
 
-void launch_topk(const float *logits, int T, int E, int k, int32_t *ids, float *w, unsigned *err,
+void launch_topk(const float *logits, int T, int E, int k, int32_t *ids, float *w, unsigned *err, void *cand_ws,
                  cudaStream_t s) {
     if (E <= 1024) {
         const int threads = 256, per = threads / 32;
@@ -176,9 +191,11 @@ void launch_topk(const float *logits, int T, int E, int k, int32_t *ids, float *
         else if (E <= 512) { k_topk_warp<16><<<blocks, threads, 0, s>>>(logits, T, E, k, ids, w, err); count_launches(1); }
         else { k_topk_warp<32><<<blocks, threads, 0, s>>>(logits, T, E, k, ids, w, err); count_launches(1); }
     } else {
-        if (E <= 8192) { k_topk_block<8><<<T, 1024, 0, s>>>(logits, T, E, k, ids, w, err); count_launches(1); }
-        else if (E <= 16384) { k_topk_block<16><<<T, 1024, 0, s>>>(logits, T, E, k, ids, w, err); count_launches(1); }
-        else { k_topk_block<32><<<T, 1024, 0, s>>>(logits, T, E, k, ids, w, err); count_launches(1); }
+        const int C = (E + kTopkChunk - 1) / kTopkChunk;            // <= 16 for E <= 32768
+        uint64_t *cand = static_cast<uint64_t *>(cand_ws);
+        k_topk_chunk<<<dim3(T, C), 256, 0, s>>>(logits, E, k, cand);
+        k_topk_merge_chunks<<<T, 32, 0, s>>>(cand, C, k, ids, w, err);
+        count_launches(2);
     }
 }
 

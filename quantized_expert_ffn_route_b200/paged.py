@@ -65,7 +65,8 @@ class PagedExpertStack:
         from . import moe_combine, moe_expert_ffn_q2, moe_expert_ffn_q4, moe_permute, moe_route_topk
         b, k, El, H, I = self.b, self.k, self.El, self.H, self.I
         s = torch.cuda.current_stream() if stream is None else stream
-        moe_route_topk(None, 0, None, 0, logits, None, 1, H, El, k, b.ids, b.w, stream=s)
+        moe_route_topk(None, 0, None, 0, logits, None, 1, H, El, k, b.ids, b.w, None, b.ws_route, b.sizes["route"],
+                       stream=s)
         moe_permute(b.ids, 1, k, El, b.offsets, b.perm_src, b.perm_dst, b.active, b.ws_perm, b.sizes["perm"],
                     stream=s)
         self.ids_h.copy_(b.ids[:k], non_blocking=True)
@@ -96,4 +97,66 @@ class PagedExpertStack:
         moe_combine(b.y_perm, b.perm_dst, b.w, None, 1, k, H, y, stream=s)
         if self.record:
             self.events.append((gids, hit, slot, victim, pf, pf_slot, pf_victim))
+        return y
+
+
+class DevicePagedExpertStack:
+    """The same L x E_l stack with device-initiated staging (devcache_*): a
+    layer step enqueues route -> permute -> the policy kernel (reading the
+    selected ids where the router left them) -> the FFN of the hits and of
+    experts computed in place from the host pool -> devcache_join (the copy
+    kernel of the admitted misses) -> the FFN of the admitted misses ->
+    combine, with no host synchronisation, so whole tokens can be enqueued
+    back to back or captured in a CUDA graph.
+
+    pool: page-locked (mapped) host tensor [L * E_l * stride] uint8; slab:
+    device [capacity * stride]; table: device int64 [L * E_l].  admit_min > 1
+    computes a missed expert used fewer than admit_min times in place instead
+    of admitting it.  log_steps > 0 keeps that many steps of events on the
+    device (DevCache.events).
+    """
+
+    def __init__(self, layers, experts_per_layer, bits, H, I, k, pool, slab, table, capacity, blob_bytes, stride,
+                 decay_period=256, admit_min=0, log_steps=0, device="cuda"):
+        import torch
+        from . import DEVCACHE_ACT_INTS, MOE_MODE_GEMV, DevCache, alloc_step_buffers
+        self.L, self.El, self.bits, self.H, self.I, self.k = layers, experts_per_layer, bits, H, I, k
+        self.pool, self.slab, self.table = pool, slab, table
+        self.cache = DevCache(layers * experts_per_layer, capacity, blob_bytes, stride, pool, slab, table,
+                              decay_period, admit_min, log_steps)
+        self.dev = torch.device(device)
+        self.b = alloc_step_buffers(1, H, I, experts_per_layer, k, bits, MOE_MODE_GEMV, self.dev, False)
+        self.act = torch.zeros(DEVCACHE_ACT_INTS, dtype=torch.int32, device=self.dev)
+        self.copy_stream = torch.cuda.Stream(device=self.dev)
+        self.ids_log = None                 # optional device int32 [steps, k]: each step's ids (local)
+        self.steps = 0
+
+    def close(self):
+        self.cache.close()
+
+    def layer_step(self, layer, x, x_dtype, logits, y_out=None, stream=None):
+        """One token through one layer: logits [E_l] fp32 device, x [H] device;
+        returns the output buffer (fp32 [H])."""
+        import torch
+        from . import MOE_MODE_GEMV, moe_combine, moe_expert_ffn_q2, moe_expert_ffn_q4, moe_permute, moe_route_topk
+        b, k, El, H, I = self.b, self.k, self.El, self.H, self.I
+        s = torch.cuda.current_stream() if stream is None else stream
+        moe_route_topk(None, 0, None, 0, logits, None, 1, H, El, k, b.ids, b.w, None, b.ws_route, b.sizes["route"],
+                       stream=s)
+        moe_permute(b.ids, 1, k, El, b.offsets, b.perm_src, b.perm_dst, b.active, b.ws_perm, b.sizes["perm"],
+                    stream=s)
+        if self.ids_log is not None:
+            with torch.cuda.stream(s):
+                self.ids_log[self.steps].copy_(b.ids[:k])
+        self.cache.stage(b.ids, k, self.act, id_base=layer * El, stream=s, copy_stream=self.copy_stream)
+        self.steps += 1
+        ffn = moe_expert_ffn_q4 if self.bits == 4 else moe_expert_ffn_q2
+        tview = self.table[layer * El:(layer + 1) * El]
+        ffn(tview, b.offsets, self.act[0:], b.perm_src, x, x_dtype, 1, k, H, I, El, None, b.y_perm, None,
+            MOE_MODE_GEMV, b.ws_ffn, b.sizes["ffn"], stream=s)   # hits and in-place experts, overlapping the copies
+        self.cache.join(stream=s)
+        ffn(tview, b.offsets, self.act[33:], b.perm_src, x, x_dtype, 1, k, H, I, El, None, b.y_perm, None,
+            MOE_MODE_GEMV, b.ws_ffn, b.sizes["ffn"], stream=s)   # the admitted misses
+        y = b.y if y_out is None else y_out
+        moe_combine(b.y_perm, b.perm_dst, b.w, None, 1, k, H, y, stream=s)
         return y

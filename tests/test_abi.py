@@ -19,7 +19,7 @@ ROOT = Path(__file__).resolve().parents[1]
 def _declared():
     src = M.HEADER.read_text()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    names = re.findall(r"\b((?:moe|expcache)_[a-z0-9_]+)\s*\(", src)
+    names = re.findall(r"\b((?:moe|expcache|devcache)_[a-z0-9_]+)\s*\(", src)
     return sorted(set(names))
 
 
@@ -30,7 +30,7 @@ def test_library_exports_every_declared_symbol():
     for n in names:
         assert hasattr(L, n), n
     out = subprocess.run(["nm", "-D", "--defined-only", str(M.LIB_PATH)], capture_output=True, text=True).stdout
-    exported = set(re.findall(r" T ((?:moe|expcache)_\w+)$", out, flags=re.M))
+    exported = set(re.findall(r" T ((?:moe|expcache|devcache)_\w+)$", out, flags=re.M))
     assert set(names) <= exported
     assert M.moe_version() == 100
 
@@ -164,7 +164,7 @@ def test_debug_build_exports_every_symbol_and_reports_its_flag():
     path = build_lib(debug=True)
     assert path.parent.name == "_build_debug"
     out = subprocess.run(["nm", "-D", "--defined-only", str(path)], capture_output=True, text=True).stdout
-    exported = set(re.findall(r" T ((?:moe|expcache)_\w+)$", out, flags=re.M))
+    exported = set(re.findall(r" T ((?:moe|expcache|devcache)_\w+)$", out, flags=re.M))
     assert set(_declared()) <= exported
     code = ("import quantized_expert_ffn_route_b200 as M; "
             "print(M.LIB_PATH.parent.name, M.lib().moe_build_flags(), M.MOE_BUILD_DEBUG)")
@@ -173,3 +173,23 @@ def test_debug_build_exports_every_symbol_and_reports_its_flag():
         r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, env=env, cwd=ROOT)
         assert r.returncode == 0, r.stderr
         assert r.stdout.split() == want.split()
+
+
+def test_devcache_rejects_bad_descriptors_on_the_host():
+    h = C.c_void_p()
+    L = M.lib()
+    assert L.devcache_create(None, C.byref(h)) == M.MOE_EINVAL
+    buf = np.zeros(4096, np.uint8)
+    p = buf.ctypes.data
+    bad = [
+        M.DevCacheDesc(10, 11, 1024, 1024, p, p, p, 0, 0, 0),      # capacity > n_experts
+        M.DevCacheDesc(10, 4, 1000, 1024, p, p, p, 0, 0, 0),       # blob_bytes not a multiple of 16
+        M.DevCacheDesc(10, 4, 1024, 1000, p, p, p, 0, 0, 0),       # stride not a multiple of 256
+        M.DevCacheDesc(10, 4, 1024, 1024, None, p, p, 0, 0, 0),    # no pool
+        M.DevCacheDesc(10, 4, 1024, 1024, p, p, p, -1, 0, 0),      # negative decay
+    ]
+    for d in bad:
+        assert L.devcache_create(C.byref(d), C.byref(h)) == M.MOE_EINVAL
+        assert h.value is None
+    assert L.devcache_stage(None, None, 0, 0, None, None, None) == M.MOE_EINVAL
+    assert L.devcache_join(None, None) == M.MOE_EINVAL

@@ -57,7 +57,9 @@ def test_topk_bit_exact(E, k, kind):
     ids_ref, w_ref, st = oracle.topk(l, k)
     ids = torch.empty(T * k, dtype=torch.int32, device="cuda")
     w = torch.empty(T * k, dtype=torch.float32, device="cuda")
-    M.moe_route_topk(None, 0, None, 0, _t(l), None, T, 0, E, k, ids, w)
+    wsb = M.moe_route_ws_size(T, E, k)                 # E > 1024: the chunked top-k's candidates
+    ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
+    M.moe_route_topk(None, 0, None, 0, _t(l), None, T, 0, E, k, ids, w, None, ws, wsb)
     err = M.moe_device_error(clear=True)
     assert np.array_equal(ids.cpu().numpy().reshape(T, k), ids_ref)
     if st == 0:
@@ -114,7 +116,8 @@ def test_router_ties_from_duplicate_rows(T):
 
 # ---------------------------------------------------------------- permute
 @pytest.mark.parametrize("T,k,E", [(1, 10, 512), (37, 10, 512), (500, 10, 512), (8192, 10, 512),
-                                   (3, 10, 24576), (2000, 3, 7), (1, 1, 1), (4096, 1, 32768)])
+                                   (3, 10, 24576), (2000, 3, 7), (1, 1, 1), (4096, 1, 32768),
+                                   (1, 10, 24576), (2, 16, 32768), (3, 11, 100)])
 def test_permute_bit_exact(T, k, E):
     rng = np.random.default_rng(T + 13 * k + E)
     ids = np.stack([rng.choice(E, size=k, replace=False) for _ in range(T)]).astype(np.int32)

@@ -342,6 +342,14 @@ int expcache_lookup(moe_expcache *c, const int32_t *ids_host, int n, int32_t *sl
 int expcache_stage(moe_expcache *c, const int32_t *ids_host, int n, moe_stream_t compute,
                    int32_t *hit_out, int32_t *slot_out, int32_t *victim_out);
 
+/* expcache_stage with the misses copied from caller-given page-locked host
+ * addresses (src_host[i] for ids_host[i]; entries of hits are ignored and may
+ * be NULL) instead of host_pool + id * slot_stride: the RAM tier of an
+ * expert store (expstore_fetch) feeding the cache.  A miss with a NULL
+ * source returns MOE_EINVAL before anything changes.  Not with use_staging. */
+int expcache_stage_from(moe_expcache *c, const int32_t *ids_host, int n, const void *const *src_host,
+                        moe_stream_t compute, int32_t *hit_out, int32_t *slot_out, int32_t *victim_out);
+
 /* Loads experts expected soon (the next layer's likely experts) without a
  * use: for each id of ids_host (-1 = none), in order, a resident id is left
  * alone; otherwise it enters the lowest free slot, else the slot of the
@@ -385,6 +393,55 @@ int expcache_copy_times(moe_expcache *c, const void *ref_event, float *start_ms,
 
 /* Test hook: the next `n` copies report failure before being issued (MOE_EIO). */
 int expcache_inject_copy_failures(moe_expcache *c, int n);
+
+/* ------------------------------------------------ NVMe tier (expert store)
+ * The third tier below the page-locked RAM pool: a file holding every expert
+ * blob (expert e at byte offset e * slot_stride), read on demand into a RAM
+ * tier of `ram_slots` slots of the caller's page-locked buffer (Strata
+ * article, section 2 item 2 and its three-tier summary: experts on SSD, the
+ * hot ones in RAM and VRAM; Janas-LLM page: experts read from NVMe per token
+ * with O_DIRECT into a RAM cache of capped size).  Host calls only.
+ * expstore_fetch makes the given experts resident in the RAM tier: the
+ * missing ones are read by io_threads threads in parallel (pread; with
+ * use_direct the file is opened O_DIRECT, so reads bypass the page cache --
+ * then slot_stride and ram_buffer must be 4096-byte aligned and each read is
+ * rounded up to whole 4096-byte blocks inside the slot), each taking the
+ * least recently fetched slot that holds none of the call's ids.  It returns
+ * once every read has landed.  A slot may be reused by the next fetch, so
+ * copies out of it (expcache_stage_from) must have completed before then
+ * (expcache_wait).  Calls on one store must not overlap.
+ */
+typedef struct moe_expstore moe_expstore;
+
+typedef struct {
+    const char *path;       /* the file of n_experts * slot_stride bytes (the last blob may end the file) */
+    int32_t n_experts;
+    int64_t blob_bytes;     /* bytes per expert */
+    int64_t slot_stride;    /* bytes between experts in the file and between RAM slots (multiple of 256) */
+    int32_t ram_slots;      /* experts the RAM tier holds */
+    void *ram_buffer;       /* host [ram_slots * slot_stride], page-locked, caller-owned */
+    int32_t io_threads;     /* concurrent reads, 1..64 */
+    int32_t use_direct;     /* 1: O_DIRECT */
+} moe_expstore_desc;
+
+typedef struct {
+    int64_t fetches, hits, reads, bytes_read, evictions;
+    double read_seconds;    /* wall time spent waiting for reads */
+} moe_expstore_stats;
+
+/* Opens the file.  MOE_EIO if it cannot be opened (O_DIRECT on a file system
+ * without it included), MOE_EINVAL if it is too short or the descriptor is bad. */
+int expstore_create(const moe_expstore_desc *d, moe_expstore **out);
+void expstore_destroy(moe_expstore *s);
+
+/* ids: n distinct experts (n <= 32 and <= ram_slots, else MOE_EINVAL /
+ * MOE_EBUSY).  ram_ptrs_out[i] (optional): id i's address in the RAM tier;
+ * hit_out[i] (optional): 1 if it was already there.  A failed read returns
+ * MOE_EIO (that expert's pointer is NULL; the others are valid). */
+int expstore_fetch(moe_expstore *s, const int32_t *ids, int n, void **ram_ptrs_out, int8_t *hit_out);
+int expstore_stats(moe_expstore *s, moe_expstore_stats *out);
+/* Host copy of each expert's RAM slot (-1 = on the drive only), n_experts entries. */
+int expstore_snapshot(moe_expstore *s, int32_t *slot_of_out);
 
 /* ------------------------------------------ device-initiated expert staging
  * The expert cache's policy and copies on the GPU (Strata article, section 2

@@ -66,6 +66,17 @@ class DevCacheStats(C.Structure):
                 ("in_place", C.c_int64), ("bytes_copied", C.c_int64), ("bad_steps", C.c_int64)]
 
 
+class ExpStoreDesc(C.Structure):
+    _fields_ = [("path", C.c_char_p), ("n_experts", C.c_int32), ("blob_bytes", C.c_int64),
+                ("slot_stride", C.c_int64), ("ram_slots", C.c_int32), ("ram_buffer", C.c_void_p),
+                ("io_threads", C.c_int32), ("use_direct", C.c_int32)]
+
+
+class ExpStoreStats(C.Structure):
+    _fields_ = [("fetches", C.c_int64), ("hits", C.c_int64), ("reads", C.c_int64), ("bytes_read", C.c_int64),
+                ("evictions", C.c_int64), ("read_seconds", C.c_double)]
+
+
 DEVCACHE_ACT_INTS = 66          # two active-expert lists: [0] n_a, [1..32] ids; [33] n_b, [34..65] ids
 DEVCACHE_HIT, DEVCACHE_MISS, DEVCACHE_IN_PLACE = 1, 0, 3
 
@@ -116,6 +127,12 @@ def lib():
         "expcache_inject_copy_failures": (I, [P, I]),
         "expcache_copy_times": (I, [P, P, C.POINTER(C.c_float), C.POINTER(C.c_float)]),
         "expcache_prefetch": (I, [P, P, I, S, P, P, C.POINTER(C.c_int)]),
+        "expcache_stage_from": (I, [P, P, I, P, S, P, P, P]),
+        "expstore_create": (I, [C.POINTER(ExpStoreDesc), C.POINTER(P)]),
+        "expstore_destroy": (None, [P]),
+        "expstore_fetch": (I, [P, P, I, P, P]),
+        "expstore_stats": (I, [P, C.POINTER(ExpStoreStats)]),
+        "expstore_snapshot": (I, [P, P]),
         "devcache_create": (I, [C.POINTER(DevCacheDesc), C.POINTER(P)]),
         "devcache_destroy": (None, [P]),
         "devcache_stage": (I, [P, P, I, C.c_int32, P, S, S]),
@@ -303,6 +320,19 @@ class ExpCache:
         _check(lib().expcache_stage(self.h, _p(ids), ids.size, _stream(stream), _p(hit), _p(slot), _p(victim)))
         return hit, slot, victim
 
+    def stage_from(self, ids, srcs, stream=None):
+        """stage() with the misses copied from the given page-locked host
+        addresses (srcs[i] for ids[i]; 0 for hits); returns (hit, slot, victim)."""
+        import numpy as np
+        ids = np.ascontiguousarray(ids, dtype=np.int32)
+        src = np.ascontiguousarray(srcs, dtype=np.uint64)
+        hit = np.empty(ids.size, np.int32)
+        slot = np.empty(ids.size, np.int32)
+        victim = np.empty(ids.size, np.int32)
+        _check(lib().expcache_stage_from(self.h, _p(ids), ids.size, _p(src), _stream(stream), _p(hit), _p(slot),
+                                         _p(victim)))
+        return hit, slot, victim
+
     def prefetch(self, ids, stream=None):
         """Loads the given experts (-1 = none) without a use; returns (slot, victim, admitted)."""
         import numpy as np
@@ -405,3 +435,48 @@ class DevCache:
         slot = np.empty(self.n_experts, np.int32)
         _check(lib().devcache_snapshot(self.h, _p(cnt), _p(slot)))
         return cnt, slot
+
+
+class ExpStore:
+    """Handle around the expstore_* calls: expert blobs in a file, read on
+    demand into a RAM tier (the caller owns the page-locked ram_buffer)."""
+
+    def __init__(self, path, n_experts, blob_bytes, slot_stride, ram_slots, ram_buffer, io_threads=8,
+                 use_direct=False):
+        d = ExpStoreDesc(str(path).encode(), n_experts, blob_bytes, slot_stride, ram_slots, _p(ram_buffer),
+                         io_threads, 1 if use_direct else 0)
+        h = C.c_void_p()
+        _check(lib().expstore_create(C.byref(d), C.byref(h)))
+        self.h = h
+        self.n_experts = n_experts
+
+    def close(self):
+        if self.h:
+            lib().expstore_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def fetch(self, ids):
+        """Makes the experts resident in RAM; returns (addresses uint64, hit int8)."""
+        import numpy as np
+        ids = np.ascontiguousarray(ids, dtype=np.int32)
+        ptrs = np.zeros(ids.size, np.uint64)
+        hit = np.zeros(ids.size, np.int8)
+        _check(lib().expstore_fetch(self.h, _p(ids), ids.size, _p(ptrs), _p(hit)))
+        return ptrs, hit
+
+    def stats(self) -> dict:
+        st = ExpStoreStats()
+        _check(lib().expstore_stats(self.h, C.byref(st)))
+        return {f: getattr(st, f) for f, _ in ExpStoreStats._fields_}
+
+    def snapshot(self):
+        import numpy as np
+        slot = np.empty(self.n_experts, np.int32)
+        _check(lib().expstore_snapshot(self.h, _p(slot)))
+        return slot

@@ -5,6 +5,8 @@
 
 namespace moe {
 
+constexpr int kCombineBatch = 8;
+
 __global__ void __launch_bounds__(256) k_combine(const float *__restrict__ y_perm, const int32_t *__restrict__ perm_dst,
                                                   const float *__restrict__ w, const float *__restrict__ y_shared,
                                                   int T, int k, int H, float *__restrict__ y, unsigned *err) {
@@ -14,18 +16,33 @@ __global__ void __launch_bounds__(256) k_combine(const float *__restrict__ y_per
          i += static_cast<long>(gridDim.x) * blockDim.x) {
         const int t = static_cast<int>(i / h4n), h4 = static_cast<int>(i % h4n);
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int j = 0; j < k; ++j) {
-            const float g = w[static_cast<size_t>(t) * k + j];
-            const int r = perm_dst[static_cast<size_t>(t) * k + j];
-            if (r < 0 || r >= T * k) {          // never read outside y_perm
-                report(err, MOE_DEVERR_BAD_ROW);
-                continue;
+        // kCombineBatch slots at a time: their rows and gates, then their rows'
+        // values, each batch's loads in flight together (summed in slot order)
+        for (int j0 = 0; j0 < k; j0 += kCombineBatch) {
+            int rr[kCombineBatch];
+            float gg[kCombineBatch];
+#pragma unroll
+            for (int u = 0; u < kCombineBatch; ++u) {
+                const int j = j0 + u;
+                rr[u] = j < k ? perm_dst[static_cast<size_t>(t) * k + j] : -1;
+                gg[u] = j < k ? w[static_cast<size_t>(t) * k + j] : 0.f;
             }
-            const float4 v = reinterpret_cast<const float4 *>(y_perm + static_cast<size_t>(r) * H)[h4];
-            acc.x = fmaf(g, v.x, acc.x);
-            acc.y = fmaf(g, v.y, acc.y);
-            acc.z = fmaf(g, v.z, acc.z);
-            acc.w = fmaf(g, v.w, acc.w);
+            float4 v[kCombineBatch];
+#pragma unroll
+            for (int u = 0; u < kCombineBatch; ++u) {
+                const bool ok = rr[u] >= 0 && rr[u] < T * k;   // never read outside y_perm
+                if (j0 + u < k && !ok) report(err, MOE_DEVERR_BAD_ROW);
+                v[u] = ok ? reinterpret_cast<const float4 *>(y_perm + static_cast<size_t>(rr[u]) * H)[h4]
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+            for (int u = 0; u < kCombineBatch; ++u) {
+                if (j0 + u >= k || rr[u] < 0 || rr[u] >= T * k) continue;
+                acc.x = fmaf(gg[u], v[u].x, acc.x);
+                acc.y = fmaf(gg[u], v[u].y, acc.y);
+                acc.z = fmaf(gg[u], v[u].z, acc.z);
+                acc.w = fmaf(gg[u], v[u].w, acc.w);
+            }
         }
         if (y_shared) {
             const float4 v = reinterpret_cast<const float4 *>(y_shared + static_cast<size_t>(t) * H)[h4];

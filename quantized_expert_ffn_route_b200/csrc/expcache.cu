@@ -78,6 +78,7 @@ static void destroy_events(moe_expcache *c) {
 // the cache again.
 struct PendingCopy {
     int32_t id, slot;
+    const uint8_t *src;                                // NULL: the pool entry of id
 };
 
 static int issue_copies(moe_expcache *c, const PendingCopy *copies, int nc, TablePatch &patch, moe_stream_t compute) {
@@ -94,7 +95,7 @@ static int issue_copies(moe_expcache *c, const PendingCopy *copies, int nc, Tabl
     int issued = 0;
     for (int i = 0; i < nc && !rc; ++i) {
         uint8_t *dst = slab + static_cast<size_t>(copies[i].slot) * S;
-        const uint8_t *src = pool + static_cast<size_t>(copies[i].id) * S;
+        const uint8_t *src = copies[i].src ? copies[i].src : pool + static_cast<size_t>(copies[i].id) * S;
         if (c->d.use_staging) {
             const int h = c->stage_next;
             c->stage_next ^= 1;
@@ -210,9 +211,8 @@ int expcache_lookup(moe_expcache *c, const int32_t *ids_host, int n, int32_t *sl
     return MOE_OK;
 }
 
-int expcache_stage(moe_expcache *c, const int32_t *ids_host, int n, moe_stream_t compute, int32_t *hit_out,
-                   int32_t *slot_out, int32_t *victim_out) {
-    moe::NvtxRange nvtx_range("expcache_stage");
+static int stage_impl(moe_expcache *c, const int32_t *ids_host, int n, const void *const *src_host,
+                      moe_stream_t compute, int32_t *hit_out, int32_t *slot_out, int32_t *victim_out) {
     REQUIRE(c && (n == 0 || ids_host), "cache/ids are NULL");
     REQUIRE(n >= 0 && n <= 32, "n must be in [0, 32]");
     if (n > c->d.capacity) {
@@ -225,6 +225,11 @@ int expcache_stage(moe_expcache *c, const int32_t *ids_host, int n, moe_stream_t
     }
     int n_miss = 0;
     for (int i = 0; i < n; ++i) n_miss += c->slot_of[ids_host[i]] < 0;
+    if (src_host) {
+        REQUIRE(!c->d.use_staging, "expcache_stage_from does not take a staging cache");
+        for (int i = 0; i < n; ++i)
+            REQUIRE(c->slot_of[ids_host[i]] >= 0 || src_host[i], "no source for missed expert %d", ids_host[i]);
+    }
     if (n_miss > 0 && c->inject_fail > 0) {   // test hook: fail before any state changes
         c->inject_fail--;
         set_error("injected staging-copy failure");
@@ -278,7 +283,7 @@ int expcache_stage(moe_expcache *c, const int32_t *ids_host, int n, moe_stream_t
             c->slot_of[e] = slot;
             c->expert_in[slot] = e;
             c->order.emplace(c->cnt[e], c->last[e], e);
-            copies[nc++] = PendingCopy{e, slot};
+            copies[nc++] = PendingCopy{e, slot, src_host ? static_cast<const uint8_t *>(src_host[i]) : nullptr};
             c->st.misses++;
         }
         if (hit_out) hit_out[i] = resident ? (c->inflight[e] ? 2 : 1) : 0;
@@ -289,6 +294,19 @@ int expcache_stage(moe_expcache *c, const int32_t *ids_host, int n, moe_stream_t
     c->st.steps++;
     c->step_ids.assign(ids_host, ids_host + n);
     return issue_copies(c, copies, nc, patch, compute);
+}
+
+int expcache_stage(moe_expcache *c, const int32_t *ids_host, int n, moe_stream_t compute, int32_t *hit_out,
+                   int32_t *slot_out, int32_t *victim_out) {
+    moe::NvtxRange nvtx_range("expcache_stage");
+    return stage_impl(c, ids_host, n, nullptr, compute, hit_out, slot_out, victim_out);
+}
+
+int expcache_stage_from(moe_expcache *c, const int32_t *ids_host, int n, const void *const *src_host,
+                        moe_stream_t compute, int32_t *hit_out, int32_t *slot_out, int32_t *victim_out) {
+    moe::NvtxRange nvtx_range("expcache_stage_from");
+    REQUIRE(src_host || n == 0, "src_host is NULL");
+    return stage_impl(c, ids_host, n, src_host, compute, hit_out, slot_out, victim_out);
 }
 
 int expcache_prefetch(moe_expcache *c, const int32_t *ids_host, int n, moe_stream_t compute, int32_t *slot_out,

@@ -99,9 +99,9 @@ __global__ void __launch_bounds__(1024) k_permute_small(const int32_t *__restric
 // Few pairs (n = T*k <= 32, e.g. one decode token) and any E: no counting
 // array over the experts.  Warp 0 holds the n ids; the row of a valid pair is
 // the number of valid pairs with a smaller id plus the earlier pairs with the
-// same id (the stable order), and each offset is the number of valid pairs
-// with a smaller id, counted directly -- O(E * n) comparisons spread over the
-// block instead of a scan over E counters.
+// same id (the stable order) -- its position in the sorted list of valid ids
+// -- and each offset is the number of valid pairs with a smaller id, found by
+// walking that sorted list alongside the thread's increasing experts.
 constexpr int kSparsePairs = 32;
 
 __global__ void __launch_bounds__(1024) k_permute_sparse(const int32_t *__restrict__ ids, int n, int k, int E,
@@ -110,7 +110,7 @@ __global__ void __launch_bounds__(1024) k_permute_sparse(const int32_t *__restri
                                                           int32_t *__restrict__ perm_dst,
                                                           int32_t *__restrict__ active, int active_cap,
                                                           unsigned *err) {
-    __shared__ int ids_s[kSparsePairs];
+    __shared__ int ids_s[kSparsePairs], sorted_s[kSparsePairs], nv_s;
     const int tid = threadIdx.x;
     if (tid < 32) {
         const int lane = tid;
@@ -136,19 +136,20 @@ __global__ void __launch_bounds__(1024) k_permute_sparse(const int32_t *__restri
         if (ok) {
             perm_src[r] = lane / k;
             perm_dst[lane] = r;
+            sorted_s[r] = e;
             if (first && active && d < active_cap) active[1 + d] = e;
         }
         const unsigned firsts = __ballot_sync(0xffffffffu, first);
+        const unsigned valid = __ballot_sync(0xffffffffu, ok);
         if (lane == 0 && active) active[0] = __popc(firsts);
+        if (lane == 0) nv_s = __popc(valid);
     }
     __syncthreads();
+    const int nv = nv_s;
+    int p = 0;                                           // sorted ids below e (e grows with each pass)
     for (int e = tid; e <= E; e += blockDim.x) {
-        int c = 0;
-        for (int q = 0; q < n; ++q) {
-            const int f = ids_s[q];
-            c += f >= 0 && f < e;
-        }
-        offsets[e] = c;
+        while (p < nv && sorted_s[p] < e) ++p;
+        offsets[e] = p;
     }
 }
 

@@ -27,14 +27,20 @@ class PagedExpertStack:
     prefetch: experts of the next layer to prefetch per layer (0 = none),
     chosen by the number of times each expert was selected so far (ties: the
     lower id).
+    store: an ExpStore (the NVMe tier) to read missed experts from, into its
+    RAM tier, before the cache copies them to HBM; pool is then only the
+    cache's nominal pool and prefetch must be 0.
     """
 
     def __init__(self, layers, experts_per_layer, bits, H, I, k, pool, slab, table, capacity, blob_bytes, stride,
-                 decay_period=256, prefetch=10, device="cuda"):
+                 decay_period=256, prefetch=10, device="cuda", store=None):
         import torch
         from . import MOE_MODE_GEMV, ExpCache, alloc_step_buffers
         self.L, self.El, self.bits, self.H, self.I, self.k = layers, experts_per_layer, bits, H, I, k
+        if store is not None and prefetch:
+            raise ValueError("prefetch copies from the pool; with an expert store it must be 0")
         self.prefetch_n = prefetch
+        self.store = store
         self.pool, self.slab, self.table = pool, slab, table
         self.cache = ExpCache(layers * experts_per_layer, capacity, blob_bytes, stride, pool, slab, table,
                               decay_period)
@@ -73,7 +79,18 @@ class PagedExpertStack:
         s.synchronize()                                   # the ids cross to the host
         local = self.ids_h.numpy().copy()
         gids = (local + layer * El).astype(np.int32)
-        hit, slot, victim = self.cache.stage(gids, stream=s)
+        if self.store is not None:                        # missed experts: drive -> RAM tier -> HBM
+            from . import MOE_OK
+            slots, _ = self.cache.lookup(gids)
+            srcs = np.zeros(gids.size, np.uint64)
+            if (slots < 0).any():
+                if self.cache.wait(10_000_000) != MOE_OK:   # copies out of RAM slots the fetch may reuse
+                    raise RuntimeError("expert copies did not finish within 10 s")
+                ptrs, _ = self.store.fetch(gids[slots < 0])
+                srcs[slots < 0] = ptrs
+            hit, slot, victim = self.cache.stage_from(gids, srcs, stream=s)
+        else:
+            hit, slot, victim = self.cache.stage(gids, stream=s)
         np.add.at(self.freq, gids, 1)
         # hit 1: resident and settled, computed at once; hit 2 (admitted by a
         # prefetch whose copy may still be in flight) and misses after the join
@@ -89,7 +106,10 @@ class PagedExpertStack:
                 1, b.ws_ffn, b.sizes["ffn"], stream=s)
         self.cache.join(stream=s)                         # the misses' and the prefetched experts' copies
         pf = self.predict((layer + 1) % self.L)            # the next layer (of this or the next token)
-        pf_slot, pf_victim, _ = self.cache.prefetch(pf, stream=s)
+        if self.prefetch_n > 0:
+            pf_slot, pf_victim, _ = self.cache.prefetch(pf, stream=s)
+        else:
+            pf_slot = pf_victim = np.full(pf.size, -1, np.int32)
         if miss.size:
             ffn(tview, b.offsets, self.act_d[32:], b.perm_src, x, x_dtype, 1, k, H, I, El, None, b.y_perm, None,
                 1, b.ws_ffn, b.sizes["ffn"], stream=s)

@@ -19,7 +19,7 @@ ROOT = Path(__file__).resolve().parents[1]
 def _declared():
     src = M.HEADER.read_text()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    names = re.findall(r"\b((?:moe|expcache|devcache)_[a-z0-9_]+)\s*\(", src)
+    names = re.findall(r"\b((?:moe|expcache|devcache|expstore)_[a-z0-9_]+)\s*\(", src)
     return sorted(set(names))
 
 
@@ -30,7 +30,7 @@ def test_library_exports_every_declared_symbol():
     for n in names:
         assert hasattr(L, n), n
     out = subprocess.run(["nm", "-D", "--defined-only", str(M.LIB_PATH)], capture_output=True, text=True).stdout
-    exported = set(re.findall(r" T ((?:moe|expcache|devcache)_\w+)$", out, flags=re.M))
+    exported = set(re.findall(r" T ((?:moe|expcache|devcache|expstore)_\w+)$", out, flags=re.M))
     assert set(names) <= exported
     assert M.moe_version() == 100
 
@@ -164,7 +164,7 @@ def test_debug_build_exports_every_symbol_and_reports_its_flag():
     path = build_lib(debug=True)
     assert path.parent.name == "_build_debug"
     out = subprocess.run(["nm", "-D", "--defined-only", str(path)], capture_output=True, text=True).stdout
-    exported = set(re.findall(r" T ((?:moe|expcache|devcache)_\w+)$", out, flags=re.M))
+    exported = set(re.findall(r" T ((?:moe|expcache|devcache|expstore)_\w+)$", out, flags=re.M))
     assert set(_declared()) <= exported
     code = ("import quantized_expert_ffn_route_b200 as M; "
             "print(M.LIB_PATH.parent.name, M.lib().moe_build_flags(), M.MOE_BUILD_DEBUG)")

@@ -587,11 +587,13 @@ def bench_paging(args, world, rank, pk):
     else:
         cache = M.ExpCache(E, cap, nb, stride, pool, slab, table, decay_period=256)
     n_steps = args.warmup + args.steps
-    trace = np.stack(list(W.paging_trace(W.SEED["paging"] + 17 * rank, E, k, n_steps + 64, s=c["zipf_s"],
+    # untimed steps after the timed ones: 64 for the overlap pass, then the end-to-end steps
+    n_more = 64 + (0 if args.no_e2e else min(args.steps, args.e2e_steps))
+    trace = np.stack(list(W.paging_trace(W.SEED["paging"] + 17 * rank, E, k, n_steps + n_more, s=c["zipf_s"],
                                          drift_every=c["drift_every"], drift_prob=c["drift_prob"],
                                          hot=c["hot"])))
     logits = torch.from_numpy(trace).cuda()
-    x_host = W.make_tokens(W.SEED["paging"] + 1, n_steps + 64, H, "bf16")
+    x_host = W.make_tokens(W.SEED["paging"] + 1, n_steps + n_more, H, "bf16")
     xs = torch.from_numpy(x_host.view(np.int16)).view(torch.bfloat16).cuda()
     b = stack.b if dev_mode else M.alloc_step_buffers(1, H, I, E, k, 2, M.MOE_MODE_GEMV, torch.device("cuda"),
                                                          False)
@@ -727,7 +729,7 @@ def bench_paging(args, world, rank, pk):
         barrier(world)
         a.record()
         for j in range(n_e2e):
-            i = n_steps + (j % 64)
+            i = n_steps + 64 + j                         # the trace goes on: fresh steps, as in the timed region
             xd.copy_(xh[i:i + 1], non_blocking=True)
             step(i, xd)
             yh.copy_(b.y[:H], non_blocking=True)
@@ -752,6 +754,140 @@ def bench_paging(args, world, rank, pk):
     if dev_mode:
         cfg["staging"] = "device-initiated" + (f", admit_min {args.admit_min}" if args.admit_min > 1 else "")
     roof["cache"] = {"misses": st1["misses"] - st0["misses"], "hits": st1["hits"] - st0["hits"]}
+    return dict(value=value, ms=ms, steps=args.steps, roofline=roof, e2e=e2e, cpu=cpu, clocks=clk,
+                launches=launches, config=cfg, dtype="fp32 (CUDA-core FMA on 2-bit codes)")
+
+
+def paging_ssd_config(E, k, nb, c, world):
+    """The `config` object of the three-tier workload (both arms print it)."""
+    return {"workload": f"paging_ssd: {E} experts (2-bit, {nb} B each, {E * nb / 1e9:.1f} GB) in a file read with "
+                        f"O_DIRECT into {c['ram_slots']} page-locked RAM slots, {c['hbm_slots']} HBM slots, "
+                        f"top-{k}, Zipf s={c['zipf_s']} with drift every {c['drift_every']} steps",
+            "tokens_per_step": 1, "l2": "weights paged from the drive and host RAM; HBM slots > L2",
+            "parallelism": f"replicas x{world}"}
+
+
+def bench_paging_ssd(args, world, rank, pk):
+    """Three tiers: the experts in a file on the local drive (read with
+    O_DIRECT by the store's I/O threads), a page-locked RAM tier, HBM slots."""
+    import tempfile
+    import torch
+    import quantized_expert_ffn_route_b200 as M
+    import workloads as W
+    from quantized_expert_ffn_route_b200.paged import PagedExpertStack
+    c = W.PAGING_SSD
+    E, k, H, I, cap, rs = c["E"], c["k"], c["H"], c["I"], c["hbm_slots"], c["ram_slots"]
+    base = W.make_layer(W.SEED["paging_ssd"], 2, H, I, 512, k, shared=False, w_dtype="bf16")
+    nb = M.moe_expert_blob_bytes(2, H, I)
+    stride = (nb + 4095) // 4096 * 4096
+    link = host_link_gbs()
+    fd, path = tempfile.mkstemp(prefix=f"moe_experts_r{rank}_", suffix=".bin", dir=args.ssd_dir)
+    try:
+        chunk = np.zeros((512, stride), np.uint8)
+        chunk[:, :nb] = base.blobs                       # 512 distinct blobs, repeated: only bytes moved matter
+        with os.fdopen(fd, "wb") as f:
+            for _ in range(E // 512):
+                f.write(chunk.tobytes())
+            f.flush()
+            os.fsync(f.fileno())
+        raw = torch.zeros(rs * stride + 4096, dtype=torch.uint8, pin_memory=True)
+        off = (-raw.data_ptr()) % 4096
+        ram = raw[off:off + rs * stride]
+        # the drive's own rate for this access pattern: 32 random experts per
+        # batch into an empty store of 32 slots, same threads, O_DIRECT
+        probe_ram = raw[off:off + 32 * stride]
+        probe = M.ExpStore(path, E, nb, stride, 32, probe_ram, io_threads=c["io_threads"], use_direct=True)
+        rng = np.random.default_rng(7)
+        t0 = time.perf_counter()
+        nbat = 16
+        for _ in range(nbat):
+            probe.fetch(rng.choice(E, 32, replace=False))
+        drive = nbat * 32 * stride / (time.perf_counter() - t0) / 1e9
+        probe.close()
+        store = M.ExpStore(path, E, nb, stride, rs, ram, io_threads=c["io_threads"], use_direct=True)
+        slab = torch.empty(cap * stride, dtype=torch.uint8, device="cuda")
+        table = torch.zeros(E, dtype=torch.int64, device="cuda")
+        stack = PagedExpertStack(1, E, 2, H, I, k, ram, slab, table, cap, nb, stride, decay_period=256, prefetch=0,
+                                 store=store)
+        n_steps = args.warmup + args.steps
+        n_more = max(64, 0 if args.no_e2e else min(args.steps, args.e2e_steps))
+        trace = np.stack(list(W.paging_trace(W.SEED["paging_ssd"] + 17 * rank, E, k, n_steps + n_more,
+                                             s=c["zipf_s"], drift_every=c["drift_every"],
+                                             drift_prob=c["drift_prob"], hot=c["hot"])))
+        logits = torch.from_numpy(trace).cuda()
+        x_host = W.make_tokens(W.SEED["paging_ssd"] + 1, n_steps + n_more, H, "bf16")
+        xs = torch.from_numpy(x_host.view(np.int16)).view(torch.bfloat16).cuda()
+
+        def step(i, x=None):
+            return stack.layer_step(0, xs[i:i + 1] if x is None else x, M.MOE_BF16, logits[i])
+
+        for i in range(args.warmup):
+            step(i)
+        torch.cuda.synchronize()
+        st0, ss0 = stack.cache.stats(), store.stats()
+        n0 = M.moe_kernel_launches()
+        clocks = ClockSampler(torch.cuda.current_device())
+        barrier(world)
+        a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for i in range(args.warmup, n_steps):
+            step(i)
+        z.record()
+        torch.cuda.synchronize()
+        barrier(world)
+        clk = clocks.stop()
+        launches = M.moe_kernel_launches() - n0
+        assert M.moe_device_error() == 0
+        ms = max_over_ranks(a.elapsed_time(z), world)
+        st1, ss1 = stack.cache.stats(), store.stats()
+        value = sum_over_ranks(args.steps, world) / (ms / 1e3)
+        read = ss1["bytes_read"] - ss0["bytes_read"]
+        hbm_miss = st1["misses"] - st0["misses"]
+        ram_hit = ss1["hits"] - ss0["hits"]
+        drive_ach = read / (ms / 1e3) / 1e9
+        roof = {"bound": "drive", "achieved": round(drive_ach, 3), "peak": round(drive, 3), "unit": "GB/s",
+                "frac": round(drive_ach / drive, 4), "traffic": None,
+                "kernel": "expstore_fetch (O_DIRECT preads by 8 threads into the RAM tier) + expcache_stage_from",
+                "peak_source": "O_DIRECT reads of 32 random experts per batch by the same threads, this run",
+                "host_link_gbs": round(link, 2),
+                "hbm_misses_per_step": round(hbm_miss / args.steps, 3),
+                "ram_hits_per_step": round(ram_hit / args.steps, 3),
+                "drive_reads_per_step": round((ss1["reads"] - ss0["reads"]) / args.steps, 3),
+                "read_wait_ms_per_step": round((ss1["read_seconds"] - ss0["read_seconds"]) * 1e3 / args.steps, 4)}
+        e2e = None
+        if not args.no_e2e:
+            n_e2e = min(args.steps, args.e2e_steps)
+            xh = torch.from_numpy(x_host.view(np.int16)).view(torch.bfloat16).pin_memory()
+            yh = torch.empty(H, dtype=torch.float32).pin_memory()
+            xd = torch.empty(1, H, dtype=torch.bfloat16, device="cuda")
+            s = torch.cuda.current_stream()
+            barrier(world)
+            a.record()
+            for j in range(n_e2e):
+                i = n_steps + j
+                xd.copy_(xh[i:i + 1], non_blocking=True)
+                y = step(i, xd)
+                yh.copy_(y[:H], non_blocking=True)
+                s.synchronize()
+            z.record()
+            torch.cuda.synchronize()
+            e_ms = max_over_ranks(a.elapsed_time(z), world)
+            e2e = {"value": round(sum_over_ranks(n_e2e, world) / (e_ms / 1e3), 1), "unit": "tokens/s",
+                   "h2d_bytes_per_step": H * 2, "d2h_bytes_per_step": H * 4 + k * 4, "steps": n_e2e}
+        stack.close()
+        store.close()
+    finally:
+        os.unlink(path)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        blob_list = [base.blobs[e % 512] for e in range(E)]
+
+        def ostep(n):
+            i = n % n_steps
+            oracle.moe_layer(2, x_host[i:i + 1], "bf16", blob_list, k=k, H=H, I=I, E=E, logits_in=trace[i:i + 1])
+        cpu = oracle_baseline(ostep, args.cpu_seconds, 2, 1, f"paging steps (1 token, 10 of {E} experts)")
+    cfg = paging_ssd_config(E, k, nb, c, world)
     return dict(value=value, ms=ms, steps=args.steps, roofline=roof, e2e=e2e, cpu=cpu, clocks=clk,
                 launches=launches, config=cfg, dtype="fp32 (CUDA-core FMA on 2-bit codes)")
 
@@ -1004,7 +1140,21 @@ def bench_reference(args, world, rank):
             one(i)
         dt = time.perf_counter() - t0
         return dict(value=args.steps / L / dt, ms=dt * 1e3, config=cfg, sample=sample)
-    if kind == "paging":
+    if kind == "paging_ssd":
+        c = W.PAGING_SSD
+        E, k, H, I = c["E"], c["k"], c["H"], c["I"]
+        base = W.make_layer(W.SEED["paging_ssd"], 2, H, I, 512, k, shared=False, w_dtype="bf16")
+        blob_list = [base.blobs[e % 512] for e in range(E)]
+        trace = np.stack(list(W.paging_trace(W.SEED["paging_ssd"], E, k, n, s=c["zipf_s"],
+                                             drift_every=c["drift_every"], drift_prob=c["drift_prob"],
+                                             hot=c["hot"])))
+        x = W.make_tokens(W.SEED["paging_ssd"] + 1, n, H, "bf16")
+
+        def one(i):
+            oracle.moe_layer(2, x[i:i + 1], "bf16", blob_list, k=k, H=H, I=I, E=E, logits_in=trace[i:i + 1])
+        cfg = paging_ssd_config(E, k, oracle.blob_bytes(2, H, I), c, world)
+        sample = f"1 paging step (1 token, 10 of {E} experts)"
+    elif kind == "paging":
         c = W.PAGING
         E, k, H, I, cap = c["E"], c["k"], c["H"], c["I"], c["capacity"]
         base = W.make_layer(W.SEED["paging"], 2, H, I, 512, k, shared=False, w_dtype="bf16")
@@ -1045,7 +1195,9 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--workload", default="decode", choices=["decode", "verify", "prefill", "paging", "paging48"])
+    ap.add_argument("--workload", default="decode",
+                    choices=["decode", "verify", "prefill", "paging", "paging48", "paging_ssd"])
+    ap.add_argument("--ssd-dir", default=None, help="paging_ssd: directory of the expert file (default: the temp dir)")
     ap.add_argument("--prefetch", type=int, default=-1, help="paging48: experts prefetched per layer (-1: config)")
     ap.add_argument("--device-staging", action="store_true",
                     help="paging, paging48: the cache policy and copies on the device (devcache_*)")
@@ -1092,6 +1244,8 @@ def main():
         r = bench_paging(args, world, rank, pk)
     elif args.workload == "paging48":
         r = bench_paging48(args, world, rank, pk)
+    elif args.workload == "paging_ssd":
+        r = bench_paging_ssd(args, world, rank, pk)
     else:
         r = bench_layer(args, world, rank, pk)
     if rank == 0:

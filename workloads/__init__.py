@@ -208,7 +208,14 @@ PAGING = dict(bits=2, H=2048, I=512, E=24576, k=10, capacity=2048, steps=5000,
 PAGING48 = dict(bits=2, H=2048, I=512, layers=48, experts_per_layer=512, k=10, capacity=2048, tokens=100,
                 drift_every=50, drift_prob=0.1, hot_per_layer=42, zipf_s=1.1, prefetch=10)
 
-SEED = {"tiny": 1001, "decode": 1002, "verify": 1003, "prefill": 1004, "paging": 1005, "paging48": 1006}
+# Three tiers: every expert in a file on the drive, the most used in a
+# page-locked RAM tier, the hottest in HBM (the pages' SSD -> RAM -> VRAM
+# picture at a size whose file a test box can write in seconds).
+PAGING_SSD = dict(bits=2, H=2048, I=512, E=4096, k=10, hbm_slots=512, ram_slots=1536, steps=2000,
+                  drift_every=200, drift_prob=0.1, hot=512, zipf_s=1.1, io_threads=8)
+
+SEED = {"tiny": 1001, "decode": 1002, "verify": 1003, "prefill": 1004, "paging": 1005, "paging48": 1006,
+        "paging_ssd": 1007}
 
 
 def tiny_case(seed: int = SEED["tiny"], **over):

@@ -251,6 +251,28 @@ int moe_layer_decode(int bits, const void *x, int x_dtype, const void *w_router,
                      float *topk_w, float *logits_out, float *y, void *ws, size_t ws_bytes,
                      moe_stream_t s);
 
+/* ------------------------------------------------------ decode session
+ * moe_layer_decode for a serving loop with host buffers: at creation the
+ * host->device copy of x_host, the fused step (router logits from w_router,
+ * top-k, experts, combine) and the device->host copies of y (and of the ids
+ * when ids_host is given) are recorded once into a CUDA graph on stream `s`
+ * (after one eager call that checks every argument as moe_layer_decode does
+ * and zero-fills ws); each moe_decode_session_run replays it and returns when
+ * y_host holds the step's output.  x_host [H] (x_dtype) and y_host [H] fp32
+ * (ids_host [k] int32 or NULL) are page-locked host buffers the caller
+ * fills / reads between runs; x_dev [H], ids_dev [k], w_dev [k], y_dev [H] and
+ * ws (moe_layer_decode_ws_size bytes) are device buffers; all stay owned by
+ * the caller and must outlive the session.  `s` must not be the legacy
+ * default stream.  Runs of one session must not overlap. */
+typedef struct moe_decode_session moe_decode_session;
+int moe_decode_session_create(int bits, const void *x_host, int x_dtype, const void *w_router, int w_dtype,
+                              const float *bias, const void *const *expert_blobs, const void *shared_blob,
+                              int H, int I, int E, int k, float *y_host, int32_t *ids_host, void *x_dev,
+                              int32_t *ids_dev, float *w_dev, float *y_dev, void *ws, size_t ws_bytes,
+                              moe_stream_t s, moe_decode_session **out);
+int moe_decode_session_run(moe_decode_session *ds);
+void moe_decode_session_destroy(moe_decode_session *ds);
+
 /* ------------------------------------------------- allocation-free FFN
  * The pages have no counterpart of this call; it serves callers that cannot
  * allocate device memory when they run the step: engines held to a device

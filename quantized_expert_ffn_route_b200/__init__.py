@@ -133,6 +133,10 @@ def lib():
         "expstore_fetch": (I, [P, P, I, P, P]),
         "expstore_stats": (I, [P, C.POINTER(ExpStoreStats)]),
         "expstore_snapshot": (I, [P, P]),
+        "moe_decode_session_create": (I, [I, P, I, P, I, P, P, P, I, I, I, I, P, P, P, P, P, P, P, Z, S,
+                                          C.POINTER(P)]),
+        "moe_decode_session_run": (I, [P]),
+        "moe_decode_session_destroy": (None, [P]),
         "devcache_create": (I, [C.POINTER(DevCacheDesc), C.POINTER(P)]),
         "devcache_destroy": (None, [P]),
         "devcache_stage": (I, [P, P, I, C.c_int32, P, S, S]),

@@ -150,6 +150,17 @@ class MoELayer:
                          b["w"], b["logits"], b["y"], b["ws"], b["ws_bytes"], stream)
         return b
 
+    def decode_session(self, x_host, x_dtype, y_host, stream, ids_host=None, bufs=None):
+        """A DecodeSession over page-locked host buffers x_host [H] (x_dtype)
+        and y_host [H] fp32 (ids_host [k] int32 optional): each run() copies x
+        in, runs the step and copies y back, replaying one CUDA graph recorded
+        on `stream` (a torch.cuda.Stream, not the default stream)."""
+        import torch
+        b = bufs or self.decode_buffers()
+        x_dev = torch.empty(self.H, dtype=torch.bfloat16 if x_host.dtype == torch.bfloat16 else torch.float32,
+                            device=self.device)
+        return DecodeSession(self, x_host, x_dtype, y_host, ids_host, x_dev, b, stream)
+
     def prepare_decode(self, x, x_dtype, stream=None, bufs=None):
         """A prepared one-token step on fixed buffers: every argument of
         moe_layer_decode is marshalled once, so each call of the returned
@@ -184,3 +195,34 @@ class MoELayer:
             b.y_shared, mode, b.ws_ffn, b.sizes["ffn"], stream)
         moe_combine(b.y_perm, b.perm_dst, b.w, b.y_shared, T, k, H, b.y, stream)
         return b
+
+
+class DecodeSession:
+    """Handle around moe_decode_session_* (keeps the buffers it records alive)."""
+
+    def __init__(self, layer, x_host, x_dtype, y_host, ids_host, x_dev, bufs, stream):
+        import ctypes as C
+        from . import _check, _p, lib
+        self._keep = (layer, x_host, y_host, ids_host, x_dev, bufs, stream)
+        h = C.c_void_p()
+        _check(lib().moe_decode_session_create(
+            layer.bits, _p(x_host), x_dtype, _p(layer.w_router), layer.w_dtype, _p(layer.bias), _p(layer.table),
+            _p(layer.shared), layer.H, layer.I, layer.E, layer.k, _p(y_host), _p(ids_host), _p(x_dev), _p(bufs["ids"]),
+            _p(bufs["w"]), _p(bufs["y"]), _p(bufs["ws"]), bufs["ws_bytes"], stream.cuda_stream, C.byref(h)))
+        self.h = h
+
+    def run(self):
+        from . import _check, lib
+        _check(lib().moe_decode_session_run(self.h))
+
+    def close(self):
+        from . import lib
+        if self.h:
+            lib().moe_decode_session_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

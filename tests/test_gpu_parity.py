@@ -652,3 +652,32 @@ def test_gemm_wait_timeout_recovers():
     for _ in range(2):
         out = run_gpu(g, x, "bf16", mode=M.MOE_MODE_GEMM)
         _check_layer(out, ref, layer, x, "bf16")
+
+
+def test_decode_session_matches_forward_decode():
+    """The decode session (x copied in, the step, y and ids copied out, one
+    recorded graph per call) gives forward_decode's output bit for bit, token
+    after token; it refuses the legacy default stream."""
+    layer = W.make_layer(450, 4, 256, 256, 24, 4, shared=True, w_dtype="bf16")
+    x = W.make_tokens(451, 5, 256, "bf16")
+    g = _layer_gpu(layer)
+    x_in = torch.empty(256, dtype=torch.bfloat16).pin_memory()
+    y_out = torch.empty(256, dtype=torch.float32).pin_memory()
+    ids_out = torch.empty(4, dtype=torch.int32).pin_memory()
+    s = torch.cuda.Stream()
+    sess = g.decode_session(x_in, M.MOE_BF16, y_out, s, ids_host=ids_out)
+    try:
+        for t in range(5):
+            x_in.copy_(torch.from_numpy(x[t].view(np.int16)).view(torch.bfloat16))
+            n0 = M.moe_kernel_launches()
+            sess.run()
+            assert M.moe_kernel_launches() - n0 == 3
+            ref = _run_fused(g, x[t:t + 1], "bf16")
+            assert ref["err"] == 0 and M.moe_device_error() == 0
+            assert np.array_equal(y_out.numpy(), ref["y"]) and np.array_equal(ids_out.numpy(), ref["ids"])
+    finally:
+        sess.close()
+    with pytest.raises(M.MoEError) as ei:
+        M.lib()                                               # the default stream cannot be captured
+        g.decode_session(x_in, M.MOE_BF16, y_out, torch.cuda.default_stream())
+    assert ei.value.status == M.MOE_EINVAL

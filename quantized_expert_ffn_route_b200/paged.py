@@ -122,8 +122,9 @@ class PagedExpertStack:
 
 class DevicePagedExpertStack:
     """The same L x E_l stack with device-initiated staging (devcache_*): a
-    layer step enqueues route -> permute -> the policy kernel (reading the
-    selected ids where the router left them) -> the FFN of the hits and of
+    layer step enqueues route -> the policy kernel (reading the selected ids
+    where the router left them; its copy kernel starts at once) -> permute ->
+    the FFN of the hits and of
     experts computed in place from the host pool -> devcache_join (the copy
     kernel of the admitted misses) -> the FFN of the admitted misses ->
     combine, with no host synchronisation, so whole tokens can be enqueued
@@ -163,13 +164,14 @@ class DevicePagedExpertStack:
         s = torch.cuda.current_stream() if stream is None else stream
         moe_route_topk(None, 0, None, 0, logits, None, 1, H, El, k, b.ids, b.w, None, b.ws_route, b.sizes["route"],
                        stream=s)
-        moe_permute(b.ids, 1, k, El, b.offsets, b.perm_src, b.perm_dst, b.active, b.ws_perm, b.sizes["perm"],
-                    stream=s)
         if self.ids_log is not None:
             with torch.cuda.stream(s):
                 self.ids_log[self.steps].copy_(b.ids[:k])
+        # the policy needs only the ids: its copies start before the permute, which only the FFN needs
         self.cache.stage(b.ids, k, self.act, id_base=layer * El, stream=s, copy_stream=self.copy_stream)
         self.steps += 1
+        moe_permute(b.ids, 1, k, El, b.offsets, b.perm_src, b.perm_dst, b.active, b.ws_perm, b.sizes["perm"],
+                    stream=s)
         ffn = moe_expert_ffn_q4 if self.bits == 4 else moe_expert_ffn_q2
         tview = self.table[layer * El:(layer + 1) * El]
         ffn(tview, b.offsets, self.act[0:], b.perm_src, x, x_dtype, 1, k, H, I, El, None, b.y_perm, None,

@@ -1099,7 +1099,7 @@ def paging_config(E, k, nb, cap, c, world):
 def workload_shape(kind, args):
     """(layer copies, FFN mode, fused) of a resident-layer workload as bench_layer runs it."""
     n_layers = args.layers or (2 if kind == "prefill" else 16)
-    mode = 2 if kind == "prefill" else 0
+    mode = {"gemv": 1, "gemm": 2}.get(getattr(args, "ffn_mode", "auto"), 2 if kind == "prefill" else 0)
     fused = kind == "decode" and not args.unfused
     return n_layers, mode, fused
 
@@ -1202,6 +1202,8 @@ def main():
                     choices=["decode", "verify", "prefill", "paging", "paging48", "paging_ssd"])
     ap.add_argument("--ssd-dir", default=None, help="paging_ssd: directory of the expert file (default: the temp dir)")
     ap.add_argument("--prefetch", type=int, default=-1, help="paging48: experts prefetched per layer (-1: config)")
+    ap.add_argument("--ffn-mode", default="auto", choices=["auto", "gemv", "gemm"],
+                    help="verify/prefill: the expert FFN mode (auto: GEMV up to 16 tokens, else the grouped GEMM)")
     ap.add_argument("--device-staging", action="store_true",
                     help="paging, paging48: the cache policy and copies on the device (devcache_*)")
     ap.add_argument("--admit-min", type=int, default=0,

@@ -722,6 +722,12 @@ def bench_paging(args, world, rank, pk):
     if dev_mode:
         roof["in_place_per_step"] = round(in_place / args.steps, 3)
         roof["admit_min"] = args.admit_min
+    else:
+        cache.wait(30_000_000)
+        bins, nh = cache.copy_histogram()
+        roof["copy_time_histogram"] = {"bins_log2_us": bins.tolist(), "steps": int(nh),
+                                       "definition": "steps whose copies (first issued -> table patched) took "
+                                                     "[2^i, 2^(i+1)) microseconds, all steps of this run"}
 
     e2e = None
     if not args.no_e2e:

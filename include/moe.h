@@ -413,6 +413,15 @@ int expcache_snapshot(moe_expcache *c, int64_t *counts_out, int32_t *slot_of_out
  * staged a copy.  Used to measure how much copy time compute hides. */
 int expcache_copy_times(moe_expcache *c, const void *ref_event, float *start_ms, float *end_ms);
 
+/* Histogram of the copy time of the steps that staged copies (first copy
+ * issued -> table patched, from events on the cache's stream): bins_out[i]
+ * (MOE_COPY_HIST_BINS entries) counts the steps whose copies took
+ * [2^i, 2^(i+1)) microseconds, bin 0 also everything shorter and the last bin
+ * everything longer.  A step is counted once its copies have completed (all
+ * are after expcache_wait); *steps_out (optional) = the steps counted. */
+#define MOE_COPY_HIST_BINS 24
+int expcache_copy_histogram(moe_expcache *c, int64_t *bins_out, int64_t *steps_out);
+
 /* Test hook: the next `n` copies report failure before being issued (MOE_EIO). */
 int expcache_inject_copy_failures(moe_expcache *c, int n);
 

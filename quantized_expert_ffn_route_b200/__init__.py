@@ -77,6 +77,7 @@ class ExpStoreStats(C.Structure):
                 ("evictions", C.c_int64), ("read_seconds", C.c_double)]
 
 
+MOE_COPY_HIST_BINS = 24
 DEVCACHE_ACT_INTS = 66          # two active-expert lists: [0] n_a, [1..32] ids; [33] n_b, [34..65] ids
 DEVCACHE_HIT, DEVCACHE_MISS, DEVCACHE_IN_PLACE = 1, 0, 3
 
@@ -128,6 +129,7 @@ def lib():
         "expcache_copy_times": (I, [P, P, C.POINTER(C.c_float), C.POINTER(C.c_float)]),
         "expcache_prefetch": (I, [P, P, I, S, P, P, C.POINTER(C.c_int)]),
         "expcache_stage_from": (I, [P, P, I, P, S, P, P, P]),
+        "expcache_copy_histogram": (I, [P, P, P]),
         "expstore_create": (I, [C.POINTER(ExpStoreDesc), C.POINTER(P)]),
         "expstore_destroy": (None, [P]),
         "expstore_fetch": (I, [P, P, I, P, P]),
@@ -376,6 +378,15 @@ class ExpCache:
 
     def inject_copy_failures(self, n: int):
         _check(lib().expcache_inject_copy_failures(self.h, n))
+
+    def copy_histogram(self):
+        """(bins int64 [MOE_COPY_HIST_BINS], steps): bin i counts the steps whose
+        copies took [2^i, 2^(i+1)) microseconds."""
+        import numpy as np
+        bins = np.zeros(MOE_COPY_HIST_BINS, np.int64)
+        n = C.c_int64(0)
+        _check(lib().expcache_copy_histogram(self.h, _p(bins), C.byref(n)))
+        return bins, n.value
 
     def copy_times(self, ref_event):
         """(start_ms, end_ms) of the last step's copies, measured from `ref_event`

@@ -50,6 +50,13 @@ struct moe_expcache {
     cudaEvent_t ev_stage[2] = {nullptr, nullptr};   // staging halves free again
     cudaEvent_t ev_t0 = nullptr, ev_t1 = nullptr;     // timed: start / end of the last step's copies
     bool timed = false;                               // ev_t0/ev_t1 have been recorded
+    // copy-time histogram: start/end events of the steps whose copies are not
+    // yet counted (a ring, oldest at ring_tail; the copy stream completes
+    // them in order)
+    static constexpr int kRing = 32;
+    cudaEvent_t ring0[kRing] = {}, ring1[kRing] = {};
+    int ring_tail = 0, ring_pending = 0;
+    int64_t hist[MOE_COPY_HIST_BINS] = {};
     int stage_next = 0;
     std::vector<int32_t> slot_of, expert_in;
     std::vector<int64_t> cnt, last;
@@ -69,6 +76,10 @@ static void destroy_events(moe_expcache *c) {
         if (e) cudaEventDestroy(e);
     if (c->ev_t0) cudaEventDestroy(c->ev_t0);
     if (c->ev_t1) cudaEventDestroy(c->ev_t1);
+    for (int i = 0; i < moe_expcache::kRing; ++i) {
+        if (c->ring0[i]) cudaEventDestroy(c->ring0[i]);
+        if (c->ring1[i]) cudaEventDestroy(c->ring1[i]);
+    }
     if (c->copy) cudaStreamDestroy(c->copy);
 }
 
@@ -81,6 +92,33 @@ struct PendingCopy {
     const uint8_t *src;                                // NULL: the pool entry of id
 };
 
+// Counts the timed steps whose copies have completed into the histogram
+// (bin i: [2^i, 2^(i+1)) microseconds, the first and last bins open-ended).
+// wait_oldest: block on the oldest pending step first (the ring is full).
+static int harvest_copy_times(moe_expcache *c, bool wait_oldest) {
+    while (c->ring_pending > 0) {
+        const int i = c->ring_tail;
+        if (wait_oldest) {
+            int rc = cuda_status(cudaEventSynchronize(c->ring1[i]), "copy timing wait");
+            if (rc) return rc;
+            wait_oldest = false;
+        } else {
+            const cudaError_t q = cudaEventQuery(c->ring1[i]);
+            if (q == cudaErrorNotReady) break;
+            if (q != cudaSuccess) return cuda_status(q, "copy timing query");
+        }
+        float ms = 0.f;
+        int rc = cuda_status(cudaEventElapsedTime(&ms, c->ring0[i], c->ring1[i]), "copy timing");
+        if (rc) return rc;
+        int bin = 0;
+        for (double us = ms * 1e3; us >= 2.0 && bin < MOE_COPY_HIST_BINS - 1; us /= 2.0) ++bin;
+        c->hist[bin]++;
+        c->ring_tail = (i + 1) % moe_expcache::kRing;
+        c->ring_pending--;
+    }
+    return MOE_OK;
+}
+
 static int issue_copies(moe_expcache *c, const PendingCopy *copies, int nc, TablePatch &patch, moe_stream_t compute) {
     if (nc == 0 && patch.n == 0) return MOE_OK;
     int rc = MOE_OK;
@@ -88,6 +126,11 @@ static int issue_copies(moe_expcache *c, const PendingCopy *copies, int nc, Tabl
         rc = cuda_status(cudaEventRecord(c->ev_compute, reinterpret_cast<cudaStream_t>(compute)), "event record");
         if (!rc) rc = cuda_status(cudaStreamWaitEvent(c->copy, c->ev_compute, 0), "stream wait");
         if (!rc) rc = cuda_status(cudaEventRecord(c->ev_t0, c->copy), "event record");
+        if (!rc) rc = harvest_copy_times(c, c->ring_pending == moe_expcache::kRing);
+        if (!rc) {
+            const int slot = (c->ring_tail + c->ring_pending) % moe_expcache::kRing;
+            rc = cuda_status(cudaEventRecord(c->ring0[slot], c->copy), "event record");
+        }
     }
     const size_t B = static_cast<size_t>(c->d.blob_bytes), S = static_cast<size_t>(c->d.slot_stride);
     auto *slab = static_cast<uint8_t *>(c->d.hbm_slab);
@@ -128,6 +171,11 @@ static int issue_copies(moe_expcache *c, const PendingCopy *copies, int nc, Tabl
     int rc2 = launch_table_patch(reinterpret_cast<const void **>(c->d.dev_table), patch, c->copy);
     if (!rc2) rc2 = cuda_status(cudaEventRecord(c->ev_done, c->copy), "event record");
     if (!rc2 && nc > 0) rc2 = cuda_status(cudaEventRecord(c->ev_t1, c->copy), "event record");
+    if (!rc2 && nc > 0) {
+        const int slot = (c->ring_tail + c->ring_pending) % moe_expcache::kRing;
+        rc2 = cuda_status(cudaEventRecord(c->ring1[slot], c->copy), "event record");
+        if (!rc2) c->ring_pending++;
+    }
     if (!rc2 && nc > 0) c->timed = true;
     return rc ? rc : rc2;
 }
@@ -161,6 +209,10 @@ int expcache_create(const moe_expcache_desc *d, moe_expcache **out) {
         rc = cuda_status(cudaEventCreateWithFlags(&c->ev_stage[i], cudaEventDisableTiming), "event");
     if (!rc) rc = cuda_status(cudaEventCreate(&c->ev_t0), "event");
     if (!rc) rc = cuda_status(cudaEventCreate(&c->ev_t1), "event");
+    for (int i = 0; i < moe_expcache::kRing && !rc; ++i) {
+        rc = cuda_status(cudaEventCreate(&c->ring0[i]), "event");
+        if (!rc) rc = cuda_status(cudaEventCreate(&c->ring1[i]), "event");
+    }
     if (!rc)
         rc = cuda_status(cudaMemsetAsync(d->dev_table, 0, sizeof(void *) * static_cast<size_t>(d->n_experts), c->copy),
                          "table clear");
@@ -373,6 +425,20 @@ int expcache_copy_times(moe_expcache *c, const void *ref_event, float *start_ms,
     int rc = cuda_status(cudaEventElapsedTime(start_ms, ref, c->ev_t0), "elapsed time");
     if (!rc) rc = cuda_status(cudaEventElapsedTime(end_ms, ref, c->ev_t1), "elapsed time");
     return rc;
+}
+
+int expcache_copy_histogram(moe_expcache *c, int64_t *bins_out, int64_t *steps_out) {
+    REQUIRE(c && bins_out, "cache/bins_out are NULL");
+    DeviceGuard guard(c->device);
+    int rc = harvest_copy_times(c, false);
+    if (rc) return rc;
+    int64_t n = 0;
+    for (int b = 0; b < MOE_COPY_HIST_BINS; ++b) {
+        bins_out[b] = c->hist[b];
+        n += c->hist[b];
+    }
+    if (steps_out) *steps_out = n;
+    return MOE_OK;
 }
 
 int expcache_join(moe_expcache *c, moe_stream_t s) {

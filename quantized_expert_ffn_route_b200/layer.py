@@ -154,7 +154,9 @@ class MoELayer:
         """A DecodeSession over page-locked host buffers x_host [H] (x_dtype)
         and y_host [H] fp32 (ids_host [k] int32 optional): each run() copies x
         in, runs the step and copies y back, replaying one CUDA graph recorded
-        on `stream` (a torch.cuda.Stream, not the default stream)."""
+        on `stream` (a torch.cuda.Stream, not the default stream).  Creation
+        runs the step once on x_host's current contents, so it should hold a
+        valid token (or the device error word may report it)."""
         import torch
         b = bufs or self.decode_buffers()
         x_dev = torch.empty(self.H, dtype=torch.bfloat16 if x_host.dtype == torch.bfloat16 else torch.float32,

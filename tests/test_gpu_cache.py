@@ -161,3 +161,34 @@ def test_cache_events_full_paging_trace():
         assert np.array_equal(cnt, ref["counts"])
     finally:
         cache.close()
+
+
+def test_cache_copy_time_histogram():
+    """Every step that staged copies is counted once in the copy-time
+    histogram after the copies complete -- more steps than the event ring
+    holds included -- and steps without misses are not counted."""
+    E, k, cap = 12, 2, 8                             # hits are common: some steps stage nothing
+    layer = W.make_layer(97, 2, 256, 128, E, k, shared=False, w_dtype="bf16")
+    cache, keep = _make_cache(layer, cap, 0)
+    rng = np.random.default_rng(3)
+    with_copies = 0
+    try:
+        for step in range(80):                       # more than the 32-entry ring
+            ids = rng.choice(E, k, replace=False)
+            hit, _, _ = cache.stage(ids)
+            with_copies += int((hit == 0).any())
+            if step % 10 == 9:
+                cache.join()
+        assert cache.wait(30_000_000) == M.MOE_OK
+        bins, n = cache.copy_histogram()
+        assert n == with_copies == int(bins.sum()) and 0 < n < 80
+        nz = np.nonzero(bins)[0]
+        assert nz.min() >= 1 and nz.max() <= 16       # between 2 us and 130 ms per step's copies
+        cache.stage(np.zeros(0, np.int32))           # an empty step: nothing to count
+        resident = np.nonzero(cache.snapshot()[1] >= 0)[0][:k].astype(np.int32)
+        hit, _, _ = cache.stage(resident)            # an all-hit step: nothing to count
+        assert (hit == 1).all()
+        assert cache.wait(30_000_000) == M.MOE_OK and cache.copy_histogram()[1] == n
+    finally:
+        torch.cuda.synchronize()
+        cache.close()

@@ -665,7 +665,10 @@ def test_decode_session_matches_forward_decode():
     y_out = torch.empty(256, dtype=torch.float32).pin_memory()
     ids_out = torch.empty(4, dtype=torch.int32).pin_memory()
     s = torch.cuda.Stream()
+    x_in.copy_(torch.from_numpy(x[0].view(np.int16)).view(torch.bfloat16))   # creation runs one step on x_in
     sess = g.decode_session(x_in, M.MOE_BF16, y_out, s, ids_host=ids_out)
+    torch.cuda.synchronize()
+    assert M.moe_device_error(clear=True) == 0
     try:
         for t in range(5):
             x_in.copy_(torch.from_numpy(x[t].view(np.int16)).view(torch.bfloat16))

@@ -18,6 +18,7 @@
 #include <chrono>
 #include <condition_variable>
 #include <cstring>
+#include <exception>
 #include <list>
 #include <mutex>
 #include <thread>
@@ -146,15 +147,26 @@ int expstore_create(const moe_expstore_desc *d, moe_expstore **out) {
                   d->n_experts, static_cast<long long>(need));
         return MOE_EINVAL;
     }
-    auto *s = new moe_expstore();
-    s->d = *d;
-    s->fd = fd;
-    s->read_bytes = rb;
-    s->slot_of.assign(d->n_experts, -1);
-    s->expert_in.assign(d->ram_slots, -1);
-    s->pos.resize(d->ram_slots);
-    for (int i = 0; i < d->ram_slots; ++i) s->pos[i] = s->lru.insert(s->lru.end(), i);
-    s->io = new IoPool(d->io_threads);
+    moe_expstore *s = nullptr;
+    try {
+        s = new moe_expstore();
+        s->d = *d;
+        s->fd = fd;
+        s->read_bytes = rb;
+        s->slot_of.assign(d->n_experts, -1);
+        s->expert_in.assign(d->ram_slots, -1);
+        s->pos.resize(d->ram_slots);
+        for (int i = 0; i < d->ram_slots; ++i) s->pos[i] = s->lru.insert(s->lru.end(), i);
+        s->io = new IoPool(d->io_threads);
+    } catch (const std::exception &ex) {          // out of memory, or threads that could not start
+        if (s) {
+            s->fd = -1;
+            expstore_destroy(s);
+        }
+        close(fd);
+        set_error("expert store: %s", ex.what());
+        return MOE_ENOMEM;
+    }
     *out = s;
     return MOE_OK;
 }

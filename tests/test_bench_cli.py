@@ -123,3 +123,27 @@ def test_oracle_baseline_adds_a_one_thread_run():
     assert one["cores"] == 1 and one["value"] > 0 and "1 thread" in one["sample"]
     assert 1 in calls and bench.host_cores() in calls           # both runs used their thread count
     assert oracle.max_threads() == bench.host_cores()            # restored afterwards
+
+
+def test_reference_arm_of_the_three_tier_workload():
+    """The reference arm runs the oracle on the three-tier workload's steps and
+    prints the same `config` the measured arm builds."""
+    import bench
+    import workloads as W
+    out = subprocess.run([sys.executable, str(ROOT / "bench.py"), "--impl", "reference", "--workload", "paging_ssd",
+                          "--steps", "1", "--warmup", "1"], capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert out.returncode == 0, out.stderr
+    d = json.loads([l for l in out.stdout.splitlines() if l.strip()][-1])
+    c = W.PAGING_SSD
+    assert d["impl"] == "reference" and d["value"] > 0
+    assert d["config"] == bench.paging_ssd_config(c["E"], c["k"], 983040, c, 1)
+    assert "4096 experts" in d["config"]["workload"] and "O_DIRECT" in d["config"]["workload"]
+
+
+def test_ffn_mode_override():
+    import argparse
+    import bench
+    for name, want in (("auto", 0), ("gemv", 1), ("gemm", 2)):
+        args = argparse.Namespace(layers=0, unfused=False, ffn_mode=name)
+        assert bench.workload_shape("verify", args)[1] == want
+    assert bench.workload_shape("prefill", argparse.Namespace(layers=0, unfused=False, ffn_mode="auto"))[1] == 2

@@ -96,36 +96,6 @@ __device__ __forceinline__ void warp_take(uint64_t (&keys)[N], int k, int lane, 
     }
 }
 
-// Top-k (k <= 32) of E <= 1024 logits by one block of NW warps: each warp
-// takes the k best of its keys, then warp 0 the k best of the NW*k
-// candidates.  sel[0..k-1] receives the selection keys in rank order.
-template <int NW>
-__device__ void block_topk(const float *logits, int E, int k, uint64_t *cand, uint64_t *sel) {
-    constexpr int KPT = 1024 / (32 * NW);            // keys per thread
-    constexpr int CPL = NW;                          // candidates per lane in the second stage (NW*32/32)
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    {
-        uint64_t keys[KPT];
-#pragma unroll
-        for (int q = 0; q < KPT; ++q) {
-            const int e = threadIdx.x + 32 * NW * q;
-            keys[q] = e < E ? sel_key(__ldcg(logits + e), e) : 0ull;
-        }
-        warp_take(keys, k, lane, cand + warp * k);
-    }
-    __syncthreads();
-    if (warp == 0) {
-        uint64_t keys[CPL];
-#pragma unroll
-        for (int q = 0; q < CPL; ++q) {
-            const int i = lane + 32 * q;
-            keys[q] = i < NW * k ? cand[i] : 0ull;
-        }
-        warp_take(keys, k, lane, sel);
-    }
-    __syncthreads();
-}
-
 // Top-k (k <= 32) of E <= 32 * NW * KPT logits by one block of NW warps in
 // two short stages: each warp takes the k best of its keys (KPT per lane),
 // then warp 0 merges the NW sorted candidate lists as a tournament (lane l

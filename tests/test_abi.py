@@ -193,3 +193,11 @@ def test_devcache_rejects_bad_descriptors_on_the_host():
         assert h.value is None
     assert L.devcache_stage(None, None, 0, 0, None, None, None) == M.MOE_EINVAL
     assert L.devcache_join(None, None) == M.MOE_EINVAL
+
+
+@pytest.mark.parametrize("lang", ["c", "c++"])
+def test_header_compiles_as_c_and_cpp(lang):
+    """include/moe.h is a plain C header (extern "C" in C++)."""
+    r = subprocess.run(["gcc" if lang == "c" else "g++", "-fsyntax-only", "-Wall", "-Werror", "-x", lang,
+                        str(M.HEADER)], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr

@@ -365,7 +365,7 @@ int oracle_moe_layer(int bits, int T, int H, int I, int E, int k,
     for (size_t i = 0; i < TH; ++i)
         xd[i] = load_value(x, x_dtype, i);
 
-    double *yp = y_perm ? y_perm : (double *)malloc(sizeof(double) * (TK * H ? TK * H : 1));
+    double *yp = y_perm ? y_perm : (double *)malloc(sizeof(double) * (TK * H > 0 ? TK * H : 1));
     /* row r belongs to the expert e with offsets[e] <= r < offsets[e+1] */
     int32_t *row_expert = (int32_t *)malloc(sizeof(int32_t) * (TK ? TK : 1));
     for (int e = 0; e < E; ++e)

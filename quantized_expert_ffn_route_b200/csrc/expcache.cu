@@ -408,7 +408,7 @@ int expcache_prefetch(moe_expcache *c, const int32_t *ids_host, int n, moe_strea
         c->expert_in[slot] = e;
         c->order.emplace(c->cnt[e], c->last[e], e);
         c->inflight[e] = 1;
-        copies[nc++] = PendingCopy{e, slot};
+        copies[nc++] = PendingCopy{e, slot, nullptr};
         if (slot_out) slot_out[i] = slot;
         if (victim_out) victim_out[i] = victim;
     }

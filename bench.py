@@ -536,6 +536,19 @@ def bench_layer(args, world, rank, pk):
                 else ("fp32 (CUDA-core FMA on 2-bit codes)" if kind == "verify" else "fp16 tensor cores, fp32 accum"))
 
 
+def require_host_memory(what, need, spare=16 << 30):
+    """Stops with a message (not a failed allocation) when the host cannot
+    page-lock `need` bytes and keep `spare` free."""
+    try:
+        import psutil
+        avail = psutil.virtual_memory().available
+    except Exception:
+        return
+    if avail < need + spare:
+        raise SystemExit(f"{what}: {need / 2**30:.1f} GiB of page-locked host memory needed, "
+                         f"{avail / 2**30:.1f} GiB available")
+
+
 def host_link_gbs(nbytes=1 << 30):
     """Pinned host -> device copy bandwidth (best of 3)."""
     import torch
@@ -566,14 +579,7 @@ def bench_paging(args, world, rank, pk):
     link = host_link_gbs()
     # page-locked pool of all experts (512 distinct blobs repeated: only bytes moved matter here)
     need = E * stride
-    try:
-        import psutil
-        avail = psutil.virtual_memory().available
-    except Exception:
-        avail = None
-    if avail is not None and avail < need + (16 << 30):
-        raise SystemExit(f"paging: {need / 2**30:.1f} GiB of page-locked host memory needed, "
-                         f"{avail / 2**30:.1f} GiB available")
+    require_host_memory("paging", need)
     pool = torch.empty(need, dtype=torch.uint8, pin_memory=True)
     pv = pool.view(E, stride)
     bt = torch.from_numpy(base.blobs)
@@ -917,6 +923,7 @@ def bench_paging48(args, world, rank, pk):
     nb = M.moe_expert_blob_bytes(2, H, I)
     stride = (nb + 255) // 256 * 256
     link = host_link_gbs()
+    require_host_memory("paging48", E * stride)
     pool = torch.empty(E * stride, dtype=torch.uint8, pin_memory=True)
     pv = pool.view(E, stride)
     bt = torch.from_numpy(base.blobs)

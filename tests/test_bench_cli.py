@@ -6,6 +6,8 @@ import subprocess
 import sys
 from pathlib import Path
 
+import pytest
+
 ROOT = Path(__file__).resolve().parents[1]
 sys.path.insert(0, str(ROOT))
 
@@ -147,3 +149,11 @@ def test_ffn_mode_override():
         args = argparse.Namespace(layers=0, unfused=False, ffn_mode=name)
         assert bench.workload_shape("verify", args)[1] == want
     assert bench.workload_shape("prefill", argparse.Namespace(layers=0, unfused=False, ffn_mode="auto"))[1] == 2
+
+
+def test_host_memory_guard_stops_with_a_message():
+    import bench
+    bench.require_host_memory("tiny", 1 << 20, spare=0)          # a megabyte is always there
+    with pytest.raises(SystemExit) as ei:
+        bench.require_host_memory("huge", 1 << 60)
+    assert "huge" in str(ei.value) and "page-locked" in str(ei.value)
